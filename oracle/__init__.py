@@ -1,0 +1,218 @@
+"""CPU oracle for SRHT + per-group int4 KV quantisation and decode attention.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import this package. The
+product library (``compressed_domain_attention_b200``) never imports, loads or
+calls it, and the two share no code: the oracle is a plain single-threaded C++
+file (``tq_oracle.cpp``) reached through ctypes, with numpy arrays in and out.
+
+What each function computes, and the page passage it follows, is documented in
+``tq_oracle.cpp``. Parity pins live in ``tests/test_oracle_pins.py``; the sign
+vector's generator convention is the one part with no pin ("parity unpinned":
+any seeded +-1 diagonal is equally correct).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import LIB, build_oracle
+
+STATUS_NONFINITE = 1
+STATUS_CAPACITY = 2
+
+_lib = None
+
+
+def _signatures():
+    P = ctypes.c_void_p
+    i32, i64, u64, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+    return {
+        "oracle_status_nonfinite": ([], i32),
+        "oracle_status_capacity": ([], i32),
+        "oracle_splitmix64": ([u64, ctypes.c_int, P], None),
+        "oracle_sign_vector": ([u64, ctypes.c_int, P], None),
+        "oracle_norm_const": ([ctypes.c_int], f32),
+        "oracle_f32_to_f16": ([P, i64, P], None),
+        "oracle_f16_to_f32": ([P, i64, P], None),
+        "oracle_fwht": ([P, ctypes.c_int, i64], None),
+        "oracle_srht_forward": ([P, P, ctypes.c_int, i64, P], None),
+        "oracle_srht_inverse": ([P, P, ctypes.c_int, i64, P], None),
+        "oracle_quantize_rotated": ([P, ctypes.c_int, i64, P, P], i32),
+        "oracle_pack": ([P, ctypes.c_int, i64, P], None),
+        "oracle_unpack": ([P, ctypes.c_int, i64, P], None),
+        "oracle_encode": ([P, P, ctypes.c_int, i64, P, P], i32),
+        "oracle_quantize_append": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P, P, P, P], i32),
+        "oracle_decode_attention": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, P, f32, P, P], i32),
+        "oracle_dequantize": ([ctypes.c_int] * 4 + [P, P, P, P, ctypes.c_int, P], i32),
+    }
+
+
+def bind(lib):
+    """Attach argument/result types to a loaded oracle library (the built one, or a test's variant)."""
+    for name, (args, res) in _signatures().items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    assert lib.oracle_status_nonfinite() == STATUS_NONFINITE
+    assert lib.oracle_status_capacity() == STATUS_CAPACITY
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            build_oracle()
+        _lib = bind(ctypes.CDLL(LIB))
+    return _lib
+
+
+def _c(a, dtype):
+    """Contiguous array of the exact dtype (copies only if needed)."""
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def splitmix64(seed: int, n: int) -> np.ndarray:
+    out = np.empty(n, np.uint64)
+    _load().oracle_splitmix64(ctypes.c_uint64(seed), n, _p(out))
+    return out
+
+
+def sign_vector(seed: int, D: int) -> np.ndarray:
+    out = np.empty(D, np.float32)
+    _load().oracle_sign_vector(ctypes.c_uint64(seed), D, _p(out))
+    return out
+
+
+def norm_const(D: int) -> np.float32:
+    return np.float32(_load().oracle_norm_const(D))
+
+
+def f32_to_f16_bits(x) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _load().oracle_f32_to_f16(_p(x), x.size, _p(out))
+    return out
+
+
+def f16_bits_to_f32(h) -> np.ndarray:
+    h = _c(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().oracle_f16_to_f32(_p(h), h.size, _p(out))
+    return out
+
+
+def fwht(x) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform along the last axis (binary32)."""
+    u = _c(x, np.float32).copy()
+    D = u.shape[-1]
+    _load().oracle_fwht(_p(u), D, u.size // D)
+    return u
+
+
+def srht_forward(x, signs) -> np.ndarray:
+    x = _c(x, np.float32)
+    s = _c(signs, np.float32)
+    D = x.shape[-1]
+    y = np.empty_like(x)
+    _load().oracle_srht_forward(_p(x), _p(s), D, x.size // D, _p(y))
+    return y
+
+
+def srht_inverse(y, signs) -> np.ndarray:
+    y = _c(y, np.float32)
+    s = _c(signs, np.float32)
+    D = y.shape[-1]
+    x = np.empty_like(y)
+    _load().oracle_srht_inverse(_p(y), _p(s), D, y.size // D, _p(x))
+    return x
+
+
+def quantize_rotated(y):
+    """Per-group abs-max int4 of rotated vectors -> (codes int8 [...,D], scale bits uint16 [...,D/32], status)."""
+    y = _c(y, np.float32)
+    D = y.shape[-1]
+    codes = np.empty(y.shape, np.int8)
+    scales = np.empty(y.shape[:-1] + (D // 32,), np.uint16)
+    st = _load().oracle_quantize_rotated(_p(y), D, y.size // D, _p(codes), _p(scales))
+    return codes, scales, int(st)
+
+
+def pack(codes) -> np.ndarray:
+    codes = _c(codes, np.int8)
+    D = codes.shape[-1]
+    out = np.empty(codes.shape[:-1] + (D // 2,), np.uint8)
+    _load().oracle_pack(_p(codes), D, codes.size // D, _p(out))
+    return out
+
+
+def unpack(packed, D: int) -> np.ndarray:
+    packed = _c(packed, np.uint8)
+    out = np.empty(packed.shape[:-1] + (D,), np.int8)
+    _load().oracle_unpack(_p(packed), D, packed.size // (D // 2), _p(out))
+    return out
+
+
+def encode(x, signs):
+    """SRHT + quantise + pack raw vectors -> (packed uint8 [...,D/2], scale bits [...,D/32], status)."""
+    x = _c(x, np.float32)
+    s = _c(signs, np.float32)
+    D = x.shape[-1]
+    packed = np.empty(x.shape[:-1] + (D // 2,), np.uint8)
+    scales = np.empty(x.shape[:-1] + (D // 32,), np.uint16)
+    st = _load().oracle_encode(_p(x), _p(s), D, x.size // D, _p(packed), _p(scales))
+    return packed, scales, int(st)
+
+
+def new_cache(batch, max_seq, n_kv, D):
+    """Zeroed host cache arrays (codes [B][S][Hkv][D/2] uint8, scales [B][S][Hkv][D/32] uint16)."""
+    codes = np.zeros((batch, max_seq, n_kv, D // 2), np.uint8)
+    scales = np.zeros((batch, max_seq, n_kv, D // 32), np.uint16)
+    return codes, scales
+
+
+def quantize_append(signs, k, v, start_pos, k_codes, k_scales, v_codes, v_scales) -> int:
+    """Append k, v [B][n_new][Hkv][D] at start_pos[b] into the given caches (in place). Returns status bits."""
+    k = _c(k, np.float32)
+    v = _c(v, np.float32)
+    B, n_new, n_kv, D = k.shape
+    max_seq = k_codes.shape[1]
+    for a, dt in ((k_codes, np.uint8), (v_codes, np.uint8), (k_scales, np.uint16), (v_scales, np.uint16)):
+        assert a.dtype == dt and a.flags.c_contiguous
+    sp = _c(start_pos, np.int32)
+    s = _c(signs, np.float32)
+    return int(_load().oracle_quantize_append(B, max_seq, n_kv, D, _p(s), _p(k), _p(v), n_new, _p(sp),
+                                              _p(k_codes), _p(k_scales), _p(v_codes), _p(v_scales)))
+
+
+def decode_attention(signs, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, which=None):
+    """Decode attention on the packed cache. q [B][Hq][D] -> (out [B][Hq][D] float32, status)."""
+    q = _c(q, np.float32)
+    B, n_q, D = q.shape
+    max_seq, n_kv = k_codes.shape[1], k_codes.shape[2]
+    sl = _c(seq_lens, np.int32)
+    s = _c(signs, np.float32)
+    out = np.zeros((B, n_q, D), np.float32)
+    w = None if which is None else _c(which, np.uint8)
+    st = _load().oracle_decode_attention(
+        B, max_seq, n_kv, n_q, D, _p(s), _p(q), _p(sl),
+        _p(_c(k_codes, np.uint8)), _p(_c(k_scales, np.uint16)),
+        _p(_c(v_codes, np.uint8)), _p(_c(v_scales, np.uint16)),
+        ctypes.c_float(sm_scale), None if w is None else _p(w), _p(out))
+    return out, int(st)
+
+
+def dequantize(signs, codes, scales, seq_lens, original_domain: bool):
+    """Dequantise a cache -> float32 [B][S][Hkv][D] (rows past seq_lens[b] are 0)."""
+    B, max_seq, n_kv, half = codes.shape
+    D = 2 * half
+    out = np.empty((B, max_seq, n_kv, D), np.float32)
+    st = _load().oracle_dequantize(B, max_seq, n_kv, D, _p(_c(signs, np.float32)),
+                                   _p(_c(codes, np.uint8)), _p(_c(scales, np.uint16)),
+                                   _p(_c(seq_lens, np.int32)), int(bool(original_domain)), _p(out))
+    return out, int(st)

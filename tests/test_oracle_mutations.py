@@ -1,0 +1,90 @@
+"""Planted mistakes in the oracle must fail at least one pin.
+
+Each case copies ``oracle/tq_oracle.cpp`` to a temporary directory, plants one
+plausible mistake (a wrong sign, a dropped term, a wrong index, a transposed
+operand), compiles it, and runs the fast pins from ``test_oracle_pins`` against
+the mutated library. The committed oracle is never modified.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.build import CXXFLAGS, SRC
+from tests import test_oracle_pins as pins
+
+MUTATIONS = {
+    "fwht_difference_sign": ("u[i + h] = a - b;", "u[i + h] = b - a;"),
+    "norm_const_1_over_D": ("return (float)(1.0 / std::sqrt((double)D));", "return (float)(1.0 / (double)D);"),
+    "scale_divisor_8": ("const float sigma32 = a / 7.0f;", "const float sigma32 = a / 8.0f;"),
+    "truncate_not_round": ("float c = std::nearbyint(r);", "float c = std::trunc(r);"),
+    "nibbles_swapped": ("bytes[j] = (uint8_t)(lo | (hi << 4));", "bytes[j] = (uint8_t)(hi | (lo << 4));"),
+    "forward_sign_dropped": ("for (int i = 0; i < D; ++i) u[i] = s[i] * x[i];", "for (int i = 0; i < D; ++i) u[i] = x[i];"),
+    "inverse_sign_dropped": ("for (int i = 0; i < D; ++i) x[i] = s[i] * (u[i] * c);",
+                             "for (int i = 0; i < D; ++i) x[i] = u[i] * c;"),
+    "gqa_map_modulo": ("const int kv = hq / G;", "const int kv = hq % n_kv;"),
+    "softmax_scale_dropped": ("z[t] = (double)sm_scale * dot;", "z[t] = dot;"),
+    "softmax_not_normalised": ("const double w = z[t] / l;", "const double w = z[t];"),
+    "k_used_for_v": ("dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());",
+                     "dequantize_rotated(k_codes + row * cb, k_scales + row * sb, D, yv.data());"),
+    "f16_ties_away": ("if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h += 1u;", "if (rem >= 0x1000u) h += 1u;"),
+    "f16_exponent_bias": ("uint32_t h = ((uint32_t)(e + 15) << 10) | (frac >> 13);",
+                          "uint32_t h = ((uint32_t)(e + 14) << 10) | (frac >> 13);"),
+}
+
+
+def quick_f16_pin(orc):
+    """A fast sample of the exhaustive binary16 pin, with forced round-to-even ties."""
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 1 << 32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    bits[: 1 << 12] = (bits[: 1 << 12] & ~np.uint32(0x1FFF)) | np.uint32(0x1000)  # exact ties
+    x = bits.view(np.float32)
+    got = orc.f32_to_f16_bits(x)
+    ref = torch.from_numpy(x).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    keep = ~np.isnan(x)
+    assert np.array_equal(got[keep], ref[keep])
+
+
+def fast_pins(orc):
+    yield lambda: pins.test_fwht_equals_sylvester_matrix(orc, 128)
+    yield lambda: pins.test_srht_orthonormal_inverse_parseval(orc, 128)
+    yield lambda: pins.test_closed_form_unit_vector(orc, 64)
+    yield lambda: pins.test_closed_form_hadamard_column(orc, 128)
+    yield lambda: pins.test_quantiser_against_brute_force(orc, 128)
+    yield lambda: pins.test_pack_unpack_identity(orc)
+    yield lambda: pins.test_attention_equals_fp64_original_domain(orc, 128, 8, 2, 33)
+    yield lambda: pins.test_attention_special_cases(orc)
+    yield lambda: pins.test_f16_to_f32_exhaustive(orc)
+    yield lambda: quick_f16_pin(orc)
+
+
+def failing_pins(orc):
+    failed = 0
+    for check in fast_pins(orc):
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_fast_pins_pass_on_committed_oracle(orc):
+    assert failing_pins(orc) == 0
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
+    before, after = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "tq_oracle_mut.cpp"
+    mutated.write_text(src.replace(before, after))
+    lib_path = tmp_path / f"libtq_oracle_{name}.so"
+    subprocess.run(["g++", *CXXFLAGS, "-o", str(lib_path), str(mutated)], check=True)
+    lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert failing_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"

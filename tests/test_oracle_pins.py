@@ -1,0 +1,428 @@
+"""Pins for the CPU oracle, independent of the oracle's own code.
+
+Each test checks the oracle against something other than itself: a library
+routine (scipy's Sylvester Hadamard matrix, torch's IEEE fp32->fp16 conversion),
+a closed form, an exact invariant, brute force on tiny inputs, or an
+original-domain fp64 attention computed here with numpy.
+
+Page references (by title and section):
+ * "Open-TQ-Metal: Fused Compressed-Domain Attention for Long-Context LLM
+   Inference on Apple Silicon", abstract (cards page): sign-randomised
+   transform + per-group abs-max + int4 nibble pack.
+ * the same paper's arXiv abstract: attention directly on the compressed
+   representation; 1/sqrt(d) attention scale.
+ * mlxcel user guide "TurboQuant KV cache compression", §"What TurboQuant
+   changes": Walsh-Hadamard rotation before low-bit storage.
+ * "TurboQuant on AMD GPUs", §4: Walsh-Hadamard spreads energy evenly.
+"""
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+DIMS = (32, 64, 128, 256)
+
+
+# ---------------------------------------------------------------- helpers (independent of the oracle)
+
+def hadamard(D):
+    return scipy.linalg.hadamard(D).astype(np.float64)  # Sylvester construction, natural order
+
+
+def np_unpack(packed, D):
+    lo = (packed & 0x0F).astype(np.int16)
+    hi = (packed >> 4).astype(np.int16)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(packed.shape[:-1] + (D,), np.int16)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def np_dequant_rotated(packed, scale_bits, D):
+    codes = np_unpack(packed, D).astype(np.float64)
+    sig = scale_bits.view(np.float16).astype(np.float64)
+    return codes * np.repeat(sig, 32, axis=-1)
+
+
+def np_dequant_original(packed, scale_bits, signs):
+    D = signs.shape[0]
+    y = np_dequant_rotated(packed, scale_bits, D)
+    return (y @ hadamard(D).T) / np.sqrt(D) * signs.astype(np.float64)
+
+
+def heavy_tailed(rng, n, D):
+    x = rng.standard_normal((n, D)) * np.exp(rng.standard_normal(D))
+    x[:, rng.permutation(D)[: D // 32]] *= 10.0
+    return x.astype(np.float32)
+
+
+# ---------------------------------------------------------------- sign vector / generator
+
+def test_splitmix64_published_sequence(orc):
+    # SplitMix64 (Vigna's public-domain reference generator), seed 0: the
+    # widely reproduced first outputs.
+    got = [int(x) for x in orc.splitmix64(0, 4)]
+    assert got == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F, 0xF88BB8A8724C81EC]
+
+
+def test_sign_vector_pm1_and_seeded(orc):
+    for D in DIMS:
+        s = orc.sign_vector(0, D)
+        assert set(np.unique(s)) <= {-1.0, 1.0}
+        assert np.array_equal(s, orc.sign_vector(0, D))
+        r = orc.splitmix64(0, D)
+        assert np.array_equal(s < 0, (r >> np.uint64(63)) == 1)
+    assert not np.array_equal(orc.sign_vector(0, 128), orc.sign_vector(1, 128))
+    # prefix property: the first 64 signs of the D=128 vector are the D=64 vector
+    assert np.array_equal(orc.sign_vector(7, 128)[:64], orc.sign_vector(7, 64))
+
+
+def test_norm_const(orc):
+    assert orc.norm_const(64) == np.float32(0.125)
+    assert orc.norm_const(256) == np.float32(0.0625)
+    for D in (32, 128):
+        c = float(orc.norm_const(D))
+        # the binary32 nearest to 1/sqrt(D): within half an ulp of the exact value
+        ulp = np.spacing(np.float32(c))
+        assert abs(c - 1.0 / np.sqrt(D)) <= 0.5 * float(ulp)
+
+
+# ---------------------------------------------------------------- Walsh-Hadamard transform
+
+@pytest.mark.parametrize("D", DIMS)
+def test_fwht_equals_sylvester_matrix(orc, D):
+    # FWHT of the identity rows is H (exact: entries are sums of +-1).
+    H = orc.fwht(np.eye(D, dtype=np.float32))
+    assert np.array_equal(H.astype(np.float64), hadamard(D))
+    # H H^T = D I exactly, via the oracle's transform applied to H's rows
+    HH = orc.fwht(H)
+    assert np.array_equal(HH, D * np.eye(D, dtype=np.float32))
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_fwht_matches_fp64_matrix_product(orc, D):
+    rng = np.random.default_rng(D)
+    x = rng.standard_normal((64, D)).astype(np.float32)
+    got = orc.fwht(x).astype(np.float64)
+    ref = x.astype(np.float64) @ hadamard(D).T
+    scale = np.abs(x).sum(axis=1, keepdims=True)
+    assert np.max(np.abs(got - ref) / scale) < 1e-6
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_srht_orthonormal_inverse_parseval(orc, D):
+    s = orc.sign_vector(3, D)
+    R = orc.srht_forward(np.eye(D, dtype=np.float32), s).astype(np.float64)  # row j = R e_j
+    # rows of the forward image of the identity: R^T R = I
+    assert np.max(np.abs(R @ R.T - np.eye(D))) < 1e-6
+    # the map is c_D H diag(s)
+    ref = (hadamard(D) * s.astype(np.float64)[None, :]).T / np.sqrt(D)
+    assert np.max(np.abs(R - ref)) < 1e-7
+    rng = np.random.default_rng(D + 1)
+    x = heavy_tailed(rng, 32, D)
+    y = orc.srht_forward(x, s)
+    xb = orc.srht_inverse(y, s)
+    assert np.max(np.abs(xb - x) / np.abs(x).max(axis=1, keepdims=True)) < 1e-6
+    nx = np.linalg.norm(x.astype(np.float64), axis=1)
+    ny = np.linalg.norm(y.astype(np.float64), axis=1)
+    assert np.max(np.abs(ny / nx - 1)) < 1e-6
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_rotated_dot_products_equal_originals(orc, D):
+    s = orc.sign_vector(0, D)
+    rng = np.random.default_rng(10 + D)
+    x = heavy_tailed(rng, 50, D)
+    z = rng.standard_normal((50, D)).astype(np.float32)
+    rx, rz = orc.srht_forward(x, s).astype(np.float64), orc.srht_forward(z, s).astype(np.float64)
+    d0 = np.sum(x.astype(np.float64) * z, axis=1)
+    d1 = np.sum(rx * rz, axis=1)
+    bound = 1e-5 * np.linalg.norm(x, axis=1) * np.linalg.norm(z, axis=1)
+    assert np.all(np.abs(d1 - d0) <= bound)
+
+
+# ---------------------------------------------------------------- closed forms of the encoder
+
+@pytest.mark.parametrize("D", DIMS)
+def test_closed_form_unit_vector(orc, D):
+    s = orc.sign_vector(5, D)
+    H = hadamard(D)
+    c = np.float32(1.0 / np.sqrt(D))
+    sig16 = (np.float32(c) / np.float32(7.0)).astype(np.float16).view(np.uint16)
+    for j in (0, 1, D // 2 - 1, D - 1):
+        x = np.zeros(D, np.float32)
+        x[j] = 1.0
+        packed, scales, st = orc.encode(x[None], s)
+        assert st == 0
+        codes = np_unpack(packed[0], D)
+        assert np.all(scales[0] == sig16)
+        assert np.array_equal(codes, (7 * s[j] * H[:, j]).astype(np.int16))
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_closed_form_hadamard_column(orc, D):
+    # x = s o H[:, j]  ->  y = fl(c_D * D) e_j exactly; one nonzero code (+7)
+    s = orc.sign_vector(9, D)
+    H = hadamard(D)
+    for j in (0, 3, D - 1):
+        x = (s.astype(np.float64) * H[:, j]).astype(np.float32)
+        y = orc.srht_forward(x[None], s)[0]
+        e = np.zeros(D, np.float32)
+        e[j] = np.float32(D) * np.float32(1.0 / np.sqrt(D))
+        assert np.array_equal(y, e)
+        packed, scales, st = orc.encode(x[None], s)
+        codes = np_unpack(packed[0], D)
+        expect = np.zeros(D, np.int16)
+        expect[j] = 7
+        assert np.array_equal(codes, expect)
+        g = j // 32
+        sig = (e[j] / np.float32(7.0)).astype(np.float16).view(np.uint16)
+        assert scales[0, g] == sig
+        assert np.all(np.delete(scales[0], g) == 0)
+
+
+# ---------------------------------------------------------------- quantiser
+
+def brute_force_codes(y, sig):
+    """argmin over c in [-7, 7] of |fl(y/sigma) - c|, ties to the even c."""
+    r = (y / sig).astype(np.float32).astype(np.float64)
+    cands = np.arange(-7, 8, dtype=np.float64)
+    dist = np.abs(r[..., None] - cands)
+    best = dist.min(axis=-1, keepdims=True)
+    tie_even = np.where((dist == best) & (cands % 2 == 0), 0, 1) + np.where(dist == best, 0, 2)
+    return cands[np.argmin(tie_even, axis=-1)].astype(np.int8)
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_quantiser_against_brute_force(orc, D):
+    rng = np.random.default_rng(100 + D)
+    y = heavy_tailed(rng, 400, D)
+    # exact ties: absmax 7 gives sigma = 1, so y/sigma = k + 0.5 exactly
+    y[0, :32] = np.concatenate([np.arange(-7.0, 7.5, 0.5), [0.25, -0.75, 6.75]]).astype(np.float32)
+    codes, scales, st = orc.quantize_rotated(y)
+    assert st == 0
+    g = y.reshape(400, D // 32, 32)
+    a = np.abs(g).max(axis=-1)
+    sig16 = (a.astype(np.float32) / np.float32(7.0)).astype(np.float16)
+    assert np.array_equal(scales, sig16.view(np.uint16))
+    sig = sig16.astype(np.float32)[..., None]
+    bf = np.where(sig > 0, brute_force_codes(g, np.where(sig > 0, sig, 1)), 0)
+    assert np.array_equal(codes.reshape(bf.shape), bf)
+    err = np.abs(g.astype(np.float64) - codes.reshape(g.shape) * sig.astype(np.float64))
+    assert np.all(err <= sig.astype(np.float64) * (0.5 + 1e-6))
+    assert codes.min() >= -7 and codes.max() <= 7
+
+
+def test_quantiser_symmetries(orc):
+    rng = np.random.default_rng(7)
+    y = heavy_tailed(rng, 200, 128)
+    c0, s0, _ = orc.quantize_rotated(y)
+    c1, s1, _ = orc.quantize_rotated(-y)
+    assert np.array_equal(c1, -c0) and np.array_equal(s1, s0)
+    for k in (-3, 1, 4):
+        c2, s2, _ = orc.quantize_rotated(np.ldexp(y, k))
+        assert np.array_equal(c2, c0)
+        assert np.array_equal(s2.view(np.float16).astype(np.float64),
+                              np.ldexp(s0.view(np.float16).astype(np.float64), k))
+
+
+def test_quantiser_zero_and_nonfinite_groups(orc):
+    y = np.zeros((3, 64), np.float32)
+    y[1, 3] = np.inf
+    y[2, 40] = np.float32(1e6)  # absmax/7 overflows binary16
+    codes, scales, st = orc.quantize_rotated(y)
+    assert st & orc.STATUS_NONFINITE
+    assert np.all(codes[0] == 0) and np.all(scales[0] == 0)
+    assert scales[1, 0] == 0x7C00 and np.all(codes[1, :32] == 0) and scales[1, 1] == 0
+    assert scales[2, 1] == 0x7C00 and np.all(codes[2, 32:] == 0)
+    _, _, st0 = orc.quantize_rotated(np.ones((1, 64), np.float32))
+    assert st0 == 0
+
+
+# ---------------------------------------------------------------- binary16 conversion
+
+@pytest.mark.slow
+def test_f32_to_f16_exhaustive_against_torch(orc):
+    # torch's float32->float16 cast is IEEE round-to-nearest-even (F16C on x86).
+    n = 1 << 26
+    for c in range((1 << 32) // n):
+        bits = np.arange(c * n, (c + 1) * n, dtype=np.uint64).astype(np.uint32)
+        x = bits.view(np.float32)
+        got = orc.f32_to_f16_bits(x)
+        ref = torch.from_numpy(x).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+        nan = np.isnan(x)
+        assert np.array_equal(got[~nan], ref[~nan]), hex(c * n)
+        assert np.all((got[nan] & 0x7C00) == 0x7C00) and np.all((got[nan] & 0x3FF) != 0)
+
+
+def test_f16_to_f32_exhaustive(orc):
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = orc.f16_bits_to_f32(h)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(got.view(np.uint32)[~nan], ref.view(np.uint32)[~nan])
+    assert np.all(np.isnan(got[nan]))
+
+
+# ---------------------------------------------------------------- nibble packing
+
+def test_pack_unpack_identity(orc):
+    vals = np.arange(-7, 8, dtype=np.int8)
+    pairs = np.array(np.meshgrid(vals, vals, indexing="ij")).reshape(2, -1).T  # 225 pairs
+    flat = np.concatenate([pairs.reshape(-1), np.zeros(32 - pairs.size % 32, np.int8)]).reshape(-1, 32)
+    packed = orc.pack(flat)
+    assert np.array_equal(orc.unpack(packed, 32), flat)
+    assert np.array_equal(np_unpack(packed, 32), flat)
+    # every byte decodes, and re-encodes to itself (including the unused -8 nibble)
+    allb = np.arange(256, dtype=np.uint16).astype(np.uint8).reshape(-1, 16)
+    assert np.array_equal(orc.pack(orc.unpack(allb, 32)), allb)
+    # low nibble = even element, two's complement
+    one = np.zeros((1, 32), np.int8)
+    one[0, 0], one[0, 1] = 3, -2
+    assert orc.pack(one)[0, 0] == (3 | (0xE << 4))
+
+
+# ---------------------------------------------------------------- rotation helps (motivation check)
+
+def test_rotation_lowers_int4_roundtrip_error(orc):
+    # [AMD] §4 / [MLX]: the Walsh-Hadamard rotation spreads outlier-channel
+    # energy, so per-group abs-max wastes fewer levels.
+    rng = np.random.default_rng(11)
+    x = heavy_tailed(rng, 512, 128)
+    s = orc.sign_vector(0, 128)
+    packed, scales, _ = orc.encode(x, s)
+    xr = np_dequant_original(packed, scales, s)
+    c, sc, _ = orc.quantize_rotated(x)
+    xn = c.astype(np.float64) * np.repeat(sc.view(np.float16).astype(np.float64), 32, axis=-1)
+    mse_rot = np.mean((xr - x) ** 2)
+    mse_plain = np.mean((xn - x) ** 2)
+    assert mse_rot < 0.7 * mse_plain
+
+
+# ---------------------------------------------------------------- attention
+
+def make_cache(orc, rng, B, T, Hkv, D, s, max_seq=None, k=None, v=None):
+    max_seq = max_seq or T
+    if k is None:
+        k = np.stack([heavy_tailed(rng, T * Hkv, D).reshape(T, Hkv, D) for _ in range(B)])
+        v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    kc, ks = orc.new_cache(B, max_seq, Hkv, D)
+    vc, vs = orc.new_cache(B, max_seq, Hkv, D)
+    st = orc.quantize_append(s, k, v, np.zeros(B, np.int32), kc, ks, vc, vs)
+    assert st == 0
+    return kc, ks, vc, vs
+
+
+def brute_force_attention(q, lens, kc, ks, vc, vs, s, sm_scale):
+    """softmax(q K^T * scale) V in fp64 in the ORIGINAL domain on dequantised K, V."""
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        L = lens[b]
+        if L == 0:
+            continue
+        for hq in range(Hq):
+            kv = hq // G
+            K = np_dequant_original(kc[b, :L, kv], ks[b, :L, kv], s)
+            V = np_dequant_original(vc[b, :L, kv], vs[b, :L, kv], s)
+            z = K @ q[b, hq].astype(np.float64) * sm_scale
+            w = np.exp(z - z.max())
+            out[b, hq] = (w / w.sum()) @ V
+    return out
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,T", [(32, 4, 1, 17), (128, 4, 1, 64), (128, 8, 2, 33), (64, 2, 2, 5),
+                                        (256, 4, 1, 40)])
+def test_attention_equals_fp64_original_domain(orc, D, Hq, Hkv, T):
+    rng = np.random.default_rng(D * 1000 + T)
+    s = orc.sign_vector(0, D)
+    B = 2
+    kc, ks, vc, vs = make_cache(orc, rng, B, T, Hkv, D, s)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    lens = np.array([T, max(1, T // 2)], np.int32)
+    scale = 1.0 / np.sqrt(D)
+    got, st = orc.decode_attention(s, q, lens, kc, ks, vc, vs, scale)
+    assert st == 0
+    ref = brute_force_attention(q, lens, kc, ks, vc, vs, s, scale)
+    assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_attention_special_cases(orc):
+    rng = np.random.default_rng(42)
+    D, Hkv, Hq, T = 128, 2, 4, 24
+    s = orc.sign_vector(0, D)
+    kc, ks, vc, vs = make_cache(orc, rng, 1, T, Hkv, D, s)
+    q = rng.standard_normal((1, Hq, D)).astype(np.float32)
+    # T = 1: output = the one dequantised V row (original domain)
+    out1, _ = orc.decode_attention(s, q, np.array([1], np.int32), kc, ks, vc, vs, 0.1)
+    for hq in range(Hq):
+        ref = np_dequant_original(vc[0, 0, hq // 2], vs[0, 0, hq // 2], s)
+        assert np.max(np.abs(out1[0, hq] - ref)) < 1e-6 * max(1, np.abs(ref).max())
+    # q = 0: uniform weights -> mean of dequantised V
+    out0, _ = orc.decode_attention(s, np.zeros_like(q), np.array([T], np.int32), kc, ks, vc, vs, 0.1)
+    for hq in range(Hq):
+        ref = np_dequant_original(vc[0, :T, hq // 2], vs[0, :T, hq // 2], s).mean(axis=0)
+        assert np.max(np.abs(out0[0, hq] - ref)) < 1e-6
+    # all K rows identical -> mean of V for any q
+    kc2, ks2 = kc.copy(), ks.copy()
+    kc2[0, :] = kc[0, 0]
+    ks2[0, :] = ks[0, 0]
+    outk, _ = orc.decode_attention(s, q, np.array([T], np.int32), kc2, ks2, vc, vs, 0.3)
+    assert np.max(np.abs(outk - out0)) < 1e-6
+    # empty sequence -> zeros
+    oute, st = orc.decode_attention(s, q, np.array([0], np.int32), kc, ks, vc, vs, 0.1)
+    assert st == 0 and np.all(oute == 0)
+    # length past max_seq -> capacity status, zeros
+    outc, st = orc.decode_attention(s, q, np.array([T + 1], np.int32), kc, ks, vc, vs, 0.1)
+    assert st & orc.STATUS_CAPACITY and np.all(outc == 0)
+
+
+def test_gqa_equals_replicated_mha(orc):
+    rng = np.random.default_rng(5)
+    D, Hkv, G, T = 64, 2, 3, 19
+    s = orc.sign_vector(0, D)
+    k = np.stack([heavy_tailed(rng, T * Hkv, D).reshape(T, Hkv, D)])
+    v = rng.standard_normal((1, T, Hkv, D)).astype(np.float32)
+    kc, ks, vc, vs = make_cache(orc, rng, 1, T, Hkv, D, s, k=k, v=v)
+    kr = np.repeat(k, G, axis=2)
+    vr = np.repeat(v, G, axis=2)
+    kc2, ks2, vc2, vs2 = make_cache(orc, rng, 1, T, Hkv * G, D, s, k=kr, v=vr)
+    q = rng.standard_normal((1, Hkv * G, D)).astype(np.float32)
+    lens = np.array([T], np.int32)
+    a, _ = orc.decode_attention(s, q, lens, kc, ks, vc, vs, 0.125)
+    b, _ = orc.decode_attention(s, q, lens, kc2, ks2, vc2, vs2, 0.125)
+    assert np.array_equal(a, b)
+
+
+def test_append_positions_and_capacity(orc):
+    rng = np.random.default_rng(9)
+    D, Hkv, S = 64, 2, 8
+    s = orc.sign_vector(0, D)
+    k = rng.standard_normal((2, 3, Hkv, D)).astype(np.float32)
+    v = rng.standard_normal((2, 3, Hkv, D)).astype(np.float32)
+    kc, ks = orc.new_cache(2, S, Hkv, D)
+    vc, vs = orc.new_cache(2, S, Hkv, D)
+    st = orc.quantize_append(s, k, v, np.array([2, 6], np.int32), kc, ks, vc, vs)
+    assert st & orc.STATUS_CAPACITY  # 6 + 3 > 8: sequence 1 skipped
+    p, sc, _ = orc.encode(k[0], s)
+    assert np.array_equal(kc[0, 2:5], p) and np.array_equal(ks[0, 2:5], sc)
+    assert np.all(kc[0, :2] == 0) and np.all(kc[0, 5:] == 0) and np.all(kc[1] == 0)
+    pv, scv, _ = orc.encode(v[0], s)
+    assert np.array_equal(vc[0, 2:5], pv) and np.array_equal(vs[0, 2:5], scv)
+
+
+def test_dequantize_matches_independent(orc):
+    rng = np.random.default_rng(12)
+    D, Hkv, T = 128, 2, 10
+    s = orc.sign_vector(0, D)
+    kc, ks, _, _ = make_cache(orc, rng, 1, T, Hkv, D, s, max_seq=12)
+    lens = np.array([T], np.int32)
+    yr, _ = orc.dequantize(s, kc, ks, lens, False)
+    xo, _ = orc.dequantize(s, kc, ks, lens, True)
+    assert np.array_equal(yr[0, :T].astype(np.float64), np_dequant_rotated(kc[0, :T], ks[0, :T], D))
+    assert np.max(np.abs(xo[0, :T] - np_dequant_original(kc[0, :T], ks[0, :T], s))) < 1e-5
+    assert np.all(yr[0, T:] == 0) and np.all(xo[0, T:] == 0)
