@@ -1,0 +1,469 @@
+"""Benchmark: int4-KV decode attention on B200 (effective HBM GB/s and tokens/s).
+
+One step is the whole hot path on one batch: quantise-append one new K/V token
+per sequence (SRHT + per-group abs-max int4 + nibble pack) and one decode query
+per sequence over its packed cache (rotated query, split-K online softmax on
+tensor cores, merge + inverse SRHT). The default workload is the 32-sequence
+ragged serving batch (contexts U{1024..32768}, 32 q / 8 kv heads, D = 128,
+bf16 inputs); ``--workload`` picks another recipe from
+``compressed_domain_attention_b200.synthetic``.
+
+Timing: W warm-up steps, then K steps between a barrier + synchronize on both
+sides, CUDA events on the launching stream, max over ranks. The packed cache
+(about 1.2 GB for the default workload) is larger than the 126 MB L2, so no L2
+flush is needed. ``--gpus N`` (under torchrun) runs N independent replicas: the
+path has no exchange step, so there is no collective on the data path.
+
+``--impl reference`` times the CPU oracle (plain single-threaded C++) on a
+bounded sample of the same workload on the host cores.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "int4-KV decode attention effective HBM GB/s (packed K/V codes + fp16 scales per step)"
+UNIT = "GB/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default="ragged_serving",
+                    choices=["ragged_serving", "llama31_70b_long", "llama3_8b_layer", "tiny_single_head"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
+    return ap.parse_args(argv)
+
+
+def get_workload(name):
+    from compressed_domain_attention_b200 import synthetic as syn
+    return {"ragged_serving": syn.ragged_serving, "llama31_70b_long": syn.llama31_70b_long,
+            "llama3_8b_layer": syn.llama3_8b_layer, "tiny_single_head": syn.tiny_single_head}[name]()
+
+
+# ----------------------------------------------------------------------------- algorithmic bytes
+
+def decode_bytes(w, lens):
+    """Packed K + V codes and binary16 scales the decode must read: (D/2 + D/16) * 2 bytes per token.kv-head."""
+    per = 2 * (w.head_dim // 2 + 2 * (w.head_dim // 32))
+    return sum(lens) * w.n_kv_heads * per
+
+
+def append_bytes(w, in_bytes=2):
+    """Quantise-append traffic: raw K/V in + packed codes and scales out, per appended token."""
+    D = w.head_dim
+    per_vec = D * in_bytes + D // 2 + 2 * (D // 32)
+    return 2 * w.batch * w.n_append * w.n_kv_heads * per_vec
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def load_traffic(kernel_key):
+    """ncu DRAM bytes per launch recorded in profiles/ for the current kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "compressed_domain_attention_b200", "csrc", "tq_decode.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    ent = rec.get(kernel_key)
+    if not ent or ent.get("source_sha256_16") != digest:
+        return None
+    return ent.get("dram_bytes_per_full_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        sm = []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mx = None
+        for p in self.samples:
+            try:
+                sm.append(float(p[0]))
+                mx = float(p[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value, device=None):
+    """Max of a float over all ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value, device=None):
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def assemble_line(*, n_gpus, steps, warmup, total_bytes_all_ranks, max_time_s, workload, extra):
+    """The JSON result line (value = whole-job GB/s over all ranks)."""
+    value = total_bytes_all_ranks / max_time_s / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": n_gpus, "steps": steps,
+            "warmup": warmup, "ms_per_step": round(max_time_s / steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes, f16 tensor-core operands, f32 accumulate",
+            "data": "synthetic (seeded; outlier-channel K, no weights or datasets)", "config": workload}
+    line.update(extra)
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(w, target_tokens, longest_first=False):
+    """Sequences for a bounded oracle sample: up to about `target_tokens` KV tokens."""
+    order = sorted(range(w.batch), key=lambda b: w.seq_lens[b], reverse=longest_first)
+    picked, tot = [], 0
+    for b in order:
+        if tot >= target_tokens and picked:
+            break
+        picked.append(b)
+        tot += w.seq_lens[b]
+    return sorted(picked)
+
+
+class OracleStep:
+    """The oracle's version of one step (append one token per sequence, decode) on a sample of sequences.
+
+    The sample's caches are encoded once at construction (untimed); each step
+    re-appends the new token at position len_b and decodes over len_b + 1.
+    """
+
+    def __init__(self, w, tensors, seqs):
+        import numpy as np
+        import oracle
+        from compressed_domain_attention_b200 import synthetic as syn
+        self.oracle, self.np = oracle, np
+        D, H = w.head_dim, w.n_kv_heads
+        self.w, self.seqs = w, seqs
+        self.s = oracle.sign_vector(0, D)
+        n = len(seqs)
+        cap = max(w.seq_lens[b] for b in seqs) + 1
+        self.kc, self.ks = oracle.new_cache(n, cap, H, D)
+        self.vc, self.vs = oracle.new_cache(n, cap, H, D)
+        for i, b in enumerate(seqs):
+            k = tensors.k[b].float().cpu().numpy()[None]
+            v = tensors.v[b].float().cpu().numpy()[None]
+            oracle.quantize_append(self.s, k, v, np.zeros(1, np.int32), self.kc[i:i + 1], self.ks[i:i + 1],
+                                   self.vc[i:i + 1], self.vs[i:i + 1])
+        self.q = np.ascontiguousarray(tensors.q[seqs].float().cpu().numpy())
+        self.kn = np.ascontiguousarray(tensors.k_new[seqs].float().cpu().numpy())
+        self.vn = np.ascontiguousarray(tensors.v_new[seqs].float().cpu().numpy())
+        self.lens = np.array([w.seq_lens[b] for b in seqs], np.int32)
+        sub = syn.Workload(w.name, n, w.n_q_heads, H, D, [w.seq_lens[b] for b in seqs], w.dtype, w.seed, n_append=1)
+        self.nbytes = decode_bytes(sub, [L + 1 for L in sub.seq_lens]) + append_bytes(sub)
+        self.ntok = int(self.lens.sum()) + n
+
+    def run(self):
+        t0 = time.perf_counter()
+        self.oracle.quantize_append(self.s, self.kn, self.vn, self.lens, self.kc, self.ks, self.vc, self.vs)
+        self.oracle.decode_attention(self.s, self.q, self.lens + 1, self.kc, self.ks, self.vc, self.vs, self.w.scale)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(w, tensors, target_tokens):
+    seqs = oracle_sample(w, target_tokens)
+    o = OracleStep(w, tensors, seqs)
+    dt = o.run()
+    return {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
+                      f"({o.ntok} KV tokens x {w.n_q_heads} q heads), single-threaded C++ oracle, {dt:.2f} s",
+            "seconds": round(dt, 3)}
+
+
+# ----------------------------------------------------------------------------- main paths
+
+def run_reference(args):
+    """--impl reference: the CPU oracle on the host cores, bounded sample per step (rank 0 only)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from compressed_domain_attention_b200 import synthetic as syn
+    w = get_workload(args.workload)
+    if w.n_append == 0:
+        w.n_append = 1
+    seqs = oracle_sample(w, 8192)
+    t = syn.generate(w, device="cpu", seq_subset=seqs)
+    o = OracleStep(w, t, seqs)
+    for _ in range(args.warmup):
+        o.run()
+    tot_t = sum(o.run() for _ in range(args.steps))
+    value = o.nbytes * args.steps / tot_t / 1e9
+    sample = (f"each step: append + decode on {len(seqs)} of {w.batch} sequences "
+              f"({o.ntok} KV tokens x {w.n_q_heads} q heads), single-threaded C++ oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode / f64 attention",
+            "data": "synthetic (seeded)", "config": {"workload": w.name, "global_batch": w.batch},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tq(args):
+    import torch
+    from compressed_domain_attention_b200 import synthetic as syn
+    from compressed_domain_attention_b200 import tq
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    w = get_workload(args.workload)
+    if w.n_append == 0:
+        w.n_append = 1
+    cap = max(w.seq_lens) + w.n_append
+    t = syn.generate(w, device="cuda")
+    L = tq.tq_cache_layout(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+    kc, ks, vc, vs = tq.alloc_cache(L, dev)
+    wsp = tq.alloc_workspace(L, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # prefill (untimed): one append per sequence through a batch-1 view of the cache
+    l1 = tq.tq_cache_layout(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    cs, ss = int(L.code_stride_seq), int(L.scale_stride_seq)
+    for b in range(w.batch):
+        n = w.seq_lens[b]
+        tq.tq_quantize_append(l1, t.k[b][None], t.v[b][None], n, zero, kc[b * cs:(b + 1) * cs], ks[b * ss:],
+                              vc[b * cs:(b + 1) * cs], vs[b * ss:], status)
+    torch.cuda.synchronize()
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
+    lens1 = lens + w.n_append
+    q = t.q.contiguous()
+    k_new, v_new = t.k_new.contiguous(), t.v_new.contiguous()
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    n_ev = args.steps
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+
+    def step(i=None):
+        tq.tq_quantize_append(L, k_new, v_new, w.n_append, lens, kc, ks, vc, vs, status, stream)
+        if i is not None:
+            ev_a[i].record(stream)
+            tq.tq_decode_attention(L, q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream,
+                                   after_split_event=ev_s[i])
+            ev_b[i].record(stream)
+        else:
+            tq.tq_decode_attention(L, q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    for e in ev_s:  # torch creates the CUDA event on first record; the library re-records it later
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    clocks = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    clk = clocks.stop() if clocks else None
+    elapsed = start.elapsed_time(stop) / 1e3
+    split_ms = [ev_a[i].elapsed_time(ev_s[i]) for i in range(args.steps)]
+    merge_ms = [ev_s[i].elapsed_time(ev_b[i]) for i in range(args.steps)]
+    st = int(status.item())
+    if st != 0:
+        raise RuntimeError(f"device status {st} during the benchmark")
+
+    # e2e: host buffers in pinned memory, copies inside the timed region
+    h_k = k_new.cpu().pin_memory()
+    h_v = v_new.cpu().pin_memory()
+    h_q = q.cpu().pin_memory()
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    d_k, d_v, d_q = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(q)
+
+    def e2e_step():
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        tq.tq_quantize_append(L, d_k, d_v, w.n_append, lens, kc, ks, vc, vs, status, stream)
+        tq.tq_decode_attention(L, d_q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_s = e0.elapsed_time(e1) / 1e3
+
+    lens_step = [x + w.n_append for x in w.seq_lens]
+    bytes_decode = decode_bytes(w, lens_step)
+    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4)
+    max_t = max_over_ranks(elapsed, dev)
+    max_e2e = max_over_ranks(e2e_s, dev)
+    split_avg = max_over_ranks(statistics.mean(split_ms), dev)
+    merge_avg = max_over_ranks(statistics.mean(merge_ms), dev)
+
+    peak, peak_kind = load_peaks()
+    achieved = bytes_decode / (split_avg / 1e3) / 1e9
+    traffic = load_traffic(f"decode_split_kernel/{w.name}")
+    kv_tokens = sum(lens_step) * w.n_kv_heads
+    extra = {
+        "tokens_per_s": round(ws * w.batch * w.n_append * args.steps / max_t, 1),
+        "kv_tokens_per_s": round(ws * sum(lens_step) * args.steps / max_t, 1),
+        "pct_of_measured_hbm": round(100.0 * bytes_step / max_t * args.steps / 1e9 / peak, 2),
+        "pct_of_8tbs": round(100.0 * bytes_step / max_t * args.steps / 1e9 / 8000.0, 2),
+        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": bytes_decode, "avg_launch_ms": round(split_avg, 4),
+                     "merge_avg_ms": round(merge_avg, 4)},
+        "e2e": {"value": round(ws * bytes_step * args.steps / max_e2e / 1e9, 2), "unit": UNIT,
+                "h2d_bytes_per_step": int(k_new.numel() * k_new.element_size() * 2 + q.numel() * q.element_size()),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+        "gpu_launches": 3 * args.steps,
+    }
+    if clk:
+        extra["clocks"] = clk
+    cfg = {"workload": w.name, "global_batch": w.batch * ws, "kv_tokens_per_seq_step": lens_step if w.batch <= 4
+           else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
+           "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+           "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+           "l2": f"inputs larger than L2 (packed cache {2 * int(L.codes_bytes + L.scales_bytes) / 1e9:.2f} GB "
+                 "per replica > 126 MB), no flush",
+           "algorithmic_bytes_per_step": bytes_step}
+    total_bytes = sum_over_ranks(bytes_step * args.steps, dev)  # every rank takes part
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        extra["cpu_baseline"] = cpu_baseline(w, t, 300000)
+    if rank == 0:
+        line = assemble_line(n_gpus=ws, steps=args.steps, warmup=args.warmup, total_bytes_all_ranks=total_bytes,
+                             max_time_s=max_t, workload=cfg, extra=extra)
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_tq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,306 @@
+// C ABI of libtq_b200: argument validation, layout arithmetic, tensor-map
+// encoding and kernel launches. See include/tq.h for the contract.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tq.h"
+#include "tq_kernels.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return TQ_ERR_CUDA;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SplitMix64 (S. Vigna's public-domain generator), used to draw the fixed +-1
+// diagonal of the rotation: s_i = -1 iff the top bit of the i-th output is set.
+uint64_t splitmix64_step(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ULL;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+// Split-K grid ceiling the default workspace is sized for.
+constexpr int kMaxCtas = 1024;
+constexpr int kMaxBatchDecode = 1024;
+constexpr int kMaxTileTokens = 256;
+
+int device_sm_count(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 64 && cache[dev] > 0) {
+    *out = cache[dev];
+    return TQ_OK;
+  }
+  int n = 0;
+  e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 64) cache[dev] = n;
+  *out = n;
+  return TQ_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view of a codes buffer: (D/2 bytes, batch*max_seq tokens, n_kv heads),
+// box (D/2, tile, n_kv); the shared-memory image is [head][tile][D/2] with the
+// swizzle matching the row pitch.
+int encode_codes_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::TensorMap128* out) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
+  const int rb = L->head_dim / 2;
+  cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq, (cuuint64_t)L->n_kv_heads};
+  cuuint64_t strides[2] = {(cuuint64_t)L->code_stride_tok, (cuuint64_t)rb};
+  cuuint32_t box[3] = {(cuuint32_t)rb, (cuuint32_t)tile, (cuuint32_t)L->n_kv_heads};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                     : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap m;
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = (int)r;
+    return TQ_ERR_CUDA;
+  }
+  static_assert(sizeof(CUtensorMap) == sizeof(tqk::TensorMap128), "tensor map size");
+  std::memcpy(out, &m, sizeof(m));
+  return TQ_OK;
+}
+
+int check_layout(const tq_layout_t* L) {
+  if (L == nullptr) return TQ_ERR_INVALID_ARG;
+  tq_layout_t chk;
+  const int r = tq_cache_layout(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
+                                L->sign_seed, &chk);
+  if (r != TQ_OK) return r;
+  if (std::memcmp(&chk, L, sizeof(chk)) != 0) return TQ_ERR_INVALID_ARG;  // edited or stale layout
+  return TQ_OK;
+}
+
+void copy_signs(const tq_layout_t* L, uint64_t (&dst)[4]) {
+  for (int i = 0; i < 4; ++i) dst[i] = L->sign_bits[i];
+}
+
+uint64_t workspace_bytes(int batch, int n_q, int D, int max_ctas) {
+  const uint64_t slots = (uint64_t)max_ctas + (uint64_t)batch;
+  const uint64_t header = 8ull * (uint64_t)(batch + 2);
+  const uint64_t ml = slots * (uint64_t)n_q * 2ull * 4ull;
+  const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
+  return ((header + ml + 255) / 256) * 256 + acc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                    uint64_t sign_seed, tq_layout_t* out) {
+  if (out == nullptr) return TQ_ERR_INVALID_ARG;
+  if (batch <= 0 || max_seq <= 0 || n_kv_heads <= 0 || n_q_heads <= 0) return TQ_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads != 0) return TQ_ERR_INVALID_ARG;
+  // mlxcel §"Known limitations / head dimension": power-of-two head dims only.
+  if (!is_pow2(head_dim) || head_dim < 32 || head_dim > 256) return TQ_ERR_UNSUPPORTED;
+  if (group_size != 32) return TQ_ERR_UNSUPPORTED;
+  if ((int64_t)batch * (int64_t)max_seq > (int64_t)INT32_MAX) return TQ_ERR_UNSUPPORTED;  // tensor-copy coordinates
+  tq_layout_t L;
+  std::memset(&L, 0, sizeof(L));
+  L.batch = batch;
+  L.max_seq = max_seq;
+  L.n_kv_heads = n_kv_heads;
+  L.n_q_heads = n_q_heads;
+  L.head_dim = head_dim;
+  L.group_size = group_size;
+  L.n_groups = head_dim / 32;
+  L.c_d = (float)(1.0 / std::sqrt((double)head_dim));
+  L.sign_seed = sign_seed;
+  uint64_t st = sign_seed;
+  for (int i = 0; i < head_dim; ++i)
+    if (splitmix64_step(st) >> 63) L.sign_bits[i >> 6] |= 1ull << (i & 63);
+  L.code_stride_tok = (int64_t)n_kv_heads * head_dim / 2;
+  L.code_stride_seq = (int64_t)max_seq * L.code_stride_tok;
+  L.scale_stride_tok = (int64_t)n_kv_heads * L.n_groups;
+  L.scale_stride_seq = (int64_t)max_seq * L.scale_stride_tok;
+  L.codes_bytes = (uint64_t)batch * (uint64_t)L.code_stride_seq;
+  const uint64_t srow = (uint64_t)L.scale_stride_tok * 2ull;
+  L.scales_bytes = (uint64_t)batch * (uint64_t)L.scale_stride_seq * 2ull + kMaxTileTokens * srow + 32ull;
+  L.max_ctas = kMaxCtas;
+  L.decode_workspace_bytes = workspace_bytes(batch, n_q_heads, head_dim, kMaxCtas);
+  *out = L;
+  return TQ_OK;
+}
+
+int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                       const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
+                       uint16_t* v_scales, int32_t* d_status, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (n_new < 0) return TQ_ERR_INVALID_ARG;
+  if (n_new > layout->max_seq) return TQ_ERR_CAPACITY;
+  if (in_dtype != TQ_F32 && in_dtype != TQ_BF16 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+  if (n_new == 0) return TQ_OK;
+  if (!k || !v || !d_start_pos || !k_codes || !k_scales || !v_codes || !v_scales) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes)) return TQ_ERR_INVALID_ARG;
+  if ((int64_t)layout->batch * n_new * layout->n_kv_heads * layout->n_groups * 2 > (int64_t)INT32_MAX * 256)
+    return TQ_ERR_UNSUPPORTED;
+  tqk::QuantizeParams p;
+  p.k = k;
+  p.v = v;
+  p.in_dtype = in_dtype;
+  p.batch = layout->batch;
+  p.n_new = n_new;
+  p.n_kv = layout->n_kv_heads;
+  p.max_seq = layout->max_seq;
+  p.start_pos = d_start_pos;
+  p.k_codes = k_codes;
+  p.k_scales = k_scales;
+  p.v_codes = v_codes;
+  p.v_scales = v_scales;
+  p.status = d_status;
+  copy_signs(layout, p.sign_bits);
+  p.c_d = layout->c_d;
+  cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e);
+}
+
+int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                           const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes,
+                           const uint16_t* v_scales, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                           int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  const int D = layout->head_dim, Hkv = layout->n_kv_heads, Hq = layout->n_q_heads;
+  const int G = Hq / Hkv;
+  if (layout->batch > kMaxBatchDecode) return TQ_ERR_UNSUPPORTED;
+  if (!(Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) || G > 8) return TQ_ERR_UNSUPPORTED;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+  if (!q || !d_seq_lens || !k_codes || !k_scales || !v_codes || !v_scales || !out || !workspace)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) ||
+      !aligned16(v_scales) || !aligned16(out) || !aligned16(workspace))
+    return TQ_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return TQ_ERR_INVALID_ARG;
+  int sms = 0;
+  r = device_sm_count(&sms);
+  if (r != TQ_OK) return r;
+  int grid = sms;
+  int min_split = 128;
+  cudaEvent_t ev = nullptr;
+  if (opts != nullptr) {
+    if (opts->max_ctas < 0 || opts->max_ctas > layout->max_ctas || opts->min_split_tokens < 0)
+      return TQ_ERR_INVALID_ARG;
+    if (opts->max_ctas > 0) grid = opts->max_ctas;
+    if (opts->min_split_tokens > 0) min_split = opts->min_split_tokens;
+    ev = reinterpret_cast<cudaEvent_t>(opts->after_split_event);
+  }
+  if (grid > layout->max_ctas) grid = layout->max_ctas;
+  if (ws_bytes < workspace_bytes(layout->batch, Hq, D, grid)) return TQ_ERR_INVALID_ARG;
+  if (tqk::decode_smem_bytes(D, Hkv) <= 0) return TQ_ERR_UNSUPPORTED;
+
+  tqk::TensorMap128 km, vm;
+  r = encode_codes_map(layout, k_codes, tqk::decode_tile_tokens(D, Hkv), &km);
+  if (r != TQ_OK) return r;
+  r = encode_codes_map(layout, v_codes, tqk::decode_tile_tokens(D, Hkv), &vm);
+  if (r != TQ_OK) return r;
+
+  tqk::DecodeParams p;
+  p.q = q;
+  p.q_dtype = q_dtype;
+  p.seq_lens = d_seq_lens;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  const uint64_t header_ml =
+      ((8ull * (uint64_t)(layout->batch + 2) + (uint64_t)(grid + layout->batch) * Hq * 8ull + 255) / 256) * 256;
+  p.ws_ml = reinterpret_cast<float*>(workspace);
+  p.ws_acc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + header_ml);
+  p.out = out;
+  p.status = d_status;
+  p.batch = layout->batch;
+  p.max_seq = layout->max_seq;
+  p.n_kv = Hkv;
+  p.n_q = Hq;
+  p.group = G;
+  p.grid = grid;
+  p.min_split = min_split;
+  p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  p.c_d = layout->c_d;
+  copy_signs(layout, p.sign_bits);
+  cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e);
+}
+
+int tq_decode_attention(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                        const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes,
+                        const uint16_t* v_scales, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                        int32_t* d_status, void* stream) {
+  return tq_decode_attention_ex(layout, q, q_dtype, d_seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out,
+                                workspace, ws_bytes, d_status, nullptr, stream);
+}
+
+int tq_dequantize_debug(const tq_layout_t* layout, const uint8_t* codes, const uint16_t* scales,
+                        const int32_t* d_seq_lens, int original_domain, float* out, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (!codes || !scales || !d_seq_lens || !out) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+  tqk::DequantParams p;
+  p.codes = codes;
+  p.scales = scales;
+  p.seq_lens = d_seq_lens;
+  p.out = out;
+  p.batch = layout->batch;
+  p.max_seq = layout->max_seq;
+  p.n_kv = layout->n_kv_heads;
+  p.original_domain = original_domain ? 1 : 0;
+  p.status = nullptr;
+  copy_signs(layout, p.sign_bits);
+  p.c_d = layout->c_d;
+  cudaError_t e = tqk::launch_dequantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e);
+}
+
+const char* tq_status_string(int status) {
+  switch (status) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument";
+    case TQ_ERR_UNSUPPORTED: return "unsupported shape";
+    case TQ_ERR_CAPACITY: return "capacity exceeded";
+    case TQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int tq_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

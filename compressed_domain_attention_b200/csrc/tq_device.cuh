@@ -1,0 +1,223 @@
+// Device helpers shared by the sm_100a kernels of libtq_b200.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tqk {
+
+// ----------------------------------------------------------------------------
+// Walsh-Hadamard transform over a vector spread across a group of NG threads,
+// each thread holding 32 consecutive elements (thread p of the group holds
+// elements [32p, 32p + 32)). The butterfly stages run with stride
+// h = 1, 2, ..., D/2 in that order; the pair (i, i+h) with (i & h) == 0 becomes
+// (u_i + u_{i+h}, u_i - u_{i+h}). Strides 1..16 are in registers; strides
+// 32..D/2 pair thread p with thread p ^ (h/32) through warp shuffles: the lower
+// thread forms own + partner, the upper thread partner - own. Every add is an
+// explicit round-to-nearest binary32 operation (no contraction), so the result
+// is identical to the same stage sequence run element by element.
+// `part` is the thread's index in its group; the group's lanes must be
+// consecutive and aligned to NG inside the warp; all 32 lanes must call this.
+// ----------------------------------------------------------------------------
+template <int NG>
+__device__ __forceinline__ void fwht_group(float (&u)[32], int part) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & h) == 0) {
+        const float a = u[i], b = u[i + h];
+        u[i] = __fadd_rn(a, b);
+        u[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 1; hh < NG; hh <<= 1) {
+    const bool upper = (part & hh) != 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, u[i], hh);
+      u[i] = upper ? __fsub_rn(o, u[i]) : __fadd_rn(u[i], o);
+    }
+  }
+}
+
+// Sign flip of element e by bit e of the sign mask (exact).
+__device__ __forceinline__ float apply_sign(float x, const uint64_t* sign_bits, int e) {
+  const uint32_t bit = (uint32_t)(sign_bits[e >> 6] >> (e & 63)) & 1u;
+  return __uint_as_float(__float_as_uint(x) ^ (bit << 31));
+}
+
+// Load 32 consecutive elements of dtype `dt` starting at element index `idx`
+// of `base` (16-byte aligned run) as binary32 (exact widening).
+__device__ __forceinline__ void load32(float (&x)[32], const void* base, int64_t idx, int dt) {
+  if (dt == TQ_F32) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(base) + idx);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 w = __ldg(p + j);
+      x[4 * j + 0] = __uint_as_float(w.x);
+      x[4 * j + 1] = __uint_as_float(w.y);
+      x[4 * j + 2] = __uint_as_float(w.z);
+      x[4 * j + 3] = __uint_as_float(w.w);
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + idx);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 w = __ldg(p + j);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = ww[k] & 0xffffu, hi = ww[k] >> 16;
+        if (dt == TQ_BF16) {
+          x[8 * j + 2 * k] = __uint_as_float(lo << 16);
+          x[8 * j + 2 * k + 1] = __uint_as_float(hi << 16);
+        } else {
+          x[8 * j + 2 * k] = __half2float(__ushort_as_half((unsigned short)lo));
+          x[8 * j + 2 * k + 1] = __half2float(__ushort_as_half((unsigned short)hi));
+        }
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float load_scalar(const void* base, int64_t idx, int dt) {
+  if (dt == TQ_F32) return reinterpret_cast<const float*>(base)[idx];
+  const uint16_t h = reinterpret_cast<const uint16_t*>(base)[idx];
+  if (dt == TQ_BF16) return __uint_as_float((uint32_t)h << 16);
+  return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ void status_or(int32_t* st, int32_t bits) {
+  if (st != nullptr && bits != 0) atomicOr(st, bits);
+}
+
+// ----------------------------------------------------------------------------
+// PTX wrappers: shared-memory addresses, mbarriers, bulk / tensor copies.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete, giving up after
+// `limit_ns` nanoseconds of wall time. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 3-D tiled tensor load into this CTA's shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Contiguous bulk copy global -> this CTA's shared memory (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// Tensor-core fragments (legacy warp-level MMA, register operands).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+
+// D = A(16x16, f16) * B(16x8, f16) + C, f32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// lop3 with an explicit truth table: (a & b) ^ c.
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace tqk

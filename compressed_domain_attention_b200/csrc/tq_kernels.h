@@ -1,0 +1,65 @@
+// Kernel parameter blocks and launchers (internal to libtq_b200).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tqk {
+
+struct QuantizeParams {
+  const void* k;
+  const void* v;
+  int in_dtype;
+  int batch, n_new, n_kv, max_seq;
+  const int32_t* start_pos;
+  uint8_t* k_codes;
+  uint16_t* k_scales;
+  uint8_t* v_codes;
+  uint16_t* v_scales;
+  int32_t* status;
+  uint64_t sign_bits[4];
+  float c_d;
+};
+
+struct DequantParams {
+  const uint8_t* codes;
+  const uint16_t* scales;
+  const int32_t* seq_lens;
+  float* out;
+  int batch, max_seq, n_kv, original_domain;
+  int32_t* status;
+  uint64_t sign_bits[4];
+  float c_d;
+};
+
+// 128-byte opaque copy of a CUtensorMap (passed by value as a __grid_constant__).
+struct alignas(64) TensorMap128 {
+  uint64_t words[16];
+};
+
+struct DecodeParams {
+  const void* q;
+  int q_dtype;
+  const int32_t* seq_lens;
+  const uint16_t* k_scales;
+  const uint16_t* v_scales;
+  float* ws_ml;    // [slots][n_q][2]: running max (log2 units), running sum
+  float* ws_acc;   // [slots][n_q][D]: rotated-domain accumulator, relative to the running max
+  float* out;      // [batch][n_q][D]
+  int32_t* status;
+  int batch, max_seq, n_kv, n_q, group;
+  int grid;            // CTAs in the split-K launch
+  int min_split;       // smallest token range per CTA
+  float sm_scale_log2; // sm_scale * log2(e)
+  float c_d;
+  uint64_t sign_bits[4];
+};
+
+cudaError_t launch_quantize(const QuantizeParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_dequantize(const DequantParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, const TensorMap128& kmap, const TensorMap128& vmap, int head_dim,
+                          cudaStream_t s, cudaEvent_t after_split);
+int decode_smem_bytes(int head_dim, int n_kv);
+int decode_tile_tokens(int head_dim, int n_kv);
+
+}  // namespace tqk

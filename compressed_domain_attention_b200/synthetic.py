@@ -124,20 +124,23 @@ def generate(w: Workload, device: str = "cpu", seq_subset: Optional[List[int]] =
     """
     g = torch.Generator(device).manual_seed(w.seed)
     Hkv, D = w.n_kv_heads, w.head_dim
-    base = [torch.randn((L, Hkv, D), generator=g, device=device) for L in w.seq_lens]
+    keep = set(range(w.batch)) if seq_subset is None else set(seq_subset)
+    base = []
+    for b, L in enumerate(w.seq_lens):
+        x = torch.randn((L, Hkv, D), generator=g, device=device)
+        base.append(x if b in keep else None)  # the draw happens either way
     z = torch.randn((Hkv, D), generator=g, device=device)
     mult = torch.exp(z)
     n_out = D // 32
     for h in range(Hkv):
         idx = torch.randperm(D, generator=g, device=device)[:n_out]
         mult[h, idx] *= 10.0
-    keep = set(range(w.batch)) if seq_subset is None else set(seq_subset)
     k = [(base[b] * mult).to(w.dtype) if b in keep else None for b in range(w.batch)]
     del base
     v = []
     for b, L in enumerate(w.seq_lens):
-        t = torch.randn((L, Hkv, D), generator=g, device=device)
-        v.append(t.to(w.dtype) if b in keep else None)
+        x = torch.randn((L, Hkv, D), generator=g, device=device)
+        v.append(x.to(w.dtype) if b in keep else None)
     q = torch.randn((w.batch, w.n_q_heads, D), generator=g, device=device).to(w.dtype)
     kn = (torch.randn((w.batch, w.n_append, Hkv, D), generator=g, device=device) * mult).to(w.dtype)
     vn = torch.randn((w.batch, w.n_append, Hkv, D), generator=g, device=device).to(w.dtype)

@@ -1,0 +1,187 @@
+"""Thin ctypes binding of ``libtq_b200.so`` (declared in ``include/tq.h``).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels. Tensors are torch tensors (device memory and streams come from
+PyTorch); their ``data_ptr()`` values and the current CUDA stream handle are
+passed through unchanged. There is no CPU fallback: if the library is missing
+the first call raises.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtq_b200.so")
+
+TQ_OK = 0
+TQ_ERR_INVALID_ARG = -1
+TQ_ERR_UNSUPPORTED = -2
+TQ_ERR_CAPACITY = -3
+TQ_ERR_CUDA = -4
+
+TQ_STATUS_NONFINITE = 1
+TQ_STATUS_CAPACITY = 2
+TQ_STATUS_TIMEOUT = 4
+
+TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
+
+# C symbols declared in include/tq.h
+EXPORTS = ("tq_cache_layout", "tq_quantize_append", "tq_decode_attention", "tq_decode_attention_ex",
+           "tq_dequantize_debug", "tq_status_string", "tq_last_cuda_error")
+
+
+class TqLayout(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("max_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("group_size", ctypes.c_int32),
+        ("n_groups", ctypes.c_int32), ("c_d", ctypes.c_float),
+        ("sign_seed", ctypes.c_uint64), ("sign_bits", ctypes.c_uint64 * 4),
+        ("code_stride_tok", ctypes.c_int64), ("code_stride_seq", ctypes.c_int64),
+        ("scale_stride_tok", ctypes.c_int64), ("scale_stride_seq", ctypes.c_int64),
+        ("codes_bytes", ctypes.c_uint64), ("scales_bytes", ctypes.c_uint64),
+        ("decode_workspace_bytes", ctypes.c_uint64),
+        ("max_ctas", ctypes.c_int32), ("reserved", ctypes.c_int32),
+    ]
+
+
+class TqDecodeOpts(ctypes.Structure):
+    _fields_ = [("min_split_tokens", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
+                ("after_split_event", ctypes.c_void_p)]
+
+
+class TqError(RuntimeError):
+    def __init__(self, fn, code):
+        lib = _lib()
+        msg = lib.tq_status_string(code).decode()
+        extra = f" (cuda error {lib.tq_last_cuda_error()})" if code == TQ_ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {msg} [{code}]{extra}")
+        self.code = code
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                              "(there is no CPU fallback for this library)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+        lib.tq_cache_layout.argtypes = [I, I, I, I, I, I, U64, ctypes.POINTER(TqLayout)]
+        lib.tq_cache_layout.restype = I
+        lib.tq_quantize_append.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
+        lib.tq_quantize_append.restype = I
+        lib.tq_decode_attention.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float, P, P,
+                                            ctypes.c_size_t, P, P]
+        lib.tq_decode_attention.restype = I
+        lib.tq_decode_attention_ex.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float, P, P,
+                                               ctypes.c_size_t, P, ctypes.POINTER(TqDecodeOpts), P]
+        lib.tq_decode_attention_ex.restype = I
+        lib.tq_dequantize_debug.argtypes = [ctypes.POINTER(TqLayout), P, P, P, I, P, P]
+        lib.tq_dequantize_debug.restype = I
+        lib.tq_status_string.argtypes = [I]
+        lib.tq_status_string.restype = ctypes.c_char_p
+        lib.tq_last_cuda_error.argtypes = []
+        lib.tq_last_cuda_error.restype = I
+        _LIB = lib
+    return _LIB
+
+
+def _check(fn, code):
+    if code != TQ_OK:
+        raise TqError(fn, code)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}[t.dtype]
+
+
+def tq_cache_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size=32, sign_seed=0) -> TqLayout:
+    out = TqLayout()
+    _check("tq_cache_layout", _lib().tq_cache_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size,
+                                                     ctypes.c_uint64(sign_seed), ctypes.byref(out)))
+    return out
+
+
+def tq_cache_layout_status(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size=32, sign_seed=0):
+    """Raw status code variant (for callers that test rejection paths)."""
+    out = TqLayout()
+    code = _lib().tq_cache_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size,
+                                  ctypes.c_uint64(sign_seed), ctypes.byref(out))
+    return code, out
+
+
+def tq_quantize_append(layout, k, v, n_new, start_pos, k_codes, k_scales, v_codes, v_scales, status=None,
+                       stream=None):
+    """k, v: [batch][n_new][Hkv][D] (f32/bf16/f16, CUDA, contiguous); start_pos: int32 [batch] on the device."""
+    for t in (k, v, start_pos, k_codes, k_scales, v_codes, v_scales):
+        assert t.is_contiguous()
+    code = _lib().tq_quantize_append(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
+                                     _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                     _ptr(v_scales), _ptr(status), _stream(stream))
+    _check("tq_quantize_append", code)
+
+
+def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out, workspace,
+                        status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None):
+    """q: [batch][Hq][D]; out: float32 [batch][Hq][D]; workspace: >= layout.decode_workspace_bytes bytes."""
+    for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out, workspace):
+        assert t.is_contiguous()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    lib = _lib()
+    if min_split_tokens or max_ctas or after_split_event is not None:
+        opts = TqDecodeOpts(int(min_split_tokens), int(max_ctas),
+                            ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None)
+        code = lib.tq_decode_attention_ex(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
+                                          _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                          ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes,
+                                          _ptr(status), ctypes.byref(opts), _stream(stream))
+    else:
+        code = lib.tq_decode_attention(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
+                                       _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                       ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes,
+                                       _ptr(status), _stream(stream))
+    _check("tq_decode_attention", code)
+
+
+def tq_dequantize_debug(layout, codes, scales, seq_lens, original_domain, out, stream=None):
+    code = _lib().tq_dequantize_debug(ctypes.byref(layout), _ptr(codes), _ptr(scales), _ptr(seq_lens),
+                                      1 if original_domain else 0, _ptr(out), _stream(stream))
+    _check("tq_dequantize_debug", code)
+
+
+def sign_vector(layout):
+    """The layout's +-1 diagonal as a Python list of floats (read from its sign bits)."""
+    return [(-1.0 if (layout.sign_bits[i >> 6] >> (i & 63)) & 1 else 1.0) for i in range(layout.head_dim)]
+
+
+def alloc_cache(layout, device="cuda"):
+    """Allocate (k_codes, k_scales, v_codes, v_scales) with the layout's sizes (zero-filled)."""
+    import torch
+    cb = int(layout.codes_bytes)
+    sb = int(layout.scales_bytes)
+    k_codes = torch.zeros(cb, dtype=torch.uint8, device=device)
+    v_codes = torch.zeros(cb, dtype=torch.uint8, device=device)
+    k_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
+    v_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
+    return k_codes, k_scales, v_codes, v_scales
+
+
+def alloc_workspace(layout, device="cuda"):
+    import torch
+    return torch.empty(int(layout.decode_workspace_bytes), dtype=torch.uint8, device=device)

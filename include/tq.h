@@ -1,0 +1,174 @@
+/*
+ * tq.h - C ABI of the B200 (sm_100a) library for rotation-based int4 KV-cache
+ * quantisation and decode attention computed on the packed cache.
+ *
+ * The method (sources cited by page title and section):
+ *  - "Open-TQ-Metal: Fused Compressed-Domain Attention for Long-Context LLM
+ *    Inference on Apple Silicon", abstract (cards page): each cached K/V head
+ *    vector goes through one fused quantiser: a sign-randomised transform,
+ *    per-group abs-max scaling, int4 codes packed two per byte. The paper
+ *    exposes it as a cache object that quantises on append.
+ *  - the same paper's arXiv abstract: attention runs directly on the
+ *    compressed representation with no intermediate dequantised K/V matrix;
+ *    the attention scale (1/sqrt(d) or a model's own, e.g. 1.0) is an input.
+ *  - mlxcel user guide "TurboQuant KV cache compression", §"What TurboQuant
+ *    changes" (Walsh-Hadamard rotation before low-bit storage) and §"Known
+ *    limitations / head dimension" (power-of-two head dims only; others are
+ *    rejected when the cache is created).
+ *  - "TurboQuant on AMD GPUs", §4: the Walsh-Hadamard transform is used as the
+ *    rotation because it spreads energy evenly and suits GPU kernels.
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *  - rotation: y = c_D * H * (s o x), H the Sylvester Hadamard matrix applied
+ *    as radix-2 butterflies with stride 1, 2, ..., D/2; c_D = binary32(1/sqrt(D))
+ *    applied once; s a +-1 vector drawn from SplitMix64(sign_seed), shared by
+ *    K, V, q and every head;
+ *  - groups of 32 consecutive rotated elements; scale = binary16(absmax / 7),
+ *    codes = clamp(round_half_even(y / scale), -7, 7) against the stored scale;
+ *  - packing: two's-complement nibbles, element 2j in the low nibble of byte j.
+ *
+ * Memory (all buffers are owned by the caller; the library allocates nothing
+ * and keeps no state between calls):
+ *  - codes  [batch][max_seq][n_kv_heads][head_dim/2]  uint8   (one buffer for K, one for V)
+ *  - scales [batch][max_seq][n_kv_heads][head_dim/32] binary16 bits (one for K, one for V)
+ *    Allocate `scales_bytes` (slightly more than the array): decode reads
+ *    scale rows in tile-sized blocks that may run past the last valid token.
+ *  - every device buffer must be 16-byte aligned (cudaMalloc gives 256).
+ *
+ * Errors: argument errors return a negative tq_status and launch nothing.
+ * Errors found on the device (a length past max_seq, a non-finite group, a
+ * bounded wait that ran out) are OR-ed into *d_status when d_status is not
+ * NULL (bits TQ_STATUS_*); the affected unit is skipped, never trapped.
+ * All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream). The library never aborts the process.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = -1, /* NULL pointer, bad size, misaligned buffer, workspace too small */
+  TQ_ERR_UNSUPPORTED = -2, /* head_dim not a power of two in [32, 256], group_size != 32, shape limits */
+  TQ_ERR_CAPACITY = -3,    /* n_new larger than max_seq */
+  TQ_ERR_CUDA = -4         /* a CUDA launch or runtime call failed (see tq_last_cuda_error) */
+} tq_status;
+
+/* Bits OR-ed into *d_status by device code. */
+#define TQ_STATUS_NONFINITE 1 /* a group held a non-finite value, or its scale overflowed binary16: stored as scale +inf, codes 0 */
+#define TQ_STATUS_CAPACITY 2  /* an append past max_seq (that sequence skipped), or seq_len outside [0, max_seq] (treated as 0) */
+#define TQ_STATUS_TIMEOUT 4   /* a bounded pipeline wait ran out; that work unit's output is incomplete */
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Filled by tq_cache_layout; plain data, caller-owned, never modified by the library. */
+typedef struct {
+  int32_t batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size;
+  int32_t n_groups;            /* head_dim / 32 */
+  float c_d;                   /* binary32(1/sqrt(head_dim)) */
+  uint64_t sign_seed;
+  uint64_t sign_bits[4];       /* bit i set <=> s_i = -1 (head_dim <= 256) */
+  int64_t code_stride_tok;     /* bytes between tokens of one sequence   = n_kv * D/2 */
+  int64_t code_stride_seq;     /* bytes between sequences                 = max_seq * n_kv * D/2 */
+  int64_t scale_stride_tok;    /* binary16 elements between tokens         = n_kv * D/32 */
+  int64_t scale_stride_seq;    /* binary16 elements between sequences      = max_seq * n_kv * D/32 */
+  uint64_t codes_bytes;        /* allocation size of ONE codes buffer (K or V) */
+  uint64_t scales_bytes;       /* allocation size of ONE scales buffer, including read-ahead padding */
+  uint64_t decode_workspace_bytes; /* workspace tq_decode_attention needs with default options */
+  int32_t max_ctas;            /* largest split-K grid the workspace size allows */
+  int32_t reserved;
+} tq_layout_t;
+
+/* Optional knobs for tq_decode_attention_ex (NULL = defaults). */
+typedef struct {
+  int32_t min_split_tokens; /* 0 = default; otherwise the smallest token range one CTA takes */
+  int32_t max_ctas;         /* 0 = default (one per SM); otherwise the split-K grid, <= layout.max_ctas */
+  void* after_split_event;  /* a cudaEvent_t recorded on `stream` between the split-K and merge kernels, or NULL */
+} tq_decode_opts_t;
+
+/*
+ * Validate a cache shape and fill *out. Host only: no device work, no CUDA
+ * call. head_dim must be a power of two in [32, 256] (mlxcel §"Known
+ * limitations / head dimension"); group_size must be 32; n_q_heads must be a
+ * multiple of n_kv_heads (grouped-query attention, kv head = q head / G).
+ * Returns TQ_OK, TQ_ERR_INVALID_ARG or TQ_ERR_UNSUPPORTED.
+ */
+int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim,
+                    int group_size, uint64_t sign_seed, tq_layout_t* out);
+
+/*
+ * Quantise and append n_new tokens to every sequence (Open-TQ-Metal abstract:
+ * the fused sign-randomised transform + per-group abs-max + int4 nibble pack,
+ * run when the cache is appended to).
+ *   k, v         device, [batch][n_new][n_kv_heads][head_dim] of in_dtype
+ *   d_start_pos  device int32 [batch]: token t of sequence b is written at
+ *                position d_start_pos[b] + t. A sequence whose append would
+ *                pass max_seq (or a negative start) is skipped and sets
+ *                TQ_STATUS_CAPACITY.
+ *   k_codes, v_codes, k_scales, v_scales   device caches (layout above).
+ * n_new == 0 is a no-op. Codes and scales are bit-exact with the reference
+ * definition (IEEE binary32 steps, no contraction, round-half-even).
+ */
+int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype,
+                       int n_new, const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales,
+                       uint8_t* v_codes, uint16_t* v_scales, int32_t* d_status, void* stream);
+
+/*
+ * One decode query per sequence over its packed cache (Open-TQ-Metal arXiv
+ * abstract: attention directly on the compressed representation).
+ *   q            device [batch][n_q_heads][head_dim] of q_dtype
+ *   d_seq_lens   device int32 [batch]: attend to positions [0, len_b); len_b == 0
+ *                gives a zero output row; len_b outside [0, max_seq] is treated
+ *                as 0 and sets TQ_STATUS_CAPACITY.
+ *   sm_scale     softmax scale (1/sqrt(head_dim) for standard models)
+ *   out          device float32 [batch][n_q_heads][head_dim], original (unrotated) domain
+ *   workspace    device scratch of at least layout.decode_workspace_bytes
+ *                (split-K partials: running max, sum and rotated-domain
+ *                accumulator per q head and split; no dequantised K/V is
+ *                ever written)
+ * The query is rotated by the same transform, K and V nibbles are unpacked in
+ * registers, softmax runs online over split-K token ranges, the partials are
+ * merged, and one inverse transform produces the output.
+ * Limits: batch <= 1024; n_kv_heads in {1, 2, 4, 8}; n_q_heads / n_kv_heads <= 8
+ * (otherwise TQ_ERR_UNSUPPORTED).
+ */
+int tq_decode_attention(const tq_layout_t* layout, const void* q, int q_dtype,
+                        const int32_t* d_seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
+                        const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
+                        void* workspace, size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* tq_decode_attention with explicit options (opts may be NULL). */
+int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype,
+                           const int32_t* d_seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
+                           const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
+                           void* workspace, size_t ws_bytes, int32_t* d_status,
+                           const tq_decode_opts_t* opts, void* stream);
+
+/*
+ * Debug / comparator path: dequantise a whole cache into a dense float32
+ * array out [batch][max_seq][n_kv_heads][head_dim]; rows at t >= d_seq_lens[b]
+ * are written as 0. original_domain = 0 gives code * scale (rotated domain);
+ * 1 also applies the inverse rotation. This is the "dequantise-then-attend"
+ * baseline's first half (Open-TQ-Metal arXiv abstract); the decode path never
+ * calls it.
+ */
+int tq_dequantize_debug(const tq_layout_t* layout, const uint8_t* codes, const uint16_t* scales,
+                        const int32_t* d_seq_lens, int original_domain, float* out, void* stream);
+
+/* Human-readable text for a tq_status value. Never NULL. */
+const char* tq_status_string(int status);
+
+/* The last CUDA error code seen by a call that returned TQ_ERR_CUDA (0 if none). */
+int tq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */
