@@ -1,0 +1,102 @@
+// tq_decode_attention_noalloc: decode attention for callers that cannot
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they decode: code
+// running inside a custom allocator or memory pool that must not re-enter
+// itself, runtimes that forbid device allocation after start-up (fixed memory
+// budgets, pre-planned arenas), and plug-ins handed only the tensors they work
+// on. The regular entry point needs a caller-provided split-K workspace; this
+// one uses a fixed-size array that lives in the library's own device image
+// instead, so the caller passes only inputs and outputs.
+//
+// The array is a file-scope static device array: every GPU that loads this
+// library holds TQ_NOALLOC_WORKSPACE_BYTES of device memory for it until the
+// process exits. Host code cannot use the array's name as a device address
+// (in host code it names a host-side stand-in), so the first call on each
+// device looks up the real address with cudaGetSymbolAddress while that device
+// is current, and caches it.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/tq.h"
+
+namespace {
+
+// The shared scratch. No part of it needs to start at zero: the split-K kernel
+// writes every header entry and partial slot that the merge kernel reads in the
+// same call, so a call never depends on what an earlier call left behind.
+static __device__ __align__(256) unsigned char g_noalloc_ws[TQ_NOALLOC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Per-device address of g_noalloc_ws, set up once per device on first use.
+void* ws_address_for_current_device(int* err) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *err = (int)e;
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = (int)cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_ws);  // with `dev` current
+    if (e != cudaSuccess || p == nullptr) {
+      *err = (int)(e != cudaSuccess ? e : cudaErrorUnknown);
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+// Workspace the decode call needs for a split-K grid of `grid` CTAs: an int64
+// header (prefix sums of the lengths and the per-CTA token range), then
+// (running max, running sum) and a D-float accumulator per (slot, q head),
+// slots = grid + batch. This is the arithmetic of the documented workspace
+// layout; if it ever under-counted, the decode call itself would reject the
+// workspace size with TQ_ERR_INVALID_ARG rather than overrun it.
+uint64_t needed_bytes(int batch, int n_q, int D, int grid) {
+  const uint64_t slots = (uint64_t)grid + (uint64_t)batch;
+  const uint64_t header = 8ull * (uint64_t)(batch + 2);
+  const uint64_t ml = slots * (uint64_t)n_q * 8ull;
+  const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
+  return ((header + ml + 255) / 256) * 256 + acc;
+}
+
+}  // namespace
+
+extern "C" int tq_decode_attention_noalloc(const tq_layout_t* layout, const void* q, int q_dtype,
+                                           const int32_t* d_seq_lens, const uint8_t* k_codes,
+                                           const uint16_t* k_scales, const uint8_t* v_codes,
+                                           const uint16_t* v_scales, float sm_scale, float* out,
+                                           int32_t* d_status, void* stream) {
+  if (layout == nullptr) return TQ_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  if (sms > layout->max_ctas) sms = layout->max_ctas;
+  // Reject requests whose workspace would not fit, before touching the device.
+  if (needed_bytes(layout->batch, layout->n_q_heads, layout->head_dim, sms) > (uint64_t)TQ_NOALLOC_WORKSPACE_BYTES)
+    return TQ_ERR_CAPACITY;
+  int err = 0;
+  void* ws = ws_address_for_current_device(&err);
+  if (ws == nullptr) return TQ_ERR_CUDA;
+  tq_decode_opts_t opts;
+  opts.min_split_tokens = 0;
+  opts.max_ctas = sms;
+  opts.after_split_event = nullptr;
+  return tq_decode_attention_ex(layout, q, q_dtype, d_seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out,
+                                ws, (size_t)TQ_NOALLOC_WORKSPACE_BYTES, d_status, &opts, stream);
+}

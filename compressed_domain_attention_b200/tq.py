@@ -26,7 +26,9 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 # C symbols declared in include/tq.h
 EXPORTS = ("tq_cache_layout", "tq_quantize_append", "tq_decode_attention", "tq_decode_attention_ex",
-           "tq_dequantize_debug", "tq_status_string", "tq_last_cuda_error")
+           "tq_decode_attention_noalloc", "tq_dequantize_debug", "tq_status_string", "tq_last_cuda_error")
+
+TQ_NOALLOC_WORKSPACE_BYTES = 8 << 20
 
 
 class TqLayout(ctypes.Structure):
@@ -78,6 +80,9 @@ def _lib():
         lib.tq_decode_attention_ex.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float, P, P,
                                                ctypes.c_size_t, P, ctypes.POINTER(TqDecodeOpts), P]
         lib.tq_decode_attention_ex.restype = I
+        lib.tq_decode_attention_noalloc.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float,
+                                                    P, P, P]
+        lib.tq_decode_attention_noalloc.restype = I
         lib.tq_dequantize_debug.argtypes = [ctypes.POINTER(TqLayout), P, P, P, I, P, P]
         lib.tq_dequantize_debug.restype = I
         lib.tq_status_string.argtypes = [I]
@@ -157,6 +162,24 @@ def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scale
                                        ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes,
                                        _ptr(status), _stream(stream))
     _check("tq_decode_attention", code)
+
+
+def tq_decode_attention_noalloc(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out,
+                                status=None, stream=None):
+    """Decode without a caller workspace, for callers that cannot allocate device memory.
+
+    The split-K scratch comes from a fixed array inside the library's device
+    image (TQ_NOALLOC_WORKSPACE_BYTES per GPU), so nothing is allocated here.
+    Calls on one device share that array: do not let two of them overlap on
+    the GPU. Raises TqError (TQ_ERR_CAPACITY) when the request needs more
+    scratch than the array holds.
+    """
+    for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out):
+        assert t.is_contiguous()
+    code = _lib().tq_decode_attention_noalloc(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
+                                              _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                              ctypes.c_float(sm_scale), _ptr(out), _ptr(status), _stream(stream))
+    _check("tq_decode_attention_noalloc", code)
 
 
 def tq_dequantize_debug(layout, codes, scales, seq_lens, original_domain, out, stream=None):

@@ -151,6 +151,38 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
                            const tq_decode_opts_t* opts, void* stream);
 
 /*
+ * Decode for callers that cannot allocate device memory. (The paper has no
+ * counterpart: this is a deployment variant of tq_decode_attention.)
+ *
+ * Who needs it: code that runs where a cudaMalloc is not allowed or not
+ * possible - inside a memory pool or custom allocator that must not re-enter
+ * itself, runtimes with a fixed device-memory plan made at start-up, plug-ins
+ * that are handed only their input and output tensors. tq_decode_attention
+ * needs a caller-allocated workspace; this call instead uses a scratch array
+ * of TQ_NOALLOC_WORKSPACE_BYTES that is part of the library's own device image
+ * (a static device array: every GPU that loads the library holds it until the
+ * process exits). Inputs, outputs, results and limits are otherwise those of
+ * tq_decode_attention with the default one-CTA-per-SM split.
+ *
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture on that device.
+ *  - A request whose workspace would exceed TQ_NOALLOC_WORKSPACE_BYTES
+ *    (roughly (SMs + batch) * n_q_heads * (head_dim + 2) * 4 bytes) returns
+ *    TQ_ERR_CAPACITY and launches nothing.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents (nothing in it needs clearing: each call writes all it reads).
+ *    Calls that can overlap on the GPU (different streams, or other threads)
+ *    race on it: serialise them.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define TQ_NOALLOC_WORKSPACE_BYTES (8u << 20)
+int tq_decode_attention_noalloc(const tq_layout_t* layout, const void* q, int q_dtype,
+                                const int32_t* d_seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
+                                const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
+                                int32_t* d_status, void* stream);
+
+/*
  * Debug / comparator path: dequantise a whole cache into a dense float32
  * array out [batch][max_seq][n_kv_heads][head_dim]; rows at t >= d_seq_lens[b]
  * are written as 0. original_domain = 0 gives code * scale (rotated domain);
