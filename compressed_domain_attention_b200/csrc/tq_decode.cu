@@ -17,10 +17,13 @@
 //   warp 8      : producer. One lane streams token tiles of the contiguous
 //                 [tile][Hkv][D/2] code slabs (3-D tensor copies, swizzled to
 //                 the row pitch) and the [tile][Hkv][D/32] binary16 scale slabs
-//                 (bulk copies) into a 4-stage shared-memory ring guarded by
-//                 mbarriers.
-//   warps 0..7  : consumers. Warp w owns KV head w % Hkv and 16-token units of
-//                 each tile. Scores and P.V run on the tensor cores with
+//                 (bulk copies) into a 3- or 4-stage shared-memory ring guarded
+//                 by mbarriers.
+//   warp 9      : converter. Turns each stage's binary16 scales into fp32 in
+//                 the order the consumer lanes read them (conflict-free), with
+//                 tokens past the segment end set to 0.
+//   warps 0..7  : consumers. Warp w owns KV head w % Hkv and 32-token units
+//                 (16 at D = 256) of each tile. Scores and P.V run on the tensor cores with
 //                 register fragments (mma.m16n8k16, f16 in, f32 accumulate):
 //                 * Q.K^T: A = the rotated query of the group's q heads in
 //                   two binary16 pieces (hi + lo, rows 0-7 and 8-15), B = K
@@ -30,8 +33,12 @@
 //                   accumulator's initial value, and the per-group scale is
 //                   applied in binary32 after each group's two MMAs.
 //                 * P.V: A = V codes (pairs of tokens at one channel, from a
-//                   transposing ldmatrix), B = P times the per-(token, group)
-//                   V scale, rounded once to binary16.
+//                   transposing ldmatrix, same subnormal encoding), B = P
+//                   times the per-(token, group) V scale, rounded once to
+//                   binary16. The V codes enter signed (one binary16
+//                   subtract per pair removes the +8): an offset kept in
+//                   the accumulator would drift, because the tensor core's
+//                   fp32 sums round toward zero.
 // Kernel 2 (decode_merge_kernel): per (sequence, q head) the partials are
 // combined, normalised, and the inverse SRHT maps the result back to the
 // original domain.
@@ -43,33 +50,46 @@
 namespace tqk {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 4;
+constexpr int kProducerWarp = kConsumerWarps;       // one lane issues the copies
+constexpr int kConverterWarp = kConsumerWarps + 1;  // binary16 -> fp32 scales
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every pipeline wait
 
 template <int D, int HKV>
 struct DecodeCfg {
-  static constexpr int NG = D / 32;                    // groups per head vector
-  static constexpr int RB = D / 2;                     // code bytes per (token, head)
-  static constexpr int WPH = kConsumerWarps / HKV;     // consumer warps per KV head
-  static constexpr int UPW_MAX = 256 / D;              // 16-token units per warp per stage
-  static constexpr int UPW = UPW_MAX < 16 / WPH ? UPW_MAX : 16 / WPH;
-  static constexpr int T_TILE = 16 * UPW * WPH;        // tokens per stage (<= 256)
+  static constexpr int NG = D / 32;                  // groups per head vector
+  static constexpr int RB = D / 2;                   // code bytes per (token, head)
+  static constexpr int WPH = kConsumerWarps / HKV;   // consumer warps per KV head
+  static constexpr int UNIT = D <= 128 ? 32 : 16;    // tokens per warp work unit
+  static constexpr int NT = UNIT / 8;                // 8-token n-tiles per unit
+  static constexpr int KSP = UNIT / 16;              // 16-token k-steps of P.V per unit
+  static constexpr int UPW_A = 2048 / (UNIT * RB) > 0 ? 2048 / (UNIT * RB) : 1;
+  static constexpr int UPW_B = 256 / (UNIT * WPH) > 0 ? 256 / (UNIT * WPH) : 1;
+  static constexpr int UPW = UPW_A < UPW_B ? UPW_A : UPW_B;  // units per warp per stage
+  static constexpr int T_TILE = UNIT * UPW * WPH;    // tokens per stage (<= 256)
+  static constexpr int UNITS_TILE = T_TILE / UNIT;
   static constexpr int CODE_BYTES = T_TILE * HKV * RB;
-  static constexpr int SROW = HKV * NG * 2;            // scale bytes per token (all heads)
+  static constexpr int SROW = HKV * NG * 2;          // raw scale bytes per token (all heads)
   static constexpr int SCALE_SLAB = ((T_TILE * SROW + 15) / 16) * 16 + 16;
-  static constexpr int STAGE_BYTES = ((2 * CODE_BYTES + 2 * SCALE_SLAB + 1023) / 1024) * 1024;
+  static constexpr int SC_HEAD = T_TILE * NG + 4;    // fp32 scale floats per head (16 B pad)
+  static constexpr int SC_KV = HKV * SC_HEAD;
+  static constexpr int OFF_SC32 = 2 * CODE_BYTES + 2 * SCALE_SLAB;  // within a stage
+  static constexpr int STAGE_BYTES = ((OFF_SC32 + 2 * SC_KV * 4 + 1023) / 1024) * 1024;
   static constexpr uint32_t STAGE_TX = 2 * CODE_BYTES + 2 * SCALE_SLAB;
-  static constexpr int QSTRIDE = D + 4;                // floats per staged q row (padded)
+  static constexpr int STAGES = D == 256 ? 3 : 4;
+  static constexpr int QSTRIDE = D + 4;              // floats per staged q row (padded)
   static constexpr int SCRATCH = ((8 * QSTRIDE * 4 + 64 + 127) / 128) * 128;  // per consumer warp
   static constexpr int SWZ = RB == 128 ? 7 : RB == 64 ? 3 : RB == 32 ? 1 : 0;
-  static constexpr int OFF_SCRATCH = kStages * STAGE_BYTES;
+  static constexpr int OFF_SCRATCH = STAGES * STAGE_BYTES;
   static constexpr int OFF_BARS = OFF_SCRATCH + kConsumerWarps * SCRATCH;
-  static constexpr int OFF_MISC = OFF_BARS + 2 * kStages * 8;
+  static constexpr int OFF_MISC = OFF_BARS + 3 * STAGES * 8;
   static constexpr int OFF_PREFIX = OFF_MISC + 64;
+  static constexpr int SMEM_MAX = OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16;
   static_assert(T_TILE <= 256, "tensor-copy box limit");
   static_assert(CODE_BYTES % 1024 == 0, "V block must stay swizzle-aligned");
+  static_assert((2 * NG * NT) % 4 == 0, "ldmatrix.x4 batches");
+  static_assert(SMEM_MAX <= 232448, "shared memory per block");
 };
 
 // Workspace header: int64 prefix[batch + 1], int64 range_tokens.
@@ -177,11 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap) {
   using C = DecodeCfg<D, HKV>;
-  constexpr int NG = C::NG, RB = C::RB, T_TILE = C::T_TILE, UPW = C::UPW;
+  constexpr int NG = C::NG, RB = C::RB, T_TILE = C::T_TILE, UPW = C::UPW, NT = C::NT, KSP = C::KSP;
+  constexpr int UNIT = C::UNIT, STAGES = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
-  uint64_t* empty = full + kStages;
-  int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);  // [0] abort flag
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);  // copies landed
+  uint64_t* ready = full + STAGES;                                  // fp32 scales written
+  uint64_t* empty = ready + STAGES;                                 // stage free again
+  int* misc = reinterpret_cast<int*>(smem + C::OFF_MISC);           // [0] abort flag
   int64_t* prefix = reinterpret_cast<int64_t*>(smem + C::OFF_PREFIX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -206,9 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&ready[s], 1);
+      mbar_init(&empty[s], kConsumerWarps + 1);
     }
     misc[0] = 0;
     fence_mbar_init();
@@ -218,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileWalker walk;
   walk.start(prefix, p.batch, lo, hi);
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
     const uint64_t pol = l2_policy_evict_first();
@@ -227,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool dead = false;
     for (; !walk.done(); walk.advance<T_TILE>()) {
-      const int stage = issued % kStages;
-      const uint32_t n = (uint32_t)(issued / kStages);
+      const int stage = issued % STAGES;
+      const uint32_t n = (uint32_t)(issued / STAGES);
       if (!mbar_wait_bounded(&empty[stage], (n & 1u) ^ 1u, kWaitLimitNs)) {
         dead = true;
         break;
@@ -250,8 +273,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       status_or(p.status, TQ_STATUS_TIMEOUT);
     }
     // drain: no copy may still be in flight when this thread exits
-    for (int k = max(0, issued - kStages); k < issued; ++k)
-      (void)mbar_wait_bounded(&full[k % kStages], (uint32_t)((k / kStages) & 1), kWaitLimitNs);
+    for (int k = max(0, issued - STAGES); k < issued; ++k)
+      (void)mbar_wait_bounded(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), kWaitLimitNs);
+    return;
+  }
+
+  if (warp == kConverterWarp) {
+    // ------------------------------------------------------------ converter
+    // binary16 scale rows [token][head][group] -> fp32 [head][unit][group][tig][n-tile][e],
+    // the order in which a consumer lane reads them; tokens past the segment end get 0.
+    bool dead = false;
+    int tile_i = 0;
+    for (; !walk.done(); walk.advance<T_TILE>(), ++tile_i) {
+      const int stage = tile_i % STAGES;
+      const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
+      if (!dead) {
+        if (*reinterpret_cast<volatile int*>(&misc[0]) != 0 ||
+            !mbar_wait_bounded(&full[stage], par, kWaitLimitNs)) {
+          dead = true;
+          if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
+        }
+      }
+      if (!dead) {
+        uint8_t* sb = smem + stage * C::STAGE_BYTES;
+        const int64_t row0 = (int64_t)walk.b * p.max_seq + walk.t0;
+        const int soff = (int)((row0 * C::SROW) & 15);
+        const int nv = (int)min((int64_t)T_TILE, walk.seg_hi - walk.t0);
+        const uint32_t sc = smem_u32(sb + C::OFF_SC32);
+#pragma unroll 1
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t raw = smem_u32(sb + 2 * C::CODE_BYTES + kv * C::SCALE_SLAB + soff);
+          const uint32_t dst = sc + kv * C::SC_KV * 4;
+#pragma unroll 2
+          for (int i = lane; i < T_TILE * HKV; i += 32) {
+            const int t = i / HKV, hh = i % HKV;
+            const int u = t / UNIT, tau = t % UNIT;
+            const int nt = tau >> 3, tg = (tau & 7) >> 1, e = tau & 1;
+            const uint32_t d0 = dst + 4 * (hh * C::SC_HEAD + (u * NG * 4 + tg) * (2 * NT) + nt * 2 + e);
+            const bool ok = t < nv;
+            if constexpr (NG % 4 == 0) {
+              if ((soff & 7) == 0) {
+#pragma unroll
+                for (int g4 = 0; g4 < NG; g4 += 4) {
+                  const uint2 w = lds_u2(raw + i * NG * 2 + g4 * 2);
+                  const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+                  const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+                  sts_f32(d0 + 4 * ((g4 + 0) * 4 * 2 * NT), ok ? f01.x : 0.f);
+                  sts_f32(d0 + 4 * ((g4 + 1) * 4 * 2 * NT), ok ? f01.y : 0.f);
+                  sts_f32(d0 + 4 * ((g4 + 2) * 4 * 2 * NT), ok ? f23.x : 0.f);
+                  sts_f32(d0 + 4 * ((g4 + 3) * 4 * 2 * NT), ok ? f23.y : 0.f);
+                }
+                continue;
+              }
+            }
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              const uint32_t hb = lds_u16(raw + i * NG * 2 + g * 2);
+              sts_f32(d0 + 4 * (g * 4 * 2 * NT), ok ? __half2float(__ushort_as_half((unsigned short)hb)) : 0.f);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ready[tile_i % STAGES]);
+        mbar_arrive(&empty[tile_i % STAGES]);
+      }
+    }
     return;
   }
 
@@ -262,6 +350,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = p.group;
   float* scratch = reinterpret_cast<float*>(smem + C::OFF_SCRATCH + warp * C::SCRATCH);
   const uint32_t smem_base = smem_u32(smem);
+
+  // Per-lane ldmatrix offsets inside a head's [tile][D/2] block, relative to the
+  // unit's first row. A unit spans UNIT * RB bytes (a multiple of 1024 B, as is a
+  // head block), so the swizzle phase of a row only depends on its row inside
+  // the unit. K batch k covers matrices m = 4k..4k+3, m = (group m / NT,
+  // n-tile m % NT); V batch k the same with token blocks instead of n-tiles.
+  constexpr int NB = NG * NT / 4;
+  uint32_t k_off[NB], v_off[NB];
+  {
+    const int rr = lane & 7, mi = lane >> 3;
+#pragma unroll
+    for (int kb = 0; kb < NB; ++kb) {
+      const int m = 4 * kb + mi;
+      const int row = (m % NT) * 8 + rr;
+      const int grp = m / NT;
+      const int swz = ((h * T_TILE * RB + row * RB) >> 7) & C::SWZ;
+      k_off[kb] = (uint32_t)(row * RB + ((grp ^ swz) << 4));
+      v_off[kb] = k_off[kb];
+    }
+  }
+  static_assert((UNIT * RB) % 1024 == 0 || C::SWZ == 0 || (UNIT * RB) % ((C::SWZ + 1) * 128) == 0,
+                "unit rows must keep the swizzle phase");
 
   uint32_t qA[NG][2][4];
   float biasK[NG];
@@ -341,11 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       f_h = __int_as_float((127 + 24 - sh) << 23);  // 2^(24 - sh): MMA units -> log2 units
       __syncwarp();
 #pragma unroll
-      for (int g = 0; g < NG; ++g)
+      for (int g = 0; g < NG; ++g) {
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) acc[g][jj][r] = 0.f;
+        for (int r = 0; r < 4; ++r) {
+          acc[g][0][r] = 0.f;
+          acc[g][1][r] = 0.f;
+        }
+      }
       m_run = -INFINITY;
       l_run = 0.f;
     }
@@ -353,11 +465,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- token tiles of this segment
     bool seg_end = false;
     while (!seg_end) {
-      const int stage = tile_i % kStages;
-      const uint32_t par = (uint32_t)((tile_i / kStages) & 1);
+      const int stage = tile_i % STAGES;
+      const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
       if (!dead) {
         if (*reinterpret_cast<volatile int*>(&misc[0]) != 0 ||
-            !mbar_wait_bounded(&full[stage], par, kWaitLimitNs)) {
+            !mbar_wait_bounded(&full[stage], par, kWaitLimitNs) ||
+            !mbar_wait_bounded(&ready[stage], par, kWaitLimitNs)) {
           dead = true;
           if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
         }
@@ -366,168 +479,134 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sbase = smem_base + stage * C::STAGE_BYTES;
         const uint32_t kc = sbase + h * T_TILE * RB;
         const uint32_t vc = sbase + C::CODE_BYTES + h * T_TILE * RB;
-        const int64_t row0 = (int64_t)b * p.max_seq + walk.t0;
-        const int soff = (int)((row0 * C::SROW) & 15);
-        const uint8_t* ksr = smem + stage * C::STAGE_BYTES + 2 * C::CODE_BYTES + soff;
-        const uint8_t* vsr = ksr + C::SCALE_SLAB;
+        const uint32_t sck = sbase + C::OFF_SC32 + 4 * h * C::SC_HEAD;
+        const uint32_t scv = sck + 4 * C::SC_KV;
 #pragma unroll 1
         for (int u = 0; u < UPW; ++u) {
-          const int r0 = (sub * UPW + u) * 16;  // first tile row of this unit
+          const int uu = sub * UPW + u;  // unit index within the tile
+          const int r0 = uu * UNIT;      // first tile row of this unit
           const int64_t tok0 = walk.t0 + r0;
           if (tok0 >= seg_hi) break;
-          const int nv = (int)min((int64_t)16, seg_hi - tok0);
+          const int nv = (int)min((int64_t)UNIT, seg_hi - tok0);
 
-          // --- K and V code fragments
-          uint32_t kw[2][NG], vw[NG][2];
-          {
-            const int rr = lane & 7, mi = lane >> 3;
-            if constexpr (NG == 1) {
-              uint32_t t2[2];
-              const int row = r0 + (mi & 1) * 8 + rr;
-              ldmatrix_x2(t2, kc + row * RB);
-              kw[0][0] = t2[0];
-              kw[1][0] = t2[1];
-              ldmatrix_x2_trans(t2, vc + row * RB);
-              vw[0][0] = t2[0];
-              vw[0][1] = t2[1];
-            } else {
+          // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
+          float2 s2[NT];
 #pragma unroll
-              for (int m4 = 0; m4 < 2 * NG; m4 += 4) {
-                const int m = m4 + mi;
-                {  // K: matrix m = (n-tile m / NG, group m % NG)
-                  const int row = r0 + (m / NG) * 8 + rr;
-                  const int grp = m % NG;
-                  const int roff = (h * T_TILE + row) * RB;
-                  const uint32_t addr = kc + row * RB + ((grp ^ ((roff >> 7) & C::SWZ)) << 4);
-                  uint32_t t4[4];
-                  ldmatrix_x4(t4, addr);
+          for (int nt = 0; nt < NT; ++nt) s2[nt] = make_float2(0.f, 0.f);
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) kw[(m4 + i) / NG][(m4 + i) % NG] = t4[i];
-                }
-                {  // V: matrix m = (group m / 2, token half m % 2)
-                  const int row = r0 + (m & 1) * 8 + rr;
-                  const int grp = m >> 1;
-                  const int roff = (h * T_TILE + row) * RB;
-                  const uint32_t addr = vc + row * RB + ((grp ^ ((roff >> 7) & C::SWZ)) << 4);
-                  uint32_t t4[4];
-                  ldmatrix_x4_trans(t4, addr);
+          for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+            uint32_t kw[4];
+            ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
+            // this lane's K scales for the groups of this batch: (n-tile, e) pairs
+            float skv[4 / NT > 0 ? 4 / NT : 1][2 * NT];
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) vw[(m4 + i) >> 1][(m4 + i) & 1] = t4[i];
-                }
+            for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
+              const int g = g4 / NT + gi;
+              const uint32_t a0 = sck + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT));
+#pragma unroll
+              for (int q4 = 0; q4 < 2 * NT; q4 += 4) {
+                const float4 v = lds_f4(a0 + 4 * q4);
+                skv[gi][q4] = v.x;
+                skv[gi][q4 + 1] = v.y;
+                skv[gi][q4 + 2] = v.z;
+                skv[gi][q4 + 3] = v.w;
               }
             }
-          }
-
-          // --- binary16 scales of this unit -> binary32 (masked tokens -> 0)
-          float* sc = scratch;  // [2][16][NG]
-          {
-            constexpr int HPL = NG >= 2 ? NG / 2 : 1;      // halves per lane
-            constexpr int LPT = NG / HPL;                  // lanes per token
-            constexpr int USED = 16 * LPT;
-            if (lane < USED) {
-              const int tk = lane / LPT, first = (lane % LPT) * HPL;
-              const int so = ((r0 + tk) * HKV + h) * NG * 2 + first * 2;
 #pragma unroll
-              for (int i = 0; i < HPL; ++i) {
-                const bool ok = tk < nv;
-                const float sk = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(ksr + so + 2 * i)));
-                const float sv = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(vsr + so + 2 * i)));
-                sc[tk * NG + first + i] = ok ? sk : 0.f;
-                sc[16 * NG + tk * NG + first + i] = ok ? sv : 0.f;
-              }
-            }
-          }
-          __syncwarp();
-
-          // --- scores S[head gid][token] for tokens nt*8 + 2*tig + e
-          float s[2][2];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            s[nt][0] = 0.f;
-            s[nt][1] = 0.f;
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-              float c[4] = {biasK[g], biasK[g], 0.f, 0.f};
-              const uint32_t w = kw[nt][g];
-              mma_f16_16816(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u));
+            for (int i = 0; i < 4; ++i) {
+              const int g = (g4 + i) / NT, nt = (g4 + i) % NT;
+              const int gi = g - g4 / NT;
+              const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
+              float c[4];
+              const uint32_t w = kw[i];
+              mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
+                              biasK[g], biasK[g], 0.f, 0.f);
               const uint32_t w8 = w >> 8;
-              mma_f16_16816(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u), and_xor(w8, 0x00F000F0u, 0x00800080u));
-              const int t0i = nt * 8 + 2 * tig;
-              s[nt][0] = fmaf(sc[t0i * NG + g], c[0] + c[2], s[nt][0]);
-              s[nt][1] = fmaf(sc[(t0i + 1) * NG + g], c[1] + c[3], s[nt][1]);
+              mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
+                                and_xor(w8, 0x00F000F0u, 0x00800080u));
+              const float2 x = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
+              s2[nt] = __ffma2_rn(sk, x, s2[nt]);
             }
+          }
+          if (nv < UNIT) {
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-              if (nt * 8 + 2 * tig + e >= nv) s[nt][e] = -INFINITY;
+            for (int nt = 0; nt < NT; ++nt) {
+              if (nt * 8 + 2 * tig >= nv) s2[nt].x = -INFINITY;
+              if (nt * 8 + 2 * tig + 1 >= nv) s2[nt].y = -INFINITY;
+            }
           }
 
-          // --- online softmax (head gid; quad lanes share a head)
-          float mx = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+          // --- online softmax (head gid; the quad's lanes share a head)
+          float mx = fmaxf(s2[0].x, s2[0].y);
+#pragma unroll
+          for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s2[nt].x, s2[nt].y));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
           const float m_new = fmaxf(m_run, mx);
           const bool grow = m_new > m_run;
           if (__any_sync(0xffffffffu, grow)) {
-            const float corr = grow ? ((m_run == -INFINITY) ? 0.f : exp2f((m_run - m_new) * f_h)) : 1.f;
+            const float corr = grow ? ((m_run == -INFINITY) ? 0.f : ex2_approx((m_run - m_new) * f_h)) : 1.f;
             l_run *= corr;
-            const float c0 = __shfl_sync(0xffffffffu, corr, 8 * tig);
-            const float c1 = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
+            const float2 cc = make_float2(__shfl_sync(0xffffffffu, corr, 8 * tig),
+                                          __shfl_sync(0xffffffffu, corr, 8 * tig + 4));
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
+            for (int g = 0; g < NG; ++g) {
 #pragma unroll
               for (int jj = 0; jj < 2; ++jj) {
-                acc[g][jj][0] *= c0;
-                acc[g][jj][1] *= c1;
-                acc[g][jj][2] *= c0;
-                acc[g][jj][3] *= c1;
+                float2 a01 = __fmul2_rn(make_float2(acc[g][jj][0], acc[g][jj][1]), cc);
+                float2 a23 = __fmul2_rn(make_float2(acc[g][jj][2], acc[g][jj][3]), cc);
+                acc[g][jj][0] = a01.x;
+                acc[g][jj][1] = a01.y;
+                acc[g][jj][2] = a23.x;
+                acc[g][jj][3] = a23.y;
               }
+            }
             m_run = m_new;
           }
           const float mb = (m_run == -INFINITY) ? 0.f : m_run * f_h;
-          float pr[2][2];
+          float2 p2[NT];
+          float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              pr[nt][e] = exp2f(fmaf(s[nt][e], f_h, -mb));
-              l_run += pr[nt][e];
-            }
+          for (int nt = 0; nt < NT; ++nt) {
+            const float2 z = __ffma2_rn(s2[nt], make_float2(f_h, f_h), make_float2(-mb, -mb));
+            p2[nt] = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+            lsum = __fadd2_rn(lsum, p2[nt]);
+          }
+          l_run += lsum.x + lsum.y;
 
-          // --- P.V: acc[d][head] += sum_t v[t][d] * (p[t] * sigmaV[t][g])
-          const float* sv = sc + 16 * NG;
-          const uint32_t K8 = 0x00080008u;       // binary16 pair (8 * 2^-24, 8 * 2^-24)
-          const uint32_t NEG8 = 0x80088008u;     // (-8 * 2^-24, -8 * 2^-24)
-          const uint32_t SIXTEENTH = 0x2C002C00u;  // (1/16, 1/16)
+          // --- P.V: acc[d][head] += sum_t (c_t,d * 2^-24) * (p_t * sigmaV_t,g). The signed code
+          //     enters exactly: u = code + 8 from the lop3, then one binary16 subtract per pair
+          //     (8 * 2^-24 at the low nibble position, 128 * 2^-24 = 16 * 8 * 2^-24 at the high
+          //     one, whose rows therefore carry x16). A biased offset must not reach the
+          //     accumulator: the tensor core rounds its fp32 sums toward zero, so an all-positive
+          //     operand would drift over a long context.
+          const __half2 k8 = __ushort_as_half2_pair(0x0008u);
+          const __half2 k128 = __ushort_as_half2_pair(0x0080u);
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            const int t0i = 2 * tig;
-            const uint32_t b0 = pack_half2(pr[0][0] * sv[t0i * NG + g], pr[0][1] * sv[(t0i + 1) * NG + g]);
-            const uint32_t b1 = pack_half2(pr[1][0] * sv[(t0i + 8) * NG + g], pr[1][1] * sv[(t0i + 9) * NG + g]);
+          for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+            uint32_t vw[4];
+            ldmatrix_x4_trans(vw, vc + r0 * RB + v_off[g4 / 4]);
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const uint32_t va = jj ? (vw[g][0] >> 8) : vw[g][0];
-              const uint32_t vb = jj ? (vw[g][1] >> 8) : vw[g][1];
-              uint32_t a[4];
-              const uint32_t lo_a = and_xor(va, 0x000F000Fu, K8);
-              const uint32_t hi_a = and_xor(va, 0x00F000F0u, 0x00800080u);
-              const uint32_t lo_b = and_xor(vb, 0x000F000Fu, K8);
-              const uint32_t hi_b = and_xor(vb, 0x00F000F0u, 0x00800080u);
-              const __half2 k8 = *reinterpret_cast<const __half2*>(&K8);
-              const __half2 n8 = *reinterpret_cast<const __half2*>(&NEG8);
-              const __half2 s16 = *reinterpret_cast<const __half2*>(&SIXTEENTH);
-              __half2 r;
-              r = __hsub2(*reinterpret_cast<const __half2*>(&lo_a), k8);
-              a[0] = *reinterpret_cast<uint32_t*>(&r);
-              r = __hfma2(*reinterpret_cast<const __half2*>(&hi_a), s16, n8);
-              a[1] = *reinterpret_cast<uint32_t*>(&r);
-              r = __hsub2(*reinterpret_cast<const __half2*>(&lo_b), k8);
-              a[2] = *reinterpret_cast<uint32_t*>(&r);
-              r = __hfma2(*reinterpret_cast<const __half2*>(&hi_b), s16, n8);
-              a[3] = *reinterpret_cast<uint32_t*>(&r);
-              mma_f16_16816(acc[g][jj], a, b0, b1);
+            for (int i = 0; i < 4; i += 2) {
+              const int g = (g4 + i) / NT, tb = (g4 + i) % NT;  // token blocks tb, tb + 1 = one k-step
+              const int ks = tb >> 1;
+              const float4 sv = lds_f4(scv + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT) + ks * 4));
+              const uint32_t b0 = pack_half2_f2(__fmul2_rn(p2[2 * ks], make_float2(sv.x, sv.y)));
+              const uint32_t b1 = pack_half2_f2(__fmul2_rn(p2[2 * ks + 1], make_float2(sv.z, sv.w)));
+              const uint32_t va = vw[i], vb = vw[i + 1];
+#pragma unroll
+              for (int jj = 0; jj < 2; ++jj) {
+                const uint32_t xa = jj ? (va >> 8) : va, xb = jj ? (vb >> 8) : vb;
+                uint32_t a[4];
+                a[0] = h2_sub_u32(and_xor(xa, 0x000F000Fu, 0x00080008u), k8);
+                a[1] = h2_sub_u32(and_xor(xa, 0x00F000F0u, 0x00800080u), k128);
+                a[2] = h2_sub_u32(and_xor(xb, 0x000F000Fu, 0x00080008u), k8);
+                a[3] = h2_sub_u32(and_xor(xb, 0x00F000F0u, 0x00800080u), k128);
+                mma_f16_16816_acc(acc[g][jj], a, b0, b1);
+              }
             }
           }
-          __syncwarp();  // scale scratch is rewritten by the next unit
+          (void)KSP;
         }
       }
       __syncwarp();
@@ -543,6 +622,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
     const float m_real = (m_run == -INFINITY) ? -INFINITY : m_run * f_h;
     constexpr float kTwo24 = 16777216.f;
+    // rotated-domain accumulator of head 2*tig + e at d = 32g + 4*gid + {0, 1, 2, 3};
+    // rows of the high nibble position carry x16.
+    auto final4 = [&](int g, int e) {
+      return make_float4(acc[g][0][e] * kTwo24, acc[g][0][2 + e] * (0.0625f * kTwo24), acc[g][1][e] * kTwo24,
+                         acc[g][1][2 + e] * (0.0625f * kTwo24));
+    };
     if constexpr (C::WPH == 1) {
       if (!dead) {
         if (tig == 0 && gid < G) {
@@ -556,10 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (hh < G) {
             float* dst = p.ws_acc + ((int64_t)slot * p.n_q + h * G + hh) * D;
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
-              *reinterpret_cast<float4*>(dst + 32 * g + 4 * gid) =
-                  make_float4(acc[g][0][e] * kTwo24, acc[g][0][2 + e] * kTwo24, acc[g][1][e] * kTwo24,
-                              acc[g][1][2 + e] * kTwo24);
+            for (int g = 0; g < NG; ++g) *reinterpret_cast<float4*>(dst + 32 * g + 4 * gid) = final4(g, e);
           }
         }
       }
@@ -576,14 +658,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < NG; ++g)
           *reinterpret_cast<float4*>(scratch + hh * D + 32 * g + 4 * gid) =
-              dead ? make_float4(0.f, 0.f, 0.f, 0.f)
-                   : make_float4(acc[g][0][e] * kTwo24, acc[g][0][2 + e] * kTwo24, acc[g][1][e] * kTwo24,
-                                 acc[g][1][2 + e] * kTwo24);
+              dead ? make_float4(0.f, 0.f, 0.f, 0.f) : final4(g, e);
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
-      const int ctid = tid;  // 0 .. 255
       const int items = HKV * G * D;
-      for (int it = ctid; it < items; it += kConsumerWarps * 32) {
+      for (int it = tid; it < items; it += kConsumerWarps * 32) {
         const int hk = it / (G * D), j = (it / D) % G, d = it % D;
         float mstar = -INFINITY;
         for (int sb = 0; sb < C::WPH; ++sb) {
@@ -615,14 +694,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combine the partials of one (sequence, q head), normalise, inverse SRHT.
+// Phase 1 stages every partial's weight 2^(m_c - m*) in shared memory; phase 2
+// streams the accumulators with independent loads per thread.
 template <int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NG = D / 32;
   constexpr int F4 = D / 4;            // float4 columns
-  constexpr int PH = 128 / F4;         // slot phases
-  __shared__ float red[128];
+  constexpr int PH = 256 / F4;         // slot phases
+  constexpr int MAX_SLOTS = 1024 + kMaxBatch;
+  __shared__ float wts[MAX_SLOTS];
+  __shared__ float red[256];
   __shared__ __align__(16) float accs[PH][D];
-  __shared__ float bc[2];
   const int tid = threadIdx.x;
   const int b = blockIdx.x / p.n_q, hq = blockIdx.x % p.n_q;
   const int64_t* hdr = ws_header(p.ws_ml);
@@ -630,60 +712,64 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
   if (P1 <= P0) {  // empty sequence
-    for (int d = tid; d < D; d += 128) out[d] = 0.f;
+    for (int d = tid; d < D; d += 256) out[d] = 0.f;
     return;
   }
   const int c0 = (int)(P0 / R), c1 = (int)((P1 - 1) / R);
-  const int ns = c1 - c0 + 1;
-  // pass 1: global max
+  const int ns = min(c1 - c0 + 1, MAX_SLOTS);
+  // phase 1: max of the running maxima, then weights and the weighted sum of l
   float m = -INFINITY;
-  for (int i = tid; i < ns; i += 128) m = fmaxf(m, ml[((int64_t)(b + c0 + i) * p.n_q + hq) * 2]);
+  for (int i = tid; i < ns; i += 256) {
+    const float mi = ml[((int64_t)(b + c0 + i) * p.n_q + hq) * 2];
+    wts[i] = mi;
+    m = fmaxf(m, mi);
+  }
   red[tid] = m;
   __syncthreads();
-  for (int o = 64; o > 0; o >>= 1) {
+  for (int o = 128; o > 0; o >>= 1) {
     if (tid < o) red[tid] = fmaxf(red[tid], red[tid + o]);
     __syncthreads();
   }
   const float mstar = red[0];
   __syncthreads();
-  // pass 2: weighted sums
   float lsum = 0.f;
-  for (int i = tid; i < ns; i += 128) {
-    const float* e = ml + ((int64_t)(b + c0 + i) * p.n_q + hq) * 2;
-    if (e[0] != -INFINITY) lsum += exp2f(e[0] - mstar) * e[1];
+  for (int i = tid; i < ns; i += 256) {
+    const float mi = wts[i];
+    const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - mstar);
+    wts[i] = w;
+    lsum += w * ml[((int64_t)(b + c0 + i) * p.n_q + hq) * 2 + 1];
   }
   red[tid] = lsum;
-  const int col = tid % F4, ph = tid / F4;
-  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (ph < PH) {
-    for (int i = ph; i < ns; i += PH) {
-      const int64_t qh = (int64_t)(b + c0 + i) * p.n_q + hq;
-      const float mw = ml[qh * 2];
-      if (mw == -INFINITY) continue;
-      const float w = exp2f(mw - mstar);
-      const float4 v = reinterpret_cast<const float4*>(p.ws_acc + qh * D)[col];
-      a.x = fmaf(w, v.x, a.x);
-      a.y = fmaf(w, v.y, a.y);
-      a.z = fmaf(w, v.z, a.z);
-      a.w = fmaf(w, v.w, a.w);
-    }
-    reinterpret_cast<float4*>(accs[ph])[col] = a;
-  }
   __syncthreads();
-  for (int o = 64; o > 0; o >>= 1) {
+  for (int o = 128; o > 0; o >>= 1) {
     if (tid < o) red[tid] += red[tid + o];
     __syncthreads();
   }
-  if (tid == 0) bc[0] = red[0];
+  const float L = red[0];
+  // phase 2: weighted accumulator sums, PH slot phases x F4 float4 columns
+  const int col = tid % F4, ph = tid / F4;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* base = reinterpret_cast<const float4*>(p.ws_acc) + ((int64_t)(b + c0) * p.n_q + hq) * F4 + col;
+  const int64_t stride = (int64_t)p.n_q * F4;
+#pragma unroll 4
+  for (int i = ph; i < ns; i += PH) {
+    const float w = wts[i];
+    const float4 v = base[(int64_t)i * stride];
+    a.x = fmaf(w, v.x, a.x);
+    a.y = fmaf(w, v.y, a.y);
+    a.z = fmaf(w, v.z, a.z);
+    a.w = fmaf(w, v.w, a.w);
+  }
+  reinterpret_cast<float4*>(accs[ph])[col] = a;
   __syncthreads();
-  const float L = bc[0];
-  // inverse SRHT on the normalised rotated-domain output: first warp, NG lanes
+  // inverse SRHT on the normalised rotated-domain output: first warp, NG lanes per vector
   if (tid < 32) {
     const int part = tid % NG;
     float u[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float s = 0.f;
+#pragma unroll
       for (int q = 0; q < PH; ++q) s += accs[q][part * 32 + i];
       u[i] = (L > 0.f) ? s / L : 0.f;
     }
@@ -703,7 +789,7 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
   static bool attr_set = false;  // per instantiation; the attribute is per function
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16);
+                                         C::SMEM_MAX);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -716,7 +802,7 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
     e = cudaEventRecord(ev, s);
     if (e != cudaSuccess) return e;
   }
-  decode_merge_kernel<D><<<p.batch * p.n_q, 128, 0, s>>>(p);
+  decode_merge_kernel<D><<<p.batch * p.n_q, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
