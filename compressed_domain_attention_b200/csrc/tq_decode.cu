@@ -218,6 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i <= p.batch; i += kThreads) hdr[i] = prefix[i];
     if (tid == 0) hdr[p.batch + 1] = R;
   }
+  // the merge grid may be scheduled from here on; it waits for this grid's completion
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t lo = (int64_t)blockIdx.x * R;
   const int64_t hi = min(lo + R, T_sum);
   if (lo >= hi) return;
@@ -282,6 +284,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ converter
     // binary16 scale rows [token][head][group] -> fp32 [head][unit][group][tig][n-tile][e],
     // the order in which a consumer lane reads them; tokens past the segment end get 0.
+    // Lane work item k covers the token pair (2j, 2j + 1) of one head, j * HKV + hh =
+    // lane + 32k: both tokens land next to each other (e = 0, 1), so each group is
+    // one 8-byte store. The shared-memory offsets are the same for every tile.
+    constexpr int PAIRS = T_TILE / 2 * HKV;
+    constexpr int ITEMS = (PAIRS + 31) / 32;
+    uint32_t src_off[ITEMS], dst_off[ITEMS];
+    int tok_of[ITEMS];
+#pragma unroll
+    for (int k = 0; k < ITEMS; ++k) {
+      const int i = lane + 32 * k;
+      const int j = i / HKV, hh = i % HKV;
+      const int t = 2 * j;
+      const int u = t / UNIT, tau = t % UNIT;
+      const int nt = tau >> 3, tg = (tau & 7) >> 1;
+      src_off[k] = (uint32_t)((t * HKV + hh) * NG * 2);
+      dst_off[k] = (uint32_t)(4 * (hh * C::SC_HEAD + (u * NG * 4 + tg) * (2 * NT) + nt * 2));
+      tok_of[k] = i < PAIRS ? t : 1 << 30;
+    }
     bool dead = false;
     int tile_i = 0;
     for (; !walk.done(); walk.advance<T_TILE>(), ++tile_i) {
@@ -300,36 +320,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int soff = (int)((row0 * C::SROW) & 15);
         const int nv = (int)min((int64_t)T_TILE, walk.seg_hi - walk.t0);
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
-#pragma unroll 1
+#pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
           const uint32_t raw = smem_u32(sb + 2 * C::CODE_BYTES + kv * C::SCALE_SLAB + soff);
           const uint32_t dst = sc + kv * C::SC_KV * 4;
-#pragma unroll 2
-          for (int i = lane; i < T_TILE * HKV; i += 32) {
-            const int t = i / HKV, hh = i % HKV;
-            const int u = t / UNIT, tau = t % UNIT;
-            const int nt = tau >> 3, tg = (tau & 7) >> 1, e = tau & 1;
-            const uint32_t d0 = dst + 4 * (hh * C::SC_HEAD + (u * NG * 4 + tg) * (2 * NT) + nt * 2 + e);
-            const bool ok = t < nv;
-            if constexpr (NG % 4 == 0) {
-              if ((soff & 7) == 0) {
 #pragma unroll
-                for (int g4 = 0; g4 < NG; g4 += 4) {
-                  const uint2 w = lds_u2(raw + i * NG * 2 + g4 * 2);
-                  const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
-                  const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
-                  sts_f32(d0 + 4 * ((g4 + 0) * 4 * 2 * NT), ok ? f01.x : 0.f);
-                  sts_f32(d0 + 4 * ((g4 + 1) * 4 * 2 * NT), ok ? f01.y : 0.f);
-                  sts_f32(d0 + 4 * ((g4 + 2) * 4 * 2 * NT), ok ? f23.x : 0.f);
-                  sts_f32(d0 + 4 * ((g4 + 3) * 4 * 2 * NT), ok ? f23.y : 0.f);
-                }
-                continue;
-              }
-            }
+          for (int k = 0; k < ITEMS; ++k) {
+            const int t = tok_of[k];
+            if (t >= T_TILE) continue;
+            const bool ok0 = t < nv, ok1 = t + 1 < nv;
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
-              const uint32_t hb = lds_u16(raw + i * NG * 2 + g * 2);
-              sts_f32(d0 + 4 * (g * 4 * 2 * NT), ok ? __half2float(__ushort_as_half((unsigned short)hb)) : 0.f);
+              const uint32_t h0 = lds_u16(raw + src_off[k] + g * 2);
+              const uint32_t h1 = lds_u16(raw + src_off[k] + HKV * NG * 2 + g * 2);
+              const float f0 = ok0 ? __half2float(__ushort_as_half((unsigned short)h0)) : 0.f;
+              const float f1 = ok1 ? __half2float(__ushort_as_half((unsigned short)h1)) : 0.f;
+              sts_f2(dst + dst_off[k] + 4 * (g * 4 * 2 * NT), f0, f1);
             }
           }
         }
@@ -490,9 +496,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nv = (int)min((int64_t)UNIT, seg_hi - tok0);
 
           // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
-          float2 s2[NT];
+          float2 s2[NT], s2b[NT];  // even and odd groups: two independent chains
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) s2[nt] = make_float2(0.f, 0.f);
+          for (int nt = 0; nt < NT; ++nt) {
+            s2[nt] = make_float2(0.f, 0.f);
+            s2b[nt] = make_float2(0.f, 0.f);
+          }
 #pragma unroll
           for (int g4 = 0; g4 < NG * NT; g4 += 4) {
             uint32_t kw[4];
@@ -525,9 +534,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
                                 and_xor(w8, 0x00F000F0u, 0x00800080u));
               const float2 x = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
-              s2[nt] = __ffma2_rn(sk, x, s2[nt]);
+              if (g & 1)
+                s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
+              else
+                s2[nt] = __ffma2_rn(sk, x, s2[nt]);
             }
           }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) s2[nt] = __fadd2_rn(s2[nt], s2b[nt]);
           if (nv < UNIT) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -694,18 +708,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combine the partials of one (sequence, q head), normalise, inverse SRHT.
-// Phase 1 stages every partial's weight 2^(m_c - m*) in shared memory; phase 2
-// streams the accumulators with independent loads per thread.
+// Launched as a programmatic dependent of the split-K kernel: blocks may start
+// early and wait at griddepcontrol.wait until every split-K block has finished
+// and its writes are visible. Phase 1 stages the weights 2^(m_c - m*) of all
+// partials in shared memory; phase 2 streams the accumulators with PF
+// independent loads in flight per thread.
 template <int D>
 __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NG = D / 32;
   constexpr int F4 = D / 4;            // float4 columns
   constexpr int PH = 256 / F4;         // slot phases
+  constexpr int PF = 24;               // loads in flight per thread
   constexpr int MAX_SLOTS = 1024 + kMaxBatch;
   __shared__ float wts[MAX_SLOTS];
-  __shared__ float red[256];
+  __shared__ float lsv[MAX_SLOTS];
+  __shared__ float red[8];
   __shared__ __align__(16) float accs[PH][D];
-  const int tid = threadIdx.x;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   const int b = blockIdx.x / p.n_q, hq = blockIdx.x % p.n_q;
   const int64_t* hdr = ws_header(p.ws_ml);
   const int64_t P0 = hdr[b], P1 = hdr[b + 1], R = hdr[p.batch + 1];
@@ -717,62 +737,84 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   }
   const int c0 = (int)(P0 / R), c1 = (int)((P1 - 1) / R);
   const int ns = min(c1 - c0 + 1, MAX_SLOTS);
-  // phase 1: max of the running maxima, then weights and the weighted sum of l
+  const float* mlb = ml + ((int64_t)(b + c0) * p.n_q + hq) * 2;
+  const int64_t mls = (int64_t)p.n_q * 2;
+  const int col = tid % F4, ph = tid / F4;
+  const float4* base = reinterpret_cast<const float4*>(p.ws_acc) + ((int64_t)(b + c0) * p.n_q + hq) * F4 + col;
+  const int64_t stride = (int64_t)p.n_q * F4;
+  // The accumulator loads of the first chunk do not depend on the weights: issue them
+  // together with the (m, l) loads, so the merge costs about one memory round trip.
+  float4 v[PF];
+#pragma unroll
+  for (int k = 0; k < PF; ++k) {
+    const int i = ph + k * PH;
+    v[k] = i < ns ? __ldcg(base + (int64_t)i * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l
   float m = -INFINITY;
   for (int i = tid; i < ns; i += 256) {
-    const float mi = ml[((int64_t)(b + c0 + i) * p.n_q + hq) * 2];
-    wts[i] = mi;
-    m = fmaxf(m, mi);
+    const float2 e = __ldcg(reinterpret_cast<const float2*>(mlb + i * mls));
+    wts[i] = e.x;
+    lsv[i] = e.y;
+    m = fmaxf(m, e.x);
   }
-  red[tid] = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[wp] = m;
   __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (tid < o) red[tid] = fmaxf(red[tid], red[tid + o]);
-    __syncthreads();
-  }
-  const float mstar = red[0];
-  __syncthreads();
+  float mstar = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) mstar = fmaxf(mstar, red[w]);
   float lsum = 0.f;
   for (int i = tid; i < ns; i += 256) {
     const float mi = wts[i];
     const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - mstar);
     wts[i] = w;
-    lsum += w * ml[((int64_t)(b + c0 + i) * p.n_q + hq) * 2 + 1];
+    lsum += w * lsv[i];
   }
-  red[tid] = lsum;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  __syncthreads();  // red[] reused, wts[] complete
+  if (lane == 0) red[wp] = lsum;
   __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (tid < o) red[tid] += red[tid + o];
-    __syncthreads();
-  }
-  const float L = red[0];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) L += red[w];
   // phase 2: weighted accumulator sums, PH slot phases x F4 float4 columns
-  const int col = tid % F4, ph = tid / F4;
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* base = reinterpret_cast<const float4*>(p.ws_acc) + ((int64_t)(b + c0) * p.n_q + hq) * F4 + col;
-  const int64_t stride = (int64_t)p.n_q * F4;
-#pragma unroll 4
-  for (int i = ph; i < ns; i += PH) {
-    const float w = wts[i];
-    const float4 v = base[(int64_t)i * stride];
-    a.x = fmaf(w, v.x, a.x);
-    a.y = fmaf(w, v.y, a.y);
-    a.z = fmaf(w, v.z, a.z);
-    a.w = fmaf(w, v.w, a.w);
+  for (int i0 = ph;; i0 += PH * PF) {
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int i = i0 + k * PH;
+      const float w = i < ns ? wts[i] : 0.f;
+      a.x = fmaf(w, v[k].x, a.x);
+      a.y = fmaf(w, v[k].y, a.y);
+      a.z = fmaf(w, v[k].z, a.z);
+      a.w = fmaf(w, v[k].w, a.w);
+    }
+    if (i0 + PH * PF >= ns) break;
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int i = i0 + PH * PF + k * PH;
+      v[k] = i < ns ? __ldcg(base + (int64_t)i * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   reinterpret_cast<float4*>(accs[ph])[col] = a;
   __syncthreads();
-  // inverse SRHT on the normalised rotated-domain output: first warp, NG lanes per vector
+  // sum the slot phases per channel and normalise (D threads), then the inverse SRHT
+  const float inv_l = (L > 0.f) ? 1.f / L : 0.f;
+  if (tid < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < PH; ++q) sum += accs[q][tid];
+    lsv[tid] = sum * inv_l;  // lsv[] is free again: reused for the normalised vector
+  }
+  __syncthreads();
   if (tid < 32) {
     const int part = tid % NG;
     float u[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < PH; ++q) s += accs[q][part * 32 + i];
-      u[i] = (L > 0.f) ? s / L : 0.f;
-    }
+    for (int i = 0; i < 32; ++i) u[i] = lsv[part * 32 + i];
     fwht_group<NG>(u, part);
     if (tid < NG) {
 #pragma unroll
@@ -798,12 +840,25 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
   decode_split_kernel<D, HKV><<<p.grid, kThreads, smem, s>>>(p, kmap, vmap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (ev != nullptr) {
+  if (ev != nullptr) {  // timing split: plain stream order between the two kernels
     e = cudaEventRecord(ev, s);
     if (e != cudaSuccess) return e;
+    decode_merge_kernel<D><<<p.batch * p.n_q, 256, 0, s>>>(p);
+    return cudaGetLastError();
   }
-  decode_merge_kernel<D><<<p.batch * p.n_q, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the merge grid is set up while the split-K
+  // grid drains; griddepcontrol.wait in the merge kernel orders the reads.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.batch * p.n_q));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p);
 }
 
 template <int D>
