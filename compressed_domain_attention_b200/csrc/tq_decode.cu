@@ -51,8 +51,9 @@ namespace tqk {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kProducerWarp = kConsumerWarps;       // one lane issues the copies
-constexpr int kConverterWarp = kConsumerWarps + 1;  // binary16 -> fp32 scales
-constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr int kConverterWarp = kConsumerWarps + 1;  // first of the binary16 -> fp32 scale warps
+constexpr int kConverterWarps = 3;                  // one on each scheduler without the producer
+constexpr int kThreads = (kConsumerWarps + 1 + kConverterWarps) * 32;
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every pipeline wait
 
@@ -232,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 1);
-      mbar_init(&empty[s], kConsumerWarps + 1);
+      mbar_init(&ready[s], kConverterWarps);
+      mbar_init(&empty[s], kConsumerWarps + kConverterWarps);
     }
     misc[0] = 0;
     fence_mbar_init();
@@ -280,20 +281,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  if (warp == kConverterWarp) {
-    // ------------------------------------------------------------ converter
+  if (warp >= kConverterWarp) {
+    // ------------------------------------------------------------ converters
     // binary16 scale rows [token][head][group] -> fp32 [head][unit][group][tig][n-tile][e],
     // the order in which a consumer lane reads them; tokens past the segment end get 0.
     // Lane work item k covers the token pair (2j, 2j + 1) of one head, j * HKV + hh =
     // lane + 32k: both tokens land next to each other (e = 0, 1), so each group is
     // one 8-byte store. The shared-memory offsets are the same for every tile.
+    // The kConverterWarps warps share the items of a tile.
     constexpr int PAIRS = T_TILE / 2 * HKV;
-    constexpr int ITEMS = (PAIRS + 31) / 32;
+    constexpr int ITEMS = (PAIRS + 32 * kConverterWarps - 1) / (32 * kConverterWarps);
+    const int cw = warp - kConverterWarp;
     uint32_t src_off[ITEMS], dst_off[ITEMS];
     int tok_of[ITEMS];
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
-      const int i = lane + 32 * k;
+      const int i = lane + 32 * (cw + kConverterWarps * k);
       const int j = i / HKV, hh = i % HKV;
       const int t = 2 * j;
       const int u = t / UNIT, tau = t % UNIT;
@@ -529,11 +532,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               float c[4];
               const uint32_t w = kw[i];
               mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
-                              biasK[g], biasK[g], 0.f, 0.f);
+                              0.f, 0.f, 0.f, 0.f);
               const uint32_t w8 = w >> 8;
               mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
                                 and_xor(w8, 0x00F000F0u, 0x00800080u));
-              const float2 x = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
+              // hi + lo rows, plus the offset term -8 * sum(q) of the offset-binary code
+              const float2 x = __fadd2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
+                                          make_float2(biasK[g], biasK[g]));
               if (g & 1)
                 s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
               else
