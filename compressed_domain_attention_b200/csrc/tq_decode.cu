@@ -55,6 +55,7 @@ constexpr int kConverterWarp = kConsumerWarps + 1;  // first of the binary16 -> 
 constexpr int kConverterWarps = 3;                  // one on each scheduler without the producer
 constexpr int kThreads = (kConsumerWarps + 1 + kConverterWarps) * 32;
 constexpr int kMaxBatch = 1024;
+constexpr int kMergeThreads = 128;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every pipeline wait
 
 template <int D, int HKV>
@@ -209,6 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  // Launched as a programmatic dependent of whatever kernel precedes it on the stream
+  // (typically the append): only the launch overlaps; nothing is read before this.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   block_prefix_lengths(p, prefix, prefix + (p.batch + 1));
   const int64_t T_sum = prefix[p.batch];
   int64_t R = (T_sum + p.grid - 1) / p.grid;
@@ -310,12 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; !walk.done(); walk.advance<T_TILE>(), ++tile_i) {
       const int stage = tile_i % STAGES;
       const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
-      if (!dead) {
-        if (*reinterpret_cast<volatile int*>(&misc[0]) != 0 ||
-            !mbar_wait_bounded(&full[stage], par, kWaitLimitNs)) {
-          dead = true;
-          if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
-        }
+      // (a producer that gave up issues nothing more: these waits then run out)
+      if (!dead && !mbar_wait_bounded(&full[stage], par, kWaitLimitNs)) {
+        dead = true;
+        if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
       }
       if (!dead) {
         uint8_t* sb = smem + stage * C::STAGE_BYTES;
@@ -477,8 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = tile_i % STAGES;
       const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
       if (!dead) {
-        if (*reinterpret_cast<volatile int*>(&misc[0]) != 0 ||
-            !mbar_wait_bounded(&full[stage], par, kWaitLimitNs) ||
+        if (!mbar_wait_bounded(&full[stage], par, kWaitLimitNs) ||
             !mbar_wait_bounded(&ready[stage], par, kWaitLimitNs)) {
           dead = true;
           if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
@@ -490,13 +491,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vc = sbase + C::CODE_BYTES + h * T_TILE * RB;
         const uint32_t sck = sbase + C::OFF_SC32 + 4 * h * C::SC_HEAD;
         const uint32_t scv = sck + 4 * C::SC_KV;
+        // tokens of the segment left in this tile, from this warp's first row on
+        const int left = (int)min((int64_t)T_TILE, seg_hi - walk.t0) - sub * UPW * UNIT;
 #pragma unroll 1
         for (int u = 0; u < UPW; ++u) {
           const int uu = sub * UPW + u;  // unit index within the tile
           const int r0 = uu * UNIT;      // first tile row of this unit
-          const int64_t tok0 = walk.t0 + r0;
-          if (tok0 >= seg_hi) break;
-          const int nv = (int)min((int64_t)UNIT, seg_hi - tok0);
+          if (u * UNIT >= left) break;
+          const int nv = min(UNIT, left - u * UNIT);
 
           // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
           float2 s2[NT], s2b[NT];  // even and odd groups: two independent chains
@@ -719,15 +721,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // partials in shared memory; phase 2 streams the accumulators with PF
 // independent loads in flight per thread.
 template <int D>
-__global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NG = D / 32;
   constexpr int F4 = D / 4;            // float4 columns
-  constexpr int PH = 256 / F4;         // slot phases
-  constexpr int PF = 24;               // loads in flight per thread
+  constexpr int PH = kMergeThreads / F4;  // slot phases
+  constexpr int PF = 8;                   // loads in flight per thread
   constexpr int MAX_SLOTS = 1024 + kMaxBatch;
   __shared__ float wts[MAX_SLOTS];
   __shared__ float lsv[MAX_SLOTS];
-  __shared__ float red[8];
+  __shared__ float red[kMergeThreads / 32];
   __shared__ __align__(16) float accs[PH][D];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
@@ -737,7 +739,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
   if (P1 <= P0) {  // empty sequence
-    for (int d = tid; d < D; d += 256) out[d] = 0.f;
+    for (int d = tid; d < D; d += kMergeThreads) out[d] = 0.f;
     return;
   }
   const int c0 = (int)(P0 / R), c1 = (int)((P1 - 1) / R);
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   }
   // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l
   float m = -INFINITY;
-  for (int i = tid; i < ns; i += 256) {
+  for (int i = tid; i < ns; i += kMergeThreads) {
     const float2 e = __ldcg(reinterpret_cast<const float2*>(mlb + i * mls));
     wts[i] = e.x;
     lsv[i] = e.y;
@@ -769,9 +771,9 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   __syncthreads();
   float mstar = red[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) mstar = fmaxf(mstar, red[w]);
+  for (int w = 1; w < kMergeThreads / 32; ++w) mstar = fmaxf(mstar, red[w]);
   float lsum = 0.f;
-  for (int i = tid; i < ns; i += 256) {
+  for (int i = tid; i < ns; i += kMergeThreads) {
     const float mi = wts[i];
     const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - mstar);
     wts[i] = w;
@@ -784,7 +786,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   __syncthreads();
   float L = 0.f;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) L += red[w];
+  for (int w = 0; w < kMergeThreads / 32; ++w) L += red[w];
   // phase 2: weighted accumulator sums, PH slot phases x F4 float4 columns
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i0 = ph;; i0 += PH * PF) {
@@ -806,13 +808,13 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
   }
   reinterpret_cast<float4*>(accs[ph])[col] = a;
   __syncthreads();
-  // sum the slot phases per channel and normalise (D threads), then the inverse SRHT
+  // sum the slot phases per channel and normalise, then the inverse SRHT
   const float inv_l = (L > 0.f) ? 1.f / L : 0.f;
-  if (tid < D) {
+  for (int d = tid; d < D; d += kMergeThreads) {
     float sum = 0.f;
 #pragma unroll
-    for (int q = 0; q < PH; ++q) sum += accs[q][tid];
-    lsv[tid] = sum * inv_l;  // lsv[] is free again: reused for the normalised vector
+    for (int q = 0; q < PH; ++q) sum += accs[q][d];
+    lsv[d] = sum * inv_l;  // lsv[] is free again: reused for the normalised vector
   }
   __syncthreads();
   if (tid < 32) {
@@ -842,20 +844,29 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
   }
   const CUtensorMap& kmap = *reinterpret_cast<const CUtensorMap*>(&km);
   const CUtensorMap& vmap = *reinterpret_cast<const CUtensorMap*>(&vm);
-  decode_split_kernel<D, HKV><<<p.grid, kThreads, smem, s>>>(p, kmap, vmap);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t kcfg = {};
+  kcfg.gridDim = dim3((unsigned)p.grid);
+  kcfg.blockDim = dim3(kThreads);
+  kcfg.dynamicSmemBytes = (size_t)smem;
+  kcfg.stream = s;
+  cudaLaunchAttribute kattr[1];
+  kattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  kattr[0].val.programmaticStreamSerializationAllowed = 1;
+  kcfg.attrs = kattr;
+  kcfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
   if (ev != nullptr) {  // timing split: plain stream order between the two kernels
     e = cudaEventRecord(ev, s);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<D><<<p.batch * p.n_q, 256, 0, s>>>(p);
+    decode_merge_kernel<D><<<p.batch * p.n_q, kMergeThreads, 0, s>>>(p);
     return cudaGetLastError();
   }
   // programmatic dependent launch: the merge grid is set up while the split-K
   // grid drains; griddepcontrol.wait in the merge kernel orders the reads.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.batch * p.n_q));
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -29,22 +29,20 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantizeParams p) 
   const int t = (int)(bt % p.n_new);
   const int b = (int)(bt / p.n_new);
 
-  int64_t pos = 0;
-  bool valid = in_range;
-  if (in_range) {
-    pos = p.start_pos[b];
-    if (pos < 0 || pos + p.n_new > p.max_seq) {
-      valid = false;
-      if (which == 0 && t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
-    }
-  }
-
+  // the input rows and the start position are independent loads: issue both first
   float u[32];
-  if (valid) {
+  int64_t pos = 0;
+  if (in_range) {
     load32(u, which ? p.v : p.k, r * D + part * 32, p.in_dtype);
+    pos = p.start_pos[b];
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) u[i] = 0.f;
+  }
+  bool valid = in_range;
+  if (in_range && (pos < 0 || pos + p.n_new > p.max_seq)) {
+    valid = false;
+    if (which == 0 && t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
   }
 #pragma unroll
   for (int i = 0; i < 32; ++i) u[i] = apply_sign(u[i], p.sign_bits, part * 32 + i);
