@@ -44,6 +44,8 @@ def parse_args(argv=None):
                     choices=["ragged_serving", "llama31_70b_long", "llama3_8b_layer", "tiny_single_head"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
+    ap.add_argument("--no-references", action="store_true",
+                    help="skip the quantise-throughput, bf16 dense-KV and dequantise-then-attend reference points")
     return ap.parse_args(argv)
 
 
@@ -274,6 +276,110 @@ def cpu_baseline(w, tensors, target_tokens):
             "seconds": round(dt, 3)}
 
 
+# ----------------------------------------------------------------------------- same-run reference points
+
+def _time_cold(fn, reps, flush, stream):
+    """Median device time (ms) of fn() with the L2 flushed (a buffer > L2 rewritten) before each rep."""
+    import torch
+    ts = []
+    for _ in range(reps):
+        flush.add_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args):
+    """Quantise throughput, the bf16 dense-KV decode and dequantise-then-attend, on this GPU and workload."""
+    import torch
+    import torch.nn.functional as F
+    from compressed_domain_attention_b200 import synthetic as syn
+    from compressed_domain_attention_b200 import tq
+    out = {}
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)  # 256 MB > 126 MB L2
+    # 1. quantise-append throughput: a 4096-token prefill of one sequence (all kv heads, K and V)
+    pw = syn.Workload("prefill_4096", 1, w.n_q_heads, w.n_kv_heads, w.head_dim, [4096], w.dtype, w.seed + 100)
+    pt = syn.generate(pw, device="cuda")
+    pl = tq.tq_cache_layout(1, 4096, w.n_kv_heads, w.n_q_heads, w.head_dim)
+    pkc, pks, pvc, pvs = tq.alloc_cache(pl, dev)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    pk, pv = pt.k[0][None].contiguous(), pt.v[0][None].contiguous()
+
+    def prefill():
+        tq.tq_quantize_append(pl, pk, pv, 4096, zero, pkc, pks, pvc, pvs, None, stream)
+
+    for _ in range(3):
+        prefill()
+    ms = _time_cold(prefill, 20, flush, stream)
+    vecs = 2 * 4096 * w.n_kv_heads
+    per_vec = w.head_dim * pk.element_size() + w.head_dim // 2 + 2 * (w.head_dim // 32)
+    out["quantize"] = {"workload": f"4096-token prefill of one sequence, {w.n_kv_heads} kv heads, K and V "
+                                   f"({vecs} vectors, {pk.dtype})".replace("torch.", ""),
+                       "ms": round(ms, 4), "vectors_per_s": round(vecs / ms * 1e3, 1),
+                       "gb_per_s": round(vecs * per_vec / ms / 1e6, 1), "l2": "flushed before each rep"}
+    del pkc, pks, pvc, pvs, pk, pv, pt
+    # 2. bf16 dense-KV decode on the same (unquantised) data: torch SDPA per sequence, in a CUDA graph
+    if w.dtype != torch.float32 and not args.no_references:
+        ks_d = [t.k[b].permute(1, 0, 2).contiguous()[None] for b in range(w.batch)]  # [1][Hkv][L][D]
+        vs_d = [t.v[b].permute(1, 0, 2).contiguous()[None] for b in range(w.batch)]
+        qd = q.view(w.batch, w.n_q_heads, 1, w.head_dim)
+        outs = [None] * w.batch
+
+        def dense():
+            for b in range(w.batch):
+                outs[b] = F.scaled_dot_product_attention(qd[b:b + 1], ks_d[b], vs_d[b], scale=w.scale,
+                                                         enable_gqa=True)
+
+        try:
+            dense()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                dense()
+            ms_d = _time_cold(g.replay, 10, flush, stream)
+            dbytes = 2 * 2 * w.head_dim * w.n_kv_heads * sum(w.seq_lens)
+            out["bf16_dense_decode"] = {
+                "impl": "torch.nn.functional.scaled_dot_product_attention (enable_gqa), one call per sequence "
+                        "in a CUDA graph, bf16 K/V on the same data",
+                "ms": round(ms_d, 4), "gb_per_s": round(dbytes / ms_d / 1e6, 1),
+                "bytes": dbytes, "l2": "flushed before each rep"}
+            del g
+        except RuntimeError as e:  # noqa: BLE001
+            out["bf16_dense_decode"] = {"unavailable": str(e).splitlines()[0][:200]}
+        del ks_d, vs_d
+        torch.cuda.empty_cache()
+    # 3. dequantise-then-attend (the comparison category of the Open-TQ-Metal abstract):
+    #    tq_dequantize_debug to dense fp32 K/V in the original domain, then SDPA per sequence
+    if not args.no_references and w.batch * L.max_seq * w.n_kv_heads * w.head_dim * 4 * 2 < 24e9:
+        Kd = torch.empty((w.batch, L.max_seq, w.n_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
+        Vd = torch.empty_like(Kd)
+        qf = q.float().view(w.batch, w.n_q_heads, 1, w.head_dim)
+        lens_list = [x + w.n_append for x in w.seq_lens]
+
+        def deq_attend():
+            tq.tq_dequantize_debug(L, kc, ks, lens1, True, Kd, stream)
+            tq.tq_dequantize_debug(L, vc, vs, lens1, True, Vd, stream)
+            for b in range(w.batch):
+                n = lens_list[b]
+                F.scaled_dot_product_attention(qf[b:b + 1], Kd[b, :n].permute(1, 0, 2)[None],
+                                               Vd[b, :n].permute(1, 0, 2)[None], scale=w.scale, enable_gqa=True)
+
+        try:
+            deq_attend()
+            ms_q = _time_cold(deq_attend, 5, flush, stream)
+            out["dequantize_then_attend"] = {
+                "impl": "tq_dequantize_debug (fp32, original domain) + torch SDPA per sequence",
+                "ms": round(ms_q, 3)}
+        except RuntimeError as e:  # noqa: BLE001
+            out["dequantize_then_attend"] = {"unavailable": str(e).splitlines()[0][:200]}
+        del Kd, Vd
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------------------- main paths
 
 def run_reference(args):
@@ -414,6 +520,8 @@ def run_tq(args):
     barrier(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
 
+    refs = {} if args.no_references else reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args)
+
     lens_step = [x + w.n_append for x in w.seq_lens]
     bytes_decode = decode_bytes(w, lens_step)
     bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4)
@@ -447,6 +555,7 @@ def run_tq(args):
     }
     if clk:
         extra["clocks"] = clk
+    extra.update(refs)
     cfg = {"workload": w.name, "global_batch": w.batch * ws, "kv_tokens_per_seq_step": lens_step if w.batch <= 4
            else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
