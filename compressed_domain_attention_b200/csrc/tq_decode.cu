@@ -194,7 +194,11 @@ struct TileWalker {
   }
 };
 
-template <int D, int HKV>
+// TOK_M (query groups of at most 4 heads): the score MMAs put 16 tokens in M and
+// the query's binary16 hi/lo pieces of 4 heads in the 8 N columns, which halves
+// their count; otherwise the 8 heads' hi (rows 0-7) and lo (rows 8-15) pieces
+// are the M rows and the tokens the N columns.
+template <int D, int HKV, bool TOK_M>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap) {
@@ -296,7 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int PAIRS = T_TILE / 2 * HKV;
     constexpr int ITEMS = (PAIRS + 32 * kConverterWarps - 1) / (32 * kConverterWarps);
     const int cw = warp - kConverterWarp;
-    uint32_t src_off[ITEMS], dst_off[ITEMS];
+    // With TOK_M the K scales go to [head][unit][group][token mod 8][m-tile][e] instead
+    // (the lanes of a score row read the tokens gid + 8e + 16 m-tile): two 4-byte stores.
+    constexpr int MT = UNIT / 16;
+    uint32_t src_off[ITEMS], dst_off[ITEMS], dstk_off[ITEMS];
     int tok_of[ITEMS];
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
@@ -307,6 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nt = tau >> 3, tg = (tau & 7) >> 1;
       src_off[k] = (uint32_t)((t * HKV + hh) * NG * 2);
       dst_off[k] = (uint32_t)(4 * (hh * C::SC_HEAD + (u * NG * 4 + tg) * (2 * NT) + nt * 2));
+      dstk_off[k] = (uint32_t)(4 * (hh * C::SC_HEAD + (u * NG * 8 + (tau & 7)) * (2 * MT) + (tau >> 3)));
       tok_of[k] = i < PAIRS ? t : 1 << 30;
     }
     bool dead = false;
@@ -340,7 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t h1 = lds_u16(raw + src_off[k] + HKV * NG * 2 + g * 2);
               const float f0 = ok0 ? __half2float(__ushort_as_half((unsigned short)h0)) : 0.f;
               const float f1 = ok1 ? __half2float(__ushort_as_half((unsigned short)h1)) : 0.f;
-              sts_f2(dst + dst_off[k] + 4 * (g * 4 * 2 * NT), f0, f1);
+              if (TOK_M && kv == 0) {
+                const uint32_t a = dst + dstk_off[k] + 4 * (g * 8 * 2 * MT);
+                sts_f32(a, f0);
+                sts_f32(a + 4 * 2 * MT, f1);
+              } else {
+                sts_f2(dst + dst_off[k] + 4 * (g * 4 * 2 * NT), f0, f1);
+              }
             }
           }
         }
@@ -430,35 +444,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      const float* row = scratch + gid * C::QSTRIDE;
+      // q pieces in the score operand's k order: k-step ks of a group takes the lane's
+      // nibbles {2ks, 2ks + 4} (low position) and {2ks + 1, 2ks + 5} (high position, q / 16).
+      // TOK_M: lane (gid, tig) holds piece gid & 1 (hi, lo) of head gid >> 1 as the B
+      // operand; otherwise head gid's hi (A rows 0-7) and lo (rows 8-15) pieces.
+      const int qh = TOK_M ? (gid >> 1) : gid;
+      const float* row = scratch + qh * C::QSTRIDE;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         float qv[8];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) qv[n] = (gid < G) ? row[32 * g + 8 * tig + n] : 0.f;
+        for (int n = 0; n < 8; ++n) qv[n] = (qh < G) ? row[32 * g + 8 * tig + n] : 0.f;
         float bsum = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
-          // ks = 0 covers nibbles {0,4} (low position) and {1,5} (high position);
-          // ks = 1 covers nibbles {2,6} and {3,7}.
           const float lo0 = qv[2 * ks], lo1 = qv[2 * ks + 4];
           const float hi0 = qv[2 * ks + 1] * 0.0625f, hi1 = qv[2 * ks + 5] * 0.0625f;
           const __half a0 = __float2half_rn(lo0), a1 = __float2half_rn(lo1);
           const __half c0 = __float2half_rn(hi0), c1 = __float2half_rn(hi1);
           const __half a0l = __float2half_rn(lo0 - __half2float(a0)), a1l = __float2half_rn(lo1 - __half2float(a1));
           const __half c0l = __float2half_rn(hi0 - __half2float(c0)), c1l = __float2half_rn(hi1 - __half2float(c1));
-          qA[g][ks][0] = (uint32_t)__half_as_ushort(a0) | ((uint32_t)__half_as_ushort(a1) << 16);
-          qA[g][ks][1] = (uint32_t)__half_as_ushort(a0l) | ((uint32_t)__half_as_ushort(a1l) << 16);
-          qA[g][ks][2] = (uint32_t)__half_as_ushort(c0) | ((uint32_t)__half_as_ushort(c1) << 16);
-          qA[g][ks][3] = (uint32_t)__half_as_ushort(c0l) | ((uint32_t)__half_as_ushort(c1l) << 16);
+          const uint32_t ah = (uint32_t)__half_as_ushort(a0) | ((uint32_t)__half_as_ushort(a1) << 16);
+          const uint32_t al = (uint32_t)__half_as_ushort(a0l) | ((uint32_t)__half_as_ushort(a1l) << 16);
+          const uint32_t ch = (uint32_t)__half_as_ushort(c0) | ((uint32_t)__half_as_ushort(c1) << 16);
+          const uint32_t cl = (uint32_t)__half_as_ushort(c0l) | ((uint32_t)__half_as_ushort(c1l) << 16);
+          if constexpr (TOK_M) {
+            qA[g][ks][0] = (gid & 1) ? al : ah;
+            qA[g][ks][1] = (gid & 1) ? cl : ch;
+          } else {
+            qA[g][ks][0] = ah;
+            qA[g][ks][1] = al;
+            qA[g][ks][2] = ch;
+            qA[g][ks][3] = cl;
+          }
           bsum += (__half2float(a0) + __half2float(a0l)) + (__half2float(a1) + __half2float(a1l));
           bsum += 16.f * ((__half2float(c0) + __half2float(c0l)) + (__half2float(c1) + __half2float(c1l)));
         }
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
+        // TOK_M: the score lanes hold head tig, whose sum sits in lane 8 * tig (gid = 2 tig)
+        if constexpr (TOK_M) bsum = __shfl_sync(0xffffffffu, bsum, (8 * tig) & 31);
         biasK[g] = -bsum * (8.0f * 5.9604644775390625e-08f);  // 8 * 2^-24
       }
-      const int sh = (gid < G) ? reinterpret_cast<const int*>(scratch + 8 * C::QSTRIDE)[gid] : 0;
+      const int sh_h = TOK_M ? tig : gid;  // the head of this lane's scores
+      const int sh = (sh_h < G) ? reinterpret_cast<const int*>(scratch + 8 * C::QSTRIDE)[sh_h] : 0;
       f_h = __int_as_float((127 + 24 - sh) << 23);  // 2^(24 - sh): MMA units -> log2 units
       __syncwarp();
 #pragma unroll
@@ -500,100 +529,216 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (u * UNIT >= left) break;
           const int nv = min(UNIT, left - u * UNIT);
 
-          // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
-          float2 s2[NT], s2b[NT];  // even and odd groups: two independent chains
+          // P^T fragments for P.V, per 16-token k-step: tokens (2 tig, 2 tig + 1) and
+          // (2 tig + 8, 2 tig + 9) of head gid
+          float2 pb[KSP][2];
+          if constexpr (TOK_M) {
+            // --- scores S[token 16 mt + gid + 8 e][head tig], per group g. A = K codes (rows:
+            //     tokens gid, gid + 8 of the m-tile), B = q pieces (columns 2j, 2j + 1: hi, lo
+            //     of head j); the offset term -8 * sum(q) enters through the hi column's C.
+            constexpr int MT = UNIT / 16;
+            float2 s2[MT];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            s2[nt] = make_float2(0.f, 0.f);
-            s2b[nt] = make_float2(0.f, 0.f);
-          }
+            for (int mt = 0; mt < MT; ++mt) s2[mt] = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int g4 = 0; g4 < NG * NT; g4 += 4) {
-            uint32_t kw[4];
-            ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
-            // this lane's K scales for the groups of this batch: (n-tile, e) pairs
-            float skv[4 / NT > 0 ? 4 / NT : 1][2 * NT];
+            for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+              uint32_t kw[4];
+              ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
+              float skm[4 / NT > 0 ? 4 / NT : 1][2 * MT];
 #pragma unroll
-            for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
-              const int g = g4 / NT + gi;
-              const uint32_t a0 = sck + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT));
+              for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
+                const int g = g4 / NT + gi;
+                const uint32_t a0 = sck + 4 * (((uu * NG + g) * 8 + gid) * (2 * MT));
+                if constexpr (MT == 2) {
+                  const float4 v = lds_f4(a0);
+                  skm[gi][0] = v.x;
+                  skm[gi][1] = v.y;
+                  skm[gi][2] = v.z;
+                  skm[gi][3] = v.w;
+                } else {
+                  const float2 v = lds_f2(a0);
+                  skm[gi][0] = v.x;
+                  skm[gi][1] = v.y;
+                }
+              }
 #pragma unroll
-              for (int q4 = 0; q4 < 2 * NT; q4 += 4) {
-                const float4 v = lds_f4(a0 + 4 * q4);
-                skv[gi][q4] = v.x;
-                skv[gi][q4 + 1] = v.y;
-                skv[gi][q4 + 2] = v.z;
-                skv[gi][q4 + 3] = v.w;
+              for (int i = 0; i < 4; i += 2) {
+                const int g = (g4 + i) / NT, mt = ((g4 + i) % NT) >> 1;
+                const int gi = g - g4 / NT;
+                const uint32_t wa = kw[i], wb = kw[i + 1];  // tokens gid and gid + 8 of m-tile mt
+                float c[4];
+                uint32_t a[4];
+                a[0] = and_xor(wa, 0x000F000Fu, 0x00080008u);
+                a[1] = and_xor(wb, 0x000F000Fu, 0x00080008u);
+                a[2] = and_xor(wa, 0x00F000F0u, 0x00800080u);
+                a[3] = and_xor(wb, 0x00F000F0u, 0x00800080u);
+                mma_f16_16816_c(c, a, qA[g][0][0], qA[g][0][1], biasK[g], 0.f, biasK[g], 0.f);
+                const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+                a[0] = and_xor(wa8, 0x000F000Fu, 0x00080008u);
+                a[1] = and_xor(wb8, 0x000F000Fu, 0x00080008u);
+                a[2] = and_xor(wa8, 0x00F000F0u, 0x00800080u);
+                a[3] = and_xor(wb8, 0x00F000F0u, 0x00800080u);
+                mma_f16_16816_acc(c, a, qA[g][1][0], qA[g][1][1]);
+                const float2 x = make_float2(c[0] + c[1], c[2] + c[3]);  // hi + lo
+                s2[mt] = __ffma2_rn(make_float2(skm[gi][2 * mt], skm[gi][2 * mt + 1]), x, s2[mt]);
               }
             }
+            if (nv < UNIT) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int g = (g4 + i) / NT, nt = (g4 + i) % NT;
-              const int gi = g - g4 / NT;
-              const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
-              float c[4];
-              const uint32_t w = kw[i];
-              mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
-                              0.f, 0.f, 0.f, 0.f);
-              const uint32_t w8 = w >> 8;
-              mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
-                                and_xor(w8, 0x00F000F0u, 0x00800080u));
-              // hi + lo rows, plus the offset term -8 * sum(q) of the offset-binary code
-              const float2 x = __fadd2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
-                                          make_float2(biasK[g], biasK[g]));
-              if (g & 1)
-                s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
-              else
-                s2[nt] = __ffma2_rn(sk, x, s2[nt]);
+              for (int mt = 0; mt < MT; ++mt) {
+                if (16 * mt + gid >= nv) s2[mt].x = -INFINITY;
+                if (16 * mt + gid + 8 >= nv) s2[mt].y = -INFINITY;
+              }
             }
-          }
+            // --- online softmax (head tig; lanes with the same tig share a head)
+            float mx = fmaxf(s2[0].x, s2[0].y);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) s2[nt] = __fadd2_rn(s2[nt], s2b[nt]);
-          if (nv < UNIT) {
+            for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(s2[mt].x, s2[mt].y));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float m_new = fmaxf(m_run, mx);
+            const bool grow = m_new > m_run;
+            if (__any_sync(0xffffffffu, grow)) {
+              const float corr = grow ? ((m_run == -INFINITY) ? 0.f : ex2_approx((m_run - m_new) * f_h)) : 1.f;
+              l_run *= corr;
+              // accumulator columns are heads 2 tig, 2 tig + 1: lanes 2 tig, 2 tig + 1 hold them
+              const float2 cc = make_float2(__shfl_sync(0xffffffffu, corr, 2 * tig),
+                                            __shfl_sync(0xffffffffu, corr, 2 * tig + 1));
 #pragma unroll
+              for (int g = 0; g < NG; ++g) {
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                  float2 a01 = __fmul2_rn(make_float2(acc[g][jj][0], acc[g][jj][1]), cc);
+                  float2 a23 = __fmul2_rn(make_float2(acc[g][jj][2], acc[g][jj][3]), cc);
+                  acc[g][jj][0] = a01.x;
+                  acc[g][jj][1] = a01.y;
+                  acc[g][jj][2] = a23.x;
+                  acc[g][jj][3] = a23.y;
+                }
+              }
+              m_run = m_new;
+            }
+            const float mb = (m_run == -INFINITY) ? 0.f : m_run * f_h;
+            float2 lsum = make_float2(0.f, 0.f);
+            // p of token r of m-tile ks, head j, lives in lane 4 (r mod 8) + j, element r / 8
+            const int src0 = 8 * tig + gid, src1 = src0 + 4;
+            const bool head_ok = gid < G;  // G <= 4 here
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              const float2 z = __ffma2_rn(s2[mt], make_float2(f_h, f_h), make_float2(-mb, -mb));
+              const float2 pp = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+              lsum = __fadd2_rn(lsum, pp);
+              const float x0 = __shfl_sync(0xffffffffu, pp.x, src0 & 31);
+              const float x1 = __shfl_sync(0xffffffffu, pp.x, src1 & 31);
+              const float y0 = __shfl_sync(0xffffffffu, pp.y, src0 & 31);
+              const float y1 = __shfl_sync(0xffffffffu, pp.y, src1 & 31);
+              pb[mt][0] = head_ok ? make_float2(x0, x1) : make_float2(0.f, 0.f);
+              pb[mt][1] = head_ok ? make_float2(y0, y1) : make_float2(0.f, 0.f);
+            }
+            l_run += lsum.x + lsum.y;
+          } else {
+            // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
+            float2 s2[NT], s2b[NT];  // even and odd groups: two independent chains
+  #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              if (nt * 8 + 2 * tig >= nv) s2[nt].x = -INFINITY;
-              if (nt * 8 + 2 * tig + 1 >= nv) s2[nt].y = -INFINITY;
+              s2[nt] = make_float2(0.f, 0.f);
+              s2b[nt] = make_float2(0.f, 0.f);
             }
-          }
-
-          // --- online softmax (head gid; the quad's lanes share a head)
-          float mx = fmaxf(s2[0].x, s2[0].y);
-#pragma unroll
-          for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s2[nt].x, s2[nt].y));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float m_new = fmaxf(m_run, mx);
-          const bool grow = m_new > m_run;
-          if (__any_sync(0xffffffffu, grow)) {
-            const float corr = grow ? ((m_run == -INFINITY) ? 0.f : ex2_approx((m_run - m_new) * f_h)) : 1.f;
-            l_run *= corr;
-            const float2 cc = make_float2(__shfl_sync(0xffffffffu, corr, 8 * tig),
-                                          __shfl_sync(0xffffffffu, corr, 8 * tig + 4));
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-#pragma unroll
-              for (int jj = 0; jj < 2; ++jj) {
-                float2 a01 = __fmul2_rn(make_float2(acc[g][jj][0], acc[g][jj][1]), cc);
-                float2 a23 = __fmul2_rn(make_float2(acc[g][jj][2], acc[g][jj][3]), cc);
-                acc[g][jj][0] = a01.x;
-                acc[g][jj][1] = a01.y;
-                acc[g][jj][2] = a23.x;
-                acc[g][jj][3] = a23.y;
+  #pragma unroll
+            for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+              uint32_t kw[4];
+              ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
+              // this lane's K scales for the groups of this batch: (n-tile, e) pairs
+              float skv[4 / NT > 0 ? 4 / NT : 1][2 * NT];
+  #pragma unroll
+              for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
+                const int g = g4 / NT + gi;
+                const uint32_t a0 = sck + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT));
+  #pragma unroll
+                for (int q4 = 0; q4 < 2 * NT; q4 += 4) {
+                  const float4 v = lds_f4(a0 + 4 * q4);
+                  skv[gi][q4] = v.x;
+                  skv[gi][q4 + 1] = v.y;
+                  skv[gi][q4 + 2] = v.z;
+                  skv[gi][q4 + 3] = v.w;
+                }
+              }
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int g = (g4 + i) / NT, nt = (g4 + i) % NT;
+                const int gi = g - g4 / NT;
+                const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
+                float c[4];
+                const uint32_t w = kw[i];
+                mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
+                                0.f, 0.f, 0.f, 0.f);
+                const uint32_t w8 = w >> 8;
+                mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
+                                  and_xor(w8, 0x00F000F0u, 0x00800080u));
+                // hi + lo rows, plus the offset term -8 * sum(q) of the offset-binary code
+                const float2 x = __fadd2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
+                                            make_float2(biasK[g], biasK[g]));
+                if (g & 1)
+                  s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
+                else
+                  s2[nt] = __ffma2_rn(sk, x, s2[nt]);
               }
             }
-            m_run = m_new;
+  #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) s2[nt] = __fadd2_rn(s2[nt], s2b[nt]);
+            if (nv < UNIT) {
+  #pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                if (nt * 8 + 2 * tig >= nv) s2[nt].x = -INFINITY;
+                if (nt * 8 + 2 * tig + 1 >= nv) s2[nt].y = -INFINITY;
+              }
+            }
+
+            // --- online softmax (head gid; the quad's lanes share a head)
+            float mx = fmaxf(s2[0].x, s2[0].y);
+  #pragma unroll
+            for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s2[nt].x, s2[nt].y));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const bool grow = m_new > m_run;
+            if (__any_sync(0xffffffffu, grow)) {
+              const float corr = grow ? ((m_run == -INFINITY) ? 0.f : ex2_approx((m_run - m_new) * f_h)) : 1.f;
+              l_run *= corr;
+              const float2 cc = make_float2(__shfl_sync(0xffffffffu, corr, 8 * tig),
+                                            __shfl_sync(0xffffffffu, corr, 8 * tig + 4));
+  #pragma unroll
+              for (int g = 0; g < NG; ++g) {
+  #pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                  float2 a01 = __fmul2_rn(make_float2(acc[g][jj][0], acc[g][jj][1]), cc);
+                  float2 a23 = __fmul2_rn(make_float2(acc[g][jj][2], acc[g][jj][3]), cc);
+                  acc[g][jj][0] = a01.x;
+                  acc[g][jj][1] = a01.y;
+                  acc[g][jj][2] = a23.x;
+                  acc[g][jj][3] = a23.y;
+                }
+              }
+              m_run = m_new;
+            }
+            const float mb = (m_run == -INFINITY) ? 0.f : m_run * f_h;
+            float2 p2[NT];
+            float2 lsum = make_float2(0.f, 0.f);
+  #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float2 z = __ffma2_rn(s2[nt], make_float2(f_h, f_h), make_float2(-mb, -mb));
+              p2[nt] = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+              lsum = __fadd2_rn(lsum, p2[nt]);
+            }
+            l_run += lsum.x + lsum.y;
+  #pragma unroll
+            for (int ks = 0; ks < KSP; ++ks) {
+              pb[ks][0] = p2[2 * ks];
+              pb[ks][1] = p2[2 * ks + 1];
+            }
+
           }
-          const float mb = (m_run == -INFINITY) ? 0.f : m_run * f_h;
-          float2 p2[NT];
-          float2 lsum = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float2 z = __ffma2_rn(s2[nt], make_float2(f_h, f_h), make_float2(-mb, -mb));
-            p2[nt] = make_float2(ex2_approx(z.x), ex2_approx(z.y));
-            lsum = __fadd2_rn(lsum, p2[nt]);
-          }
-          l_run += lsum.x + lsum.y;
 
           // --- P.V: acc[d][head] += sum_t (c_t,d * 2^-24) * (p_t * sigmaV_t,g). The signed code
           //     enters exactly: u = code + 8 from the lop3, then one binary16 subtract per pair
@@ -612,8 +757,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int g = (g4 + i) / NT, tb = (g4 + i) % NT;  // token blocks tb, tb + 1 = one k-step
               const int ks = tb >> 1;
               const float4 sv = lds_f4(scv + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT) + ks * 4));
-              const uint32_t b0 = pack_half2_f2(__fmul2_rn(p2[2 * ks], make_float2(sv.x, sv.y)));
-              const uint32_t b1 = pack_half2_f2(__fmul2_rn(p2[2 * ks + 1], make_float2(sv.z, sv.w)));
+              const uint32_t b0 = pack_half2_f2(__fmul2_rn(pb[ks][0], make_float2(sv.x, sv.y)));
+              const uint32_t b1 = pack_half2_f2(__fmul2_rn(pb[ks][1], make_float2(sv.z, sv.w)));
               const uint32_t va = vw[i], vb = vw[i + 1];
 #pragma unroll
               for (int jj = 0; jj < 2; ++jj) {
@@ -639,8 +784,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- segment end: write this (sequence, CTA) partial
     const int slot = b + (int)blockIdx.x;
     float l_tot = l_run;
-    l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
-    l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+    if constexpr (TOK_M) {  // head tig: sum over gid
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 4);
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 8);
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 16);
+    } else {  // head gid: sum over tig
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+    }
+    // the lane that reports (m, l) of head hm
+    const int hm = TOK_M ? tig : gid;
+    const bool reports = TOK_M ? (gid == 0 && tig < 4) : (tig == 0);
     const float m_real = (m_run == -INFINITY) ? -INFINITY : m_run * f_h;
     constexpr float kTwo24 = 16777216.f;
     // rotated-domain accumulator of head 2*tig + e at d = 32g + 4*gid + {0, 1, 2, 3};
@@ -651,8 +805,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if constexpr (C::WPH == 1) {
       if (!dead) {
-        if (tig == 0 && gid < G) {
-          float* ml = p.ws_ml + (((int64_t)slot * p.n_q + h * G + gid) * 2) + 2 * (p.batch + 2);
+        if (reports && hm < G) {
+          float* ml = p.ws_ml + (((int64_t)slot * p.n_q + h * G + hm) * 2) + 2 * (p.batch + 2);
           ml[0] = m_real;
           ml[1] = l_tot;
         }
@@ -669,9 +823,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // several warps share a KV head: combine their states through shared memory
       float* mls = scratch + 8 * D;  // [8][2]
-      if (tig == 0 && gid < 8) {
-        mls[2 * gid] = dead ? -INFINITY : m_real;
-        mls[2 * gid + 1] = dead ? 0.f : l_tot;
+      if (reports) {
+        mls[2 * hm] = dead ? -INFINITY : m_real;
+        mls[2 * hm + 1] = dead ? 0.f : l_tot;
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -830,14 +984,14 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   }
 }
 
-template <int D, int HKV>
-static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
+template <int D, int HKV, bool TOK_M>
+static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
                                     cudaStream_t s, cudaEvent_t ev) {
   using C = DecodeCfg<D, HKV>;
   const int smem = C::OFF_PREFIX + 8 * (p.batch + 1) + 8 * 16;
   static bool attr_set = false;  // per instantiation; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV, TOK_M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_MAX);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -854,7 +1008,7 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
   kattr[0].val.programmaticStreamSerializationAllowed = 1;
   kcfg.attrs = kattr;
   kcfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV>, p, kmap, vmap);
+  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
   if (ev != nullptr) {  // timing split: plain stream order between the two kernels
     e = cudaEventRecord(ev, s);
@@ -875,6 +1029,13 @@ static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& k
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p);
+}
+
+template <int D, int HKV>
+static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
+                                    cudaStream_t s, cudaEvent_t ev) {
+  if (p.group <= 4) return launch_decode_dht<D, HKV, true>(p, km, vm, s, ev);
+  return launch_decode_dht<D, HKV, false>(p, km, vm, s, ev);
 }
 
 template <int D>
