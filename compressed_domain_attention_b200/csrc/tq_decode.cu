@@ -215,9 +215,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // Launched as a programmatic dependent of whatever kernel precedes it on the stream
-  // (typically the append): only the launch overlaps; nothing is read before this.
+  // (typically the append). Set-up that reads nothing another kernel writes (barrier
+  // initialisation, tensor-map prefetch) runs before the dependency wait; no global
+  // memory is read before it.
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], kConverterWarps);
+      mbar_init(&empty[s], kConsumerWarps + kConverterWarps);
+    }
+    misc[0] = 0;
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&kmap) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&vmap) : "memory");
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  block_prefix_lengths(p, prefix, prefix + (p.batch + 1));
+  block_prefix_lengths(p, prefix, prefix + (p.batch + 1));  // its barriers also publish the set-up
   const int64_t T_sum = prefix[p.batch];
   int64_t R = (T_sum + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
@@ -237,17 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
     return;
   }
-
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&ready[s], kConverterWarps);
-      mbar_init(&empty[s], kConsumerWarps + kConverterWarps);
-    }
-    misc[0] = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
 
   TileWalker walk;
   walk.start(prefix, p.batch, lo, hi);
@@ -874,16 +876,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and its writes are visible. Phase 1 stages the weights 2^(m_c - m*) of all
 // partials in shared memory; phase 2 streams the accumulators with PF
 // independent loads in flight per thread.
-template <int D>
-__global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+// NTH = 128 threads (8 blocks per SM) when there are many (sequence, head)
+// pairs, 1024 when there are fewer than twice the SMs: a long sequence then has
+// up to one partial per SM, and its loads should all be in flight at once.
+template <int D, int NTH>
+__global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NG = D / 32;
   constexpr int F4 = D / 4;            // float4 columns
-  constexpr int PH = kMergeThreads / F4;  // slot phases
-  constexpr int PF = 8;                   // loads in flight per thread
-  constexpr int MAX_SLOTS = 1024 + kMaxBatch;
+  constexpr int PH = NTH / F4;         // slot phases
+  constexpr int PF = 8;                // loads in flight per thread
+  constexpr int MAX_SLOTS = 1024;      // a sequence meets at most one partial per split-K CTA
   __shared__ float wts[MAX_SLOTS];
   __shared__ float lsv[MAX_SLOTS];
-  __shared__ float red[kMergeThreads / 32];
+  __shared__ float red[NTH / 32];
   __shared__ __align__(16) float accs[PH][D];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
@@ -893,7 +898,7 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
   if (P1 <= P0) {  // empty sequence
-    for (int d = tid; d < D; d += kMergeThreads) out[d] = 0.f;
+    for (int d = tid; d < D; d += NTH) out[d] = 0.f;
     return;
   }
   const int c0 = (int)(P0 / R), c1 = (int)((P1 - 1) / R);
@@ -913,7 +918,7 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   }
   // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l
   float m = -INFINITY;
-  for (int i = tid; i < ns; i += kMergeThreads) {
+  for (int i = tid; i < ns; i += NTH) {
     const float2 e = __ldcg(reinterpret_cast<const float2*>(mlb + i * mls));
     wts[i] = e.x;
     lsv[i] = e.y;
@@ -925,9 +930,9 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   __syncthreads();
   float mstar = red[0];
 #pragma unroll
-  for (int w = 1; w < kMergeThreads / 32; ++w) mstar = fmaxf(mstar, red[w]);
+  for (int w = 1; w < NTH / 32; ++w) mstar = fmaxf(mstar, red[w]);
   float lsum = 0.f;
-  for (int i = tid; i < ns; i += kMergeThreads) {
+  for (int i = tid; i < ns; i += NTH) {
     const float mi = wts[i];
     const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - mstar);
     wts[i] = w;
@@ -940,7 +945,7 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   __syncthreads();
   float L = 0.f;
 #pragma unroll
-  for (int w = 0; w < kMergeThreads / 32; ++w) L += red[w];
+  for (int w = 0; w < NTH / 32; ++w) L += red[w];
   // phase 2: weighted accumulator sums, PH slot phases x F4 float4 columns
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i0 = ph;; i0 += PH * PF) {
@@ -964,7 +969,7 @@ __global__ void __launch_bounds__(kMergeThreads, 8) decode_merge_kernel(const __
   __syncthreads();
   // sum the slot phases per channel and normalise, then the inverse SRHT
   const float inv_l = (L > 0.f) ? 1.f / L : 0.f;
-  for (int d = tid; d < D; d += kMergeThreads) {
+  for (int d = tid; d < D; d += NTH) {
     float sum = 0.f;
 #pragma unroll
     for (int q = 0; q < PH; ++q) sum += accs[q][d];
@@ -1010,17 +1015,21 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   kcfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
+  const bool few = (int64_t)p.batch * p.n_q < 2 * (int64_t)p.grid;  // merge blocks vs SMs
   if (ev != nullptr) {  // timing split: plain stream order between the two kernels
     e = cudaEventRecord(ev, s);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<D><<<p.batch * p.n_q, kMergeThreads, 0, s>>>(p);
+    if (few)
+      decode_merge_kernel<D, 1024><<<p.batch * p.n_q, 1024, 0, s>>>(p);
+    else
+      decode_merge_kernel<D, kMergeThreads><<<p.batch * p.n_q, kMergeThreads, 0, s>>>(p);
     return cudaGetLastError();
   }
   // programmatic dependent launch: the merge grid is set up while the split-K
   // grid drains; griddepcontrol.wait in the merge kernel orders the reads.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.batch * p.n_q));
-  cfg.blockDim = dim3(kMergeThreads);
+  cfg.blockDim = dim3(few ? 1024 : kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1028,7 +1037,8 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p);
+  if (few) return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 1024>, p);
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, kMergeThreads>, p);
 }
 
 template <int D, int HKV>

@@ -14,8 +14,22 @@
 
 namespace tqk {
 
+// max that propagates NaN (max.NaN): the group's abs-max doubles as its non-finite check
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+
 template <int D>
-__global__ void __launch_bounds__(256) quantize_append_kernel(QuantizeParams p) {
+__global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantizeParams p) {
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // nothing is read before this wait. The decode that usually follows may be
+  // scheduled from here on; it waits for this grid's completion before reading.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int NG = D / 32;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t vecs_per_tensor = (int64_t)p.batch * p.n_new * p.n_kv;
@@ -44,17 +58,57 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantizeParams p) 
     valid = false;
     if (which == 0 && t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
   }
+  // sign diagonal: bits [32 part, 32 part + 32) of the mask
+  const uint32_t sw = (uint32_t)(p.sign_bits[part >> 1] >> (32 * (part & 1)));
 #pragma unroll
-  for (int i = 0; i < 32; ++i) u[i] = apply_sign(u[i], p.sign_bits, part * 32 + i);
-  fwht_group<NG>(u, part);  // all lanes participate (shuffles)
+  for (int i = 0; i < 32; ++i) u[i] = __uint_as_float(__float_as_uint(u[i]) ^ ((sw << (31 - i)) & 0x80000000u));
 
-  bool finite = true;
+  // Walsh-Hadamard butterflies, strides 1, 2, ..., D/2 in that order. Stride 1
+  // pairs neighbours; from stride 2 on, element pairs (i, i+1) and (i+h, i+h+1)
+  // go through one packed add and one packed fused (b * -1 + a) = a - b, each
+  // lane rounded once as the scalar operation would be.
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float x = u[i], y = u[i + 1];
+    u[i] = __fadd_rn(x, y);
+    u[i + 1] = __fsub_rn(x, y);
+  }
+#pragma unroll
+  for (int hs = 2; hs < 32; hs <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      if ((i & hs) == 0) {
+        const float2 x = make_float2(u[i], u[i + 1]), y = make_float2(u[i + hs], u[i + hs + 1]);
+        const float2 sum = __fadd2_rn(x, y);
+        const float2 dif = __ffma2_rn(y, f2(-1.f), x);
+        u[i] = sum.x;
+        u[i + 1] = sum.y;
+        u[i + hs] = dif.x;
+        u[i + hs + 1] = dif.y;
+      }
+    }
+  }
+  // strides 32 .. D/2: partner thread part ^ hh; the lower one forms own + partner,
+  // the upper one partner - own (= partner + (-1) * own, one rounding)
+#pragma unroll
+  for (int hh = 1; hh < NG; hh <<= 1) {
+    const float sg = (part & hh) ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, u[i], hh), __shfl_xor_sync(0xffffffffu, u[i + 1], hh));
+      const float2 n = __ffma2_rn(make_float2(u[i], u[i + 1]), f2(sg), o);
+      u[i] = n.x;
+      u[i + 1] = n.y;
+    }
+  }
+
   float a = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    u[i] = __fmul_rn(u[i], p.c_d);
-    finite = finite && (fabsf(u[i]) <= 3.402823466e38f);
-    a = fmaxf(a, fabsf(u[i]));
+  for (int i = 0; i < 32; i += 2) {
+    const float2 y = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(p.c_d));
+    u[i] = y.x;
+    u[i + 1] = y.y;
+    a = fmax_nan(a, fmax_nan(fabsf(y.x), fabsf(y.y)));
   }
   if (!valid) return;
 
@@ -63,26 +117,43 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantizeParams p) 
   const float sigma = __half2float(sig16);
   uint16_t sbits = __half_as_ushort(sig16);
   uint32_t packed[4] = {0u, 0u, 0u, 0u};
-  if (!finite || !(fabsf(sigma) <= 65504.f)) {
+  if (!(a <= 3.402823466e38f) || !(fabsf(sigma) <= 65504.f)) {
     sbits = 0x7C00u;
     status_or(p.status, TQ_STATUS_NONFINITE);
   } else if (sigma != 0.f) {
-    // code = rint(fl(y / sigma)). With inv = RN(1/sigma) and r = RN(y * inv),
-    // |r - y/sigma| <= 2^-23 |y/sigma| <= 2^-20 (|y/sigma| <= 7 * (1 + 2^-11) < 8), and
-    // |fl(y/sigma) - y/sigma| <= 2^-21. So when r is more than 2^-19 away from every
-    // half-integer, y/sigma and fl(y/sigma) are more than 2^-21 away from it too and
-    // both round to rint(r). Otherwise (probability about 2^-18 per element) the IEEE
-    // division is taken. The result is the same code as the plain definition.
-    const float inv = __frcp_rn(sigma);
+    // code = clamp(rint(fl(y / sigma)), -7, 7). Fast form: r = RN(y * RN(1/sigma)); adding
+    // 1.5 * 2^23 rounds r to an integer (ties to even) in the low mantissa bits, whose
+    // low nibble is then the two's-complement code. |r - y/sigma| <= 2^-23 |y/sigma| < 2^-20
+    // and |fl(y/sigma) - y/sigma| <= 2^-21, so unless r lies within 2^-19 of a
+    // half-integer, fl(y/sigma) rounds to the same integer. A binary16-normal sigma keeps
+    // |y/sigma| <= 7 (1 + 2^-11) (1 + 2^-24), so no clamp is needed. Otherwise (a tie
+    // within 2^-19, probability about 2^-18 per element, or a subnormal sigma) the
+    // thread redoes its group with the IEEE division and the clamp.
+    bool slow = !(sigma >= 6.103515625e-05f);  // binary16 subnormal scale
+    if (!slow) {
+      const float inv = __frcp_rn(sigma);
+      constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float r = __fmul_rn(u[i], inv);
-      const float rr = rintf(r);
-      int c = (int)rr;
-      if (fabsf(fabsf(r - rr) - 0.5f) <= 1.9073486328125e-06f)  // 2^-19
-        c = __float2int_rn(__fdiv_rn(u[i], sigma));
-      c = max(-7, min(7, c));
-      packed[i >> 3] |= ((uint32_t)c & 0xFu) << (4 * (i & 7));
+      for (int i = 0; i < 32; i += 2) {
+        const float2 rv = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(inv));
+        const float2 rm = __fadd2_rn(rv, f2(kMagic));
+        const float2 rr = __fadd2_rn(rm, f2(-kMagic));
+        const float2 d = __ffma2_rn(rr, f2(-1.f), rv);  // r - rint(r), exact
+        slow |= fabsf(d.x) >= 0.49999809265136719f;    // 0.5 - 2^-19
+        slow |= fabsf(d.y) >= 0.49999809265136719f;
+        const uint32_t pair = (__float_as_uint(rm.x) & 0xFu) | ((__float_as_uint(rm.y) & 0xFu) << 4);
+        packed[i >> 3] |= pair << (4 * (i & 7));
+      }
+    }
+    if (slow) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) packed[k] = 0u;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        int c = __float2int_rn(__fdiv_rn(u[i], sigma));
+        c = max(-7, min(7, c));
+        packed[i >> 3] |= ((uint32_t)c & 0xFu) << (4 * (i & 7));
+      }
     }
   }
   const int64_t row = ((int64_t)b * p.max_seq + pos + t) * p.n_kv + h;
@@ -96,7 +167,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantizeParams p) 
 // with original_domain, the inverse rotation x = s o (c_D * H * yhat), the
 // same butterfly order as the forward transform.
 template <int D>
-__global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
+__global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__ DequantParams p) {
   constexpr int NG = D / 32;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rows = (int64_t)p.batch * p.max_seq * p.n_kv;
@@ -145,8 +216,19 @@ template <int D>
 static cudaError_t launch_quantize_d(const QuantizeParams& p, cudaStream_t s) {
   const int64_t threads = 2LL * p.batch * p.n_new * p.n_kv * (D / 32);
   const int64_t blocks = (threads + 255) / 256;
-  quantize_append_kernel<D><<<(unsigned)blocks, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: set-up overlaps the previous kernel's tail,
+  // griddepcontrol.wait in the kernel orders the reads
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_append_kernel<D>, p);
 }
 
 cudaError_t launch_quantize(const QuantizeParams& p, int D, cudaStream_t s) {
