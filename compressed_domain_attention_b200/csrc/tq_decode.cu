@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (TOK_M) {
             // --- scores S[token 16 mt + gid + 8 e][head tig], per group g. A = K codes (rows:
             //     tokens gid, gid + 8 of the m-tile), B = q pieces (columns 2j, 2j + 1: hi, lo
-            //     of head j); the offset term -8 * sum(q) enters through the hi column's C.
+            //     of head j).
             constexpr int MT = UNIT / 16;
             float2 s2[MT];
 #pragma unroll
@@ -574,14 +574,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a[1] = and_xor(wb, 0x000F000Fu, 0x00080008u);
                 a[2] = and_xor(wa, 0x00F000F0u, 0x00800080u);
                 a[3] = and_xor(wb, 0x00F000F0u, 0x00800080u);
-                mma_f16_16816_c(c, a, qA[g][0][0], qA[g][0][1], biasK[g], 0.f, biasK[g], 0.f);
+                mma_f16_16816_c(c, a, qA[g][0][0], qA[g][0][1], 0.f, 0.f, 0.f, 0.f);
                 const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
                 a[0] = and_xor(wa8, 0x000F000Fu, 0x00080008u);
                 a[1] = and_xor(wb8, 0x000F000Fu, 0x00080008u);
                 a[2] = and_xor(wa8, 0x00F000F0u, 0x00800080u);
                 a[3] = and_xor(wb8, 0x00F000F0u, 0x00800080u);
                 mma_f16_16816_acc(c, a, qA[g][1][0], qA[g][1][1]);
-                const float2 x = make_float2(c[0] + c[1], c[2] + c[3]);  // hi + lo
+                // hi + lo columns, plus the offset term -8 * sum(q) of the offset-binary code
+                const float2 x = __fadd2_rn(make_float2(c[0] + c[1], c[2] + c[3]), make_float2(biasK[g], biasK[g]));
                 s2[mt] = __ffma2_rn(make_float2(skm[gi][2 * mt], skm[gi][2 * mt + 1]), x, s2[mt]);
               }
             }
