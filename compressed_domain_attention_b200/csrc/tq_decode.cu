@@ -152,7 +152,7 @@ struct TileWalker {
   int batch;
   int64_t lo, hi;
   int b;
-  int64_t seg_lo, seg_hi, t0;
+  int seg_lo, seg_hi, t0;  // token offsets within sequence b (< max_seq)
 
   __device__ void start(const int64_t* pf, int nb, int64_t l, int64_t h) {
     prefix = pf;
@@ -175,9 +175,9 @@ struct TileWalker {
       const int64_t s0 = max(lo, prefix[b]) - prefix[b];
       const int64_t s1 = min(hi, prefix[b + 1]) - prefix[b];
       if (s0 < s1) {
-        seg_lo = s0;
-        seg_hi = s1;
-        t0 = s0;
+        seg_lo = (int)s0;
+        seg_hi = (int)s1;
+        t0 = (int)s0;
         return;
       }
     }
@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sb = smem + stage * C::STAGE_BYTES;
         const int64_t row0 = (int64_t)walk.b * p.max_seq + walk.t0;
         const int soff = (int)((row0 * C::SROW) & 15);
-        const int nv = (int)min((int64_t)T_TILE, walk.seg_hi - walk.t0);
+        const int nv = min(T_TILE, walk.seg_hi - walk.t0);
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   while (!walk.done()) {
     const int b = walk.b;
-    const int64_t seg_hi = walk.seg_hi;
+    const int seg_hi = walk.seg_hi;
     // ---------------- segment prologue: rotate this warp's q heads, build fragments
     {
       constexpr int HP = 32 / NG;  // heads rotated per pass
@@ -509,12 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (!seg_end) {
       const int stage = tile_i % STAGES;
       const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
-      if (!dead) {
-        if (!mbar_wait_bounded(&full[stage], par, kWaitLimitNs) ||
-            !mbar_wait_bounded(&ready[stage], par, kWaitLimitNs)) {
-          dead = true;
-          if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
-        }
+      // The converters arrive on `ready` only after they observed `full` complete, so
+      // its completion (release by the converters, acquire here) also orders this
+      // warp's reads after the stage's tensor copies.
+      if (!dead && !mbar_wait_bounded(&ready[stage], par, kWaitLimitNs)) {
+        dead = true;
+        if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
       }
       if (!dead) {
         const uint32_t sbase = smem_base + stage * C::STAGE_BYTES;
@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sck = sbase + C::OFF_SC32 + 4 * h * C::SC_HEAD;
         const uint32_t scv = sck + 4 * C::SC_KV;
         // tokens of the segment left in this tile, from this warp's first row on
-        const int left = (int)min((int64_t)T_TILE, seg_hi - walk.t0) - sub * UPW * UNIT;
+        const int left = min(T_TILE, seg_hi - walk.t0) - sub * UPW * UNIT;
 #pragma unroll 1
         for (int u = 0; u < UPW; ++u) {
           const int uu = sub * UPW + u;  // unit index within the tile
