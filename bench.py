@@ -492,33 +492,89 @@ def run_tq(args):
     if st != 0:
         raise RuntimeError(f"device status {st} during the benchmark")
 
-    # e2e: host buffers in pinned memory, copies inside the timed region
-    h_k = k_new.cpu().pin_memory()
-    h_v = v_new.cpu().pin_memory()
-    h_q = q.cpu().pin_memory()
-    h_out = torch.empty_like(out, device="cpu").pin_memory()
-    d_k, d_v, d_q = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(q)
+    # e2e: host buffers in pinned memory, every step's copies inside the timed region.
+    # As a serving loop would run it: a copy stream brings step i+1's inputs in and
+    # step i's output back while the compute stream runs step i (double-buffered
+    # device inputs and outputs, ordered by events).
+    h_k = [k_new.cpu().pin_memory() for _ in range(2)]
+    h_v = [v_new.cpu().pin_memory() for _ in range(2)]
+    h_q = [q.cpu().pin_memory() for _ in range(2)]
+    h_out = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(2)]
+    d_k = [torch.empty_like(k_new) for _ in range(2)]
+    d_v = [torch.empty_like(v_new) for _ in range(2)]
+    d_q = [torch.empty_like(q) for _ in range(2)]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    cstream = torch.cuda.Stream(device=dev)
+    gstream = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of the buffer landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]   # compute on the buffer finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # output of the buffer copied back
 
-    def e2e_step():
-        d_k.copy_(h_k, non_blocking=True)
-        d_v.copy_(h_v, non_blocking=True)
-        d_q.copy_(h_q, non_blocking=True)
-        tq.tq_quantize_append(L, d_k, d_v, w.n_append, lens, kc, ks, vc, vs, status, stream)
-        tq.tq_decode_attention(L, d_q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
-        h_out.copy_(out, non_blocking=True)
+    def e2e_loop(n, cs):
+        """n steps on compute stream cs; copies on cstream (forked from and joined back to cs)."""
+        cstream.wait_stream(cs)
 
-    for _ in range(3):
-        e2e_step()
+        def h2d(i):
+            j = i % 2
+            with torch.cuda.stream(cstream):
+                if i >= 2:
+                    cstream.wait_event(ev_done[j])  # step i-2 no longer reads these inputs
+                d_k[j].copy_(h_k[j], non_blocking=True)
+                d_v[j].copy_(h_v[j], non_blocking=True)
+                d_q[j].copy_(h_q[j], non_blocking=True)
+                ev_in[j].record(cstream)
+
+        h2d(0)
+        for i in range(n):
+            j = i % 2
+            if i + 1 < n:
+                h2d(i + 1)
+            cs.wait_event(ev_in[j])
+            if i >= 2:
+                cs.wait_event(ev_out[j])  # step i-2's output was copied out of d_out[j]
+            tq.tq_quantize_append(L, d_k[j], d_v[j], w.n_append, lens, kc, ks, vc, vs, status, cs)
+            tq.tq_decode_attention(L, d_q[j], lens1, kc, ks, vc, vs, w.scale, d_out[j], wsp, status, cs)
+            ev_done[j].record(cs)
+            with torch.cuda.stream(cstream):
+                cstream.wait_event(ev_done[j])
+                h_out[j].copy_(d_out[j], non_blocking=True)
+                ev_out[j].record(cstream)
+        cs.wait_stream(cstream)
+
+    e2e_loop(3, stream)
     torch.cuda.synchronize()
+    # The K steps (copies, append, decode) captured once as a CUDA graph, as a
+    # fixed-shape serving step would run; eager launches if capture is refused.
+    e2e_mode = "cuda graph of the K steps"
+    graph = torch.cuda.CUDAGraph()
+    try:
+        gstream.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=gstream):
+            e2e_loop(args.steps, gstream)
+        with torch.cuda.stream(gstream):
+            graph.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # noqa: BLE001 - reported in the output line
+        graph = None
+        e2e_mode = f"eager launches (graph capture failed: {type(exc).__name__})"
+        torch.cuda.synchronize()
     barrier(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    if graph is not None:
+        gstream.wait_stream(stream)
+        with torch.cuda.stream(gstream):  # replay() launches on the current stream
+            e0.record(gstream)
+            graph.replay()
+            e1.record(gstream)
+    else:
+        e0.record(stream)
+        e2e_loop(args.steps, stream)
+        e1.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
+    if not torch.equal(h_out[(args.steps - 1) % 2], out.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-timed output")
 
     refs = {} if args.no_references else reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args)
 
@@ -547,7 +603,9 @@ def run_tq(args):
                      "merge_avg_ms": round(merge_avg, 4)},
         "e2e": {"value": round(ws * bytes_step * args.steps / max_e2e / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(k_new.numel() * k_new.element_size() * 2 + q.numel() * q.element_size()),
-                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+                "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+                "copies": "pinned host buffers; step i+1's inputs in and step i's output out on a copy "
+                          "stream while step i computes (double-buffered, event-ordered)", "launch": e2e_mode},
         "gpu_launches": 3 * args.steps,
         "kernel_timing": "split-K/merge durations from a second pass of the same K steps with an event "
                          "between the two kernels (the timed region itself launches the merge as a "
