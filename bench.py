@@ -46,6 +46,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
     ap.add_argument("--no-references", action="store_true",
                     help="skip the quantise-throughput, bf16 dense-KV and dequantise-then-attend reference points")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-configuration report instead of the step benchmark: decode and prefill-quantise "
+                         "times (median, p10, p90; cold L2, and warm L2 where the cache fits) for every workload "
+                         "shape, one JSON line each")
     return ap.parse_args(argv)
 
 
@@ -265,15 +269,51 @@ class OracleStep:
         self.oracle.decode_attention(self.s, self.q, self.lens + 1, self.kc, self.ks, self.vc, self.vs, self.w.scale)
         return time.perf_counter() - t0
 
+    def run_parallel(self, threads):
+        """The same step with independent sequences spread over host threads.
+
+        Each thread calls the unchanged oracle on one sequence's slices; the C++
+        calls release the interpreter lock, so the threads run on separate cores.
+        """
+        from concurrent.futures import ThreadPoolExecutor
+        o, n = self.oracle, len(self.seqs)
+
+        def one(i):
+            sl = slice(i, i + 1)
+            o.quantize_append(self.s, self.kn[sl], self.vn[sl], self.lens[sl], self.kc[sl], self.ks[sl],
+                              self.vc[sl], self.vs[sl])
+            o.decode_attention(self.s, self.q[sl], self.lens[sl] + 1, self.kc[sl], self.ks[sl], self.vc[sl],
+                               self.vs[sl], self.w.scale)
+
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(one, range(n)))
+            return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux hosts
+        return os.cpu_count() or 1
+
 
 def cpu_baseline(w, tensors, target_tokens):
     seqs = oracle_sample(w, target_tokens)
     o = OracleStep(w, tensors, seqs)
     dt = o.run()
-    return {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+    line = {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
                       f"({o.ntok} KV tokens x {w.n_q_heads} q heads), single-threaded C++ oracle, {dt:.2f} s",
             "seconds": round(dt, 3)}
+    cores = host_cores()
+    if cores > 1 and len(seqs) > 1:
+        dtp = o.run_parallel(min(cores, len(seqs)))
+        line["parallel"] = {"value": round(o.nbytes / dtp / 1e9, 4), "unit": UNIT,
+                            "cores": min(cores, len(seqs)), "host_cores": cores, "seconds": round(dtp, 3),
+                            "how": "the same sample, one sequence per task on a thread pool over the unchanged "
+                                   "oracle (its C++ calls run outside the interpreter lock)"}
+    return line
 
 
 # ----------------------------------------------------------------------------- same-run reference points
@@ -379,6 +419,125 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args):
         torch.cuda.empty_cache()
     return out
 
+
+
+# ----------------------------------------------------------------------------- per-configuration sweep
+
+def _pct(xs, q):
+    xs = sorted(xs)
+    k = (len(xs) - 1) * q
+    lo, hi = int(k), min(int(k) + 1, len(xs) - 1)
+    return xs[lo] + (xs[hi] - xs[lo]) * (k - lo)
+
+
+def _time_reps(fn, reps, flush, stream):
+    """Device times (ms) of fn(), one per rep; flush (a buffer > L2 rewritten) before each rep if given."""
+    import torch
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.add_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return {"median": round(statistics.median(ts), 4), "p10": round(_pct(ts, 0.1), 4),
+            "p90": round(_pct(ts, 0.9), 4), "reps": reps}
+
+
+def run_sweep(args):
+    """Every workload shape: decode, append and prefill-quantise times, one JSON line per configuration."""
+    import torch
+    import torch.nn.functional as F
+    from compressed_domain_attention_b200 import synthetic as syn
+    from compressed_domain_attention_b200 import tq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)  # 256 MB > 126 MB L2
+    peak, peak_kind = load_peaks()
+    cfgs = [("c0", syn.tiny_single_head()), ("c1", syn.llama3_8b_layer())]
+    cfgs += [("c2", syn.gemma3_1b_sweep(T)) for T in (256, 512, 1024, 2048, 4096)]
+    cfgs += [("c3", syn.llama31_70b_long()), ("c4", syn.ragged_serving())]
+    for tag, w in cfgs:
+        t = syn.generate(w, device="cuda")
+        n_app = max(w.n_append, 1)
+        cap = max(w.seq_lens) + n_app
+        L = tq.tq_cache_layout(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+        kc, ks, vc, vs = tq.alloc_cache(L, dev)
+        wsp = tq.alloc_workspace(L, dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        l1 = tq.tq_cache_layout(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        cs, ss = int(L.code_stride_seq), int(L.scale_stride_seq)
+        kb = [t.k[b][None].contiguous() for b in range(w.batch)]
+        vb = [t.v[b][None].contiguous() for b in range(w.batch)]
+
+        def prefill():
+            for b in range(w.batch):
+                tq.tq_quantize_append(l1, kb[b], vb[b], w.seq_lens[b], zero, kc[b * cs:(b + 1) * cs], ks[b * ss:],
+                                      vc[b * cs:(b + 1) * cs], vs[b * ss:], status, stream)
+
+        prefill()
+        pre = _time_reps(prefill, 5, flush, stream)
+        vecs = 2 * sum(w.seq_lens) * w.n_kv_heads
+        lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
+        q = t.q.contiguous()
+        out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+
+        def decode():
+            tq.tq_decode_attention(L, q, lens, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
+
+        for _ in range(10):
+            decode()
+        reps = 20 if sum(w.seq_lens) * w.n_kv_heads >= 1 << 20 else 100
+        cold = _time_reps(decode, reps, flush, stream)
+        nbytes = decode_bytes(w, w.seq_lens)
+        warm = _time_reps(decode, reps, None, stream) if nbytes < 64e6 else None
+        kn, vn = t.k_new.contiguous() if w.n_append else None, t.v_new.contiguous() if w.n_append else None
+        app = None
+        if w.n_append:
+            def append():
+                tq.tq_quantize_append(L, kn, vn, w.n_append, lens, kc, ks, vc, vs, status, stream)
+            app = _time_reps(append, 50, flush, stream)
+        dense = None
+        if w.dtype != torch.float32:
+            ks_d = [t.k[b].permute(1, 0, 2).contiguous()[None] for b in range(w.batch)]
+            vs_d = [t.v[b].permute(1, 0, 2).contiguous()[None] for b in range(w.batch)]
+            qd = q.view(w.batch, w.n_q_heads, 1, w.head_dim)
+
+            def dense_fn():
+                for b in range(w.batch):
+                    F.scaled_dot_product_attention(qd[b:b + 1], ks_d[b], vs_d[b], scale=w.scale, enable_gqa=True)
+
+            dense_fn()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                dense_fn()
+            dense = _time_reps(g.replay, min(reps, 20), flush, stream)
+            del g, ks_d, vs_d
+        torch.cuda.synchronize()
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())} in the sweep ({w.name})")
+        ms = cold["median"]
+        line = {"sweep": tag, "workload": w.name, "batch": w.batch, "tokens": sum(w.seq_lens),
+                "decode_ms_cold_l2": cold, "decode_gbs": round(nbytes / ms / 1e6, 1),
+                "pct_of_8_tbs": round(nbytes / ms / 1e6 / 80.0, 2),
+                "pct_of_measured_hbm": round(nbytes / ms / 1e6 / peak * 100.0, 2), "peak_kind": peak_kind,
+                "decode_steps_per_s": round(w.batch / ms * 1e3, 1),
+                "kv_tokens_per_s": round(sum(w.seq_lens) / ms * 1e3, 1),
+                "decode_ms_warm_l2": warm,
+                "prefill_quantize": {"vectors": vecs, "launches": w.batch, "ms": pre,
+                                     "vectors_per_s": round(vecs / pre["median"] * 1e3, 1)},
+                "append_ms_cold_l2": app,
+                "bf16_dense_sdpa_ms_cold_l2": dense,
+                "speedup_vs_bf16_dense": round(dense["median"] / ms, 2) if dense else None}
+        print(json.dumps(line), flush=True)
+        del kc, ks, vc, vs, wsp, t, kb, vb
+        torch.cuda.empty_cache()
+    return 0
 
 # ----------------------------------------------------------------------------- main paths
 
@@ -638,6 +797,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_tq(args)
 
 

@@ -337,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
-          const uint32_t raw = smem_u32(sb + 2 * C::CODE_BYTES + kv * C::SCALE_SLAB + soff);
+          // plain (not volatile) shared loads: the compiler may issue a lane's loads together
+          const uint16_t* raw = reinterpret_cast<const uint16_t*>(sb + 2 * C::CODE_BYTES + kv * C::SCALE_SLAB + soff);
           const uint32_t dst = sc + kv * C::SC_KV * 4;
 #pragma unroll
           for (int k = 0; k < ITEMS; ++k) {
@@ -346,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok0 = t < nv, ok1 = t + 1 < nv;
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
-              const uint32_t h0 = lds_u16(raw + src_off[k] + g * 2);
-              const uint32_t h1 = lds_u16(raw + src_off[k] + HKV * NG * 2 + g * 2);
+              const uint32_t h0 = raw[src_off[k] / 2 + g];
+              const uint32_t h1 = raw[src_off[k] / 2 + HKV * NG + g];
               const float f0 = ok0 ? __half2float(__ushort_as_half((unsigned short)h0)) : 0.f;
               const float f1 = ok1 ? __half2float(__ushort_as_half((unsigned short)h1)) : 0.f;
               if (TOK_M && kv == 0) {
@@ -415,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       constexpr int HP = 32 / NG;  // heads rotated per pass
       const int part = lane % NG;
+      const uint32_t sw = sign_word(p.sign_bits, part);
+      const float qs = p.c_d * p.sm_scale_log2;  // 1/sqrt(D) and the softmax scale in log2 units
       for (int j0 = 0; j0 < 8; j0 += HP) {
         const int j = j0 + lane / NG;
         float u[32];
@@ -425,13 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) u[i] = 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = apply_sign(u[i], p.sign_bits, part * 32 + i);
-        fwht_group<NG>(u, part);
+        for (int i = 0; i < 32; ++i) u[i] = flip_sign(u[i], sw, i);
+        fwht_group_x2<NG>(u, part);
         float mx = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          u[i] = __fmul_rn(__fmul_rn(u[i], p.c_d), p.sm_scale_log2);
-          mx = fmaxf(mx, fabsf(u[i]));
+        for (int i = 0; i < 32; i += 2) {
+          const float2 y = __fmul2_rn(make_float2(u[i], u[i + 1]), make_float2(qs, qs));
+          u[i] = y.x;
+          u[i + 1] = y.y;
+          mx = fmaxf(mx, fmaxf(fabsf(y.x), fabsf(y.y)));
         }
 #pragma unroll
         for (int o = 1; o < NG; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -439,9 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mx > 0.f) (void)frexpf(mx, &e);
         const int sh = min(100, max(-100, 14 - e));  // scaled max < 2^14
         if (j < 8) {
-          float* row = scratch + j * C::QSTRIDE;
+          const float sc = __int_as_float((127 + sh) << 23);  // 2^sh, exact scaling
+          float4* row = reinterpret_cast<float4*>(scratch + j * C::QSTRIDE + part * 32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) row[part * 32 + i] = ldexpf(u[i], sh);
+          for (int i = 0; i < 32; i += 4) {
+            const float2 a = __fmul2_rn(make_float2(u[i], u[i + 1]), make_float2(sc, sc));
+            const float2 c = __fmul2_rn(make_float2(u[i + 2], u[i + 3]), make_float2(sc, sc));
+            row[i / 4] = make_float4(a.x, a.y, c.x, c.y);
+          }
           if (part == 0) reinterpret_cast<int*>(scratch + 8 * C::QSTRIDE)[j] = sh;
         }
       }
@@ -839,32 +849,38 @@ __global__ void __launch_bounds__(kThreads, 1)
               dead ? make_float4(0.f, 0.f, 0.f, 0.f) : final4(g, e);
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
-      const int items = HKV * G * D;
-      for (int it = tid; it < items; it += kConsumerWarps * 32) {
-        const int hk = it / (G * D), j = (it / D) % G, d = it % D;
+      // one thread per (kv head, q head): the weights 2^(m_w - m*) of the WPH partials
+      // replace their m words, and (m*, sum of weighted l) goes out
+      for (int pr = tid; pr < HKV * G; pr += kConsumerWarps * 32) {
+        const int hk = pr / G, j = pr % G;
         float mstar = -INFINITY;
         for (int sb = 0; sb < C::WPH; ++sb) {
           const float* sm = reinterpret_cast<const float*>(smem + C::OFF_SCRATCH + (hk + sb * HKV) * C::SCRATCH);
           mstar = fmaxf(mstar, sm[8 * D + 2 * j]);
         }
-        float lsum = 0.f, asum = 0.f;
-        if (mstar != -INFINITY) {
-          for (int sb = 0; sb < C::WPH; ++sb) {
-            const float* sm = reinterpret_cast<const float*>(smem + C::OFF_SCRATCH + (hk + sb * HKV) * C::SCRATCH);
-            const float mw = sm[8 * D + 2 * j];
-            if (mw == -INFINITY) continue;
-            const float wgt = exp2f(mw - mstar);
-            lsum += wgt * sm[8 * D + 2 * j + 1];
-            asum += wgt * sm[j * D + d];
-          }
+        float lsum = 0.f;
+        for (int sb = 0; sb < C::WPH; ++sb) {
+          float* sm = reinterpret_cast<float*>(smem + C::OFF_SCRATCH + (hk + sb * HKV) * C::SCRATCH);
+          const float mw = sm[8 * D + 2 * j];
+          const float wgt = (mw == -INFINITY) ? 0.f : exp2f(mw - mstar);
+          lsum += wgt * sm[8 * D + 2 * j + 1];
+          sm[8 * D + 2 * j] = wgt;
         }
-        const int64_t qh = (int64_t)slot * p.n_q + hk * G + j;
-        p.ws_acc[qh * D + d] = asum;
-        if (d == 0) {
-          float* ml = p.ws_ml + qh * 2 + 2 * (p.batch + 2);
-          ml[0] = mstar;
-          ml[1] = lsum;
+        float* ml = p.ws_ml + ((int64_t)slot * p.n_q + hk * G + j) * 2 + 2 * (p.batch + 2);
+        ml[0] = mstar;
+        ml[1] = lsum;
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+      const int items = HKV * G * D;
+      for (int it = tid; it < items; it += kConsumerWarps * 32) {
+        const int hk = it / (G * D), j = (it / D) % G, d = it % D;
+        float asum = 0.f;
+#pragma unroll
+        for (int sb = 0; sb < C::WPH; ++sb) {
+          const float* sm = reinterpret_cast<const float*>(smem + C::OFF_SCRATCH + (hk + sb * HKV) * C::SCRATCH);
+          asum = fmaf(sm[8 * D + 2 * j], sm[j * D + d], asum);
         }
+        p.ws_acc[((int64_t)slot * p.n_q + hk * G + j) * D + d] = asum;
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
     }

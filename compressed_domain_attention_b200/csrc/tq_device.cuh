@@ -46,6 +46,59 @@ __device__ __forceinline__ void fwht_group(float (&u)[32], int part) {
   }
 }
 
+// The same transform, same stage order and rounding, with the pair operations
+// packed: stride 1 runs scalar; strides 2..16 add and subtract element pairs
+// (i, i+1) and (i+h, i+h+1) with one f32x2 add and one f32x2 fma (b * -1 + a =
+// a - b, one rounding per lane); the strides across threads form partner + own
+// or partner - own as one f32x2 fma with a +-1 factor. Bit-identical to
+// fwht_group (each lane of a packed op rounds once, exactly as the scalar op).
+template <int NG>
+__device__ __forceinline__ void fwht_group_x2(float (&u)[32], int part) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float x = u[i], y = u[i + 1];
+    u[i] = __fadd_rn(x, y);
+    u[i + 1] = __fsub_rn(x, y);
+  }
+#pragma unroll
+  for (int hs = 2; hs < 32; hs <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      if ((i & hs) == 0) {
+        const float2 x = make_float2(u[i], u[i + 1]), y = make_float2(u[i + hs], u[i + hs + 1]);
+        const float2 sum = __fadd2_rn(x, y);
+        const float2 dif = __ffma2_rn(y, make_float2(-1.f, -1.f), x);
+        u[i] = sum.x;
+        u[i + 1] = sum.y;
+        u[i + hs] = dif.x;
+        u[i + hs + 1] = dif.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 1; hh < NG; hh <<= 1) {
+    const float sg = (part & hh) ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, u[i], hh), __shfl_xor_sync(0xffffffffu, u[i + 1], hh));
+      const float2 n = __ffma2_rn(make_float2(u[i], u[i + 1]), make_float2(sg, sg), o);
+      u[i] = n.x;
+      u[i + 1] = n.y;
+    }
+  }
+}
+
+// Bits [32 part, 32 part + 32) of the sign mask: the diagonal of the 32 elements
+// thread `part` of a head vector holds.
+__device__ __forceinline__ uint32_t sign_word(const uint64_t* sign_bits, int part) {
+  return (uint32_t)(sign_bits[part >> 1] >> (32 * (part & 1)));
+}
+
+// Element i of a thread's 32: flip its sign by bit i of the thread's sign word (exact).
+__device__ __forceinline__ float flip_sign(float x, uint32_t sw, int i) {
+  return __uint_as_float(__float_as_uint(x) ^ ((sw << (31 - i)) & 0x80000000u));
+}
+
 // Sign flip of element e by bit e of the sign mask (exact).
 __device__ __forceinline__ float apply_sign(float x, const uint64_t* sign_bits, int e) {
   const uint32_t bit = (uint32_t)(sign_bits[e >> 6] >> (e & 63)) & 1u;

@@ -58,49 +58,12 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
     valid = false;
     if (which == 0 && t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
   }
-  // sign diagonal: bits [32 part, 32 part + 32) of the mask
-  const uint32_t sw = (uint32_t)(p.sign_bits[part >> 1] >> (32 * (part & 1)));
+  // sign diagonal, then the Walsh-Hadamard butterflies (strides 1, 2, ..., D/2 in
+  // that order, packed pair operations that round each lane once as the scalar steps)
+  const uint32_t sw = sign_word(p.sign_bits, part);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) u[i] = __uint_as_float(__float_as_uint(u[i]) ^ ((sw << (31 - i)) & 0x80000000u));
-
-  // Walsh-Hadamard butterflies, strides 1, 2, ..., D/2 in that order. Stride 1
-  // pairs neighbours; from stride 2 on, element pairs (i, i+1) and (i+h, i+h+1)
-  // go through one packed add and one packed fused (b * -1 + a) = a - b, each
-  // lane rounded once as the scalar operation would be.
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float x = u[i], y = u[i + 1];
-    u[i] = __fadd_rn(x, y);
-    u[i + 1] = __fsub_rn(x, y);
-  }
-#pragma unroll
-  for (int hs = 2; hs < 32; hs <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      if ((i & hs) == 0) {
-        const float2 x = make_float2(u[i], u[i + 1]), y = make_float2(u[i + hs], u[i + hs + 1]);
-        const float2 sum = __fadd2_rn(x, y);
-        const float2 dif = __ffma2_rn(y, f2(-1.f), x);
-        u[i] = sum.x;
-        u[i + 1] = sum.y;
-        u[i + hs] = dif.x;
-        u[i + hs + 1] = dif.y;
-      }
-    }
-  }
-  // strides 32 .. D/2: partner thread part ^ hh; the lower one forms own + partner,
-  // the upper one partner - own (= partner + (-1) * own, one rounding)
-#pragma unroll
-  for (int hh = 1; hh < NG; hh <<= 1) {
-    const float sg = (part & hh) ? -1.f : 1.f;
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, u[i], hh), __shfl_xor_sync(0xffffffffu, u[i + 1], hh));
-      const float2 n = __ffma2_rn(make_float2(u[i], u[i + 1]), f2(sg), o);
-      u[i] = n.x;
-      u[i + 1] = n.y;
-    }
-  }
+  for (int i = 0; i < 32; ++i) u[i] = flip_sign(u[i], sw, i);
+  fwht_group_x2<NG>(u, part);
 
   float a = 0.f;
 #pragma unroll
