@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int part = lane % NG;
       const uint32_t sw = sign_word(p.sign_bits, part);
       const float qs = p.c_d * p.sm_scale_log2;  // 1/sqrt(D) and the softmax scale in log2 units
-      for (int j0 = 0; j0 < 8; j0 += HP) {
+      for (int j0 = 0; j0 < 8 && j0 < G; j0 += HP) {  // rows j >= G are never read
         const int j = j0 + lane / NG;
         float u[32];
         if (j < G && j < 8) {
@@ -464,22 +464,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* row = scratch + qh * C::QSTRIDE;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
-        float qv[8];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) qv[n] = (qh < G) ? row[32 * g + 8 * tig + n] : 0.f;
-        float bsum = 0.f;
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (qh < G) {
+          v0 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig);
+          v1 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig + 4);
+        }
+        const float qv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        // the code offset term -8 * sum(q) (the high-position pieces carry q / 16 against a
+        // 16x nibble, so every element enters with weight 1); q itself stands for its hi + lo
+        // pieces, which agree with it to 2^-22
+        float bsum = ((qv[0] + qv[1]) + (qv[2] + qv[3])) + ((qv[4] + qv[5]) + (qv[6] + qv[7]));
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
-          const float lo0 = qv[2 * ks], lo1 = qv[2 * ks + 4];
-          const float hi0 = qv[2 * ks + 1] * 0.0625f, hi1 = qv[2 * ks + 5] * 0.0625f;
-          const __half a0 = __float2half_rn(lo0), a1 = __float2half_rn(lo1);
-          const __half c0 = __float2half_rn(hi0), c1 = __float2half_rn(hi1);
-          const __half a0l = __float2half_rn(lo0 - __half2float(a0)), a1l = __float2half_rn(lo1 - __half2float(a1));
-          const __half c0l = __float2half_rn(hi0 - __half2float(c0)), c1l = __float2half_rn(hi1 - __half2float(c1));
-          const uint32_t ah = (uint32_t)__half_as_ushort(a0) | ((uint32_t)__half_as_ushort(a1) << 16);
-          const uint32_t al = (uint32_t)__half_as_ushort(a0l) | ((uint32_t)__half_as_ushort(a1l) << 16);
-          const uint32_t ch = (uint32_t)__half_as_ushort(c0) | ((uint32_t)__half_as_ushort(c1) << 16);
-          const uint32_t cl = (uint32_t)__half_as_ushort(c0l) | ((uint32_t)__half_as_ushort(c1l) << 16);
+          const float2 lo = make_float2(qv[2 * ks], qv[2 * ks + 4]);
+          const float2 hi = __fmul2_rn(make_float2(qv[2 * ks + 1], qv[2 * ks + 5]), make_float2(0.0625f, 0.0625f));
+          const __half2 lo_h = __float22half2_rn(lo), hi_h = __float22half2_rn(hi);
+          // residual pieces: x - fp16(x) is exact in binary32, then rounded to binary16
+          const float2 lo_b = __half22float2(lo_h), hi_b = __half22float2(hi_h);
+          const __half2 lo_l = __float22half2_rn(make_float2(lo.x - lo_b.x, lo.y - lo_b.y));
+          const __half2 hi_l = __float22half2_rn(make_float2(hi.x - hi_b.x, hi.y - hi_b.y));
+          const uint32_t ah = *reinterpret_cast<const uint32_t*>(&lo_h);
+          const uint32_t al = *reinterpret_cast<const uint32_t*>(&lo_l);
+          const uint32_t ch = *reinterpret_cast<const uint32_t*>(&hi_h);
+          const uint32_t cl = *reinterpret_cast<const uint32_t*>(&hi_l);
           if constexpr (TOK_M) {
             qA[g][ks][0] = (gid & 1) ? al : ah;
             qA[g][ks][1] = (gid & 1) ? cl : ch;
@@ -489,8 +496,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             qA[g][ks][2] = ch;
             qA[g][ks][3] = cl;
           }
-          bsum += (__half2float(a0) + __half2float(a0l)) + (__half2float(a1) + __half2float(a1l));
-          bsum += 16.f * ((__half2float(c0) + __half2float(c0l)) + (__half2float(c1) + __half2float(c1l)));
         }
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
