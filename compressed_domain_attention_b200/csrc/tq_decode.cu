@@ -912,11 +912,44 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   __shared__ float lsv[MAX_SLOTS];
   __shared__ float red[NTH / 32];
   __shared__ __align__(16) float accs[PH][D];
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   const int b = blockIdx.x / p.n_q, hq = blockIdx.x % p.n_q;
-  const int64_t* hdr = ws_header(p.ws_ml);
-  const int64_t P0 = hdr[b], P1 = hdr[b + 1], R = hdr[p.batch + 1];
+  // The range of this sequence's partials follows from the lengths alone, with the
+  // split-K kernel's rules (lengths outside [0, max_seq] count as 0). The lengths are
+  // read before the dependency wait: this grid is launched only once every split-K
+  // block has passed its own wait, so whatever wrote them has completed.
+  __shared__ long long red64[2][NTH / 32];
+  long long before = 0, total = 0;
+  for (int i = tid; i < p.batch; i += NTH) {
+    int x = p.seq_lens[i];
+    if (x < 0 || x > p.max_seq) x = 0;
+    total += x;
+    if (i < b) before += x;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  if (lane == 0) {
+    red64[0][wp] = before;
+    red64[1][wp] = total;
+  }
+  __syncthreads();
+  before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < NTH / 32; ++w) {
+    before += red64[0][w];
+    total += red64[1][w];
+  }
+  int len_b = p.seq_lens[b];
+  if (len_b < 0 || len_b > p.max_seq) len_b = 0;
+  int64_t R = (total + p.grid - 1) / p.grid;
+  if (R < p.min_split) R = p.min_split;
+  R = ((R + 15) / 16) * 16;
+  const int64_t P0 = before, P1 = before + len_b;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
   if (P1 <= P0) {  // empty sequence
