@@ -22,6 +22,9 @@
 //          TurboQuant changes" (a Walsh-Hadamard rotation first, then low-bit
 //          storage, unpacked when attention reads it); §"Known limitations /
 //          head dimension" (power-of-two head dims only).
+//  [MLX-modes] the same guide, §"Cache modes" and §"What TurboQuant changes":
+//          the recommended default mode (fp16+turbo4) keeps K in FP16 and
+//          compresses only V, because K decides where attention looks.
 //  [AMD]   "TurboQuant on AMD GPUs" (oracore.dev), §4: Walsh-Hadamard spreads
 //          energy evenly and suits kernels better than a dense random rotation.
 //
@@ -219,6 +222,68 @@ void dequantize_rotated(const uint8_t* bytes, const uint16_t* scales, int D, flo
   for (int i = 0; i < D; ++i) yhat[i] = (float)codes[i] * f16_to_f32(scales[i / 32]);
 }
 
+int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const float* s, const float* q,
+                    const int32_t* seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
+                    const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale,
+                    const uint8_t* which, float* out) {
+  int32_t st = 0;
+  const int G = n_q / n_kv;
+  const int64_t cb = D / 2, sb = D / 32;
+  std::vector<float> qr(D), yk(D), yv(D), o32(D);
+  std::vector<double> z, acc(D);
+  for (int b = 0; b < batch; ++b) {
+    const int len = seq_lens[b];
+    for (int hq = 0; hq < n_q; ++hq) {
+      if (which && !which[(int64_t)b * n_q + hq]) continue;
+      float* o = out + ((int64_t)b * n_q + hq) * D;
+      if (len <= 0 || len > max_seq) {
+        if (len > max_seq) st |= ORC_STATUS_CAPACITY;
+        for (int i = 0; i < D; ++i) o[i] = 0.0f;
+        continue;
+      }
+      const int kv = hq / G;
+      // int4 K lives in the rotated domain and pairs with SRHT(q); binary16 K
+      // (asymmetric cache) is in the original domain and pairs with q itself
+      if (k_f16)
+        std::memcpy(qr.data(), q + ((int64_t)b * n_q + hq) * D, sizeof(float) * D);
+      else
+        srht_forward_vec(q + ((int64_t)b * n_q + hq) * D, s, D, qr.data());
+      z.assign(len, 0.0);
+      for (int t = 0; t < len; ++t) {
+        const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
+        if (k_f16) {
+          for (int i = 0; i < D; ++i) yk[i] = f16_to_f32(k_f16[row * D + i]);
+        } else {
+          dequantize_rotated(k_codes + row * cb, k_scales + row * sb, D, yk.data());
+        }
+        double dot = 0.0;
+        for (int i = 0; i < D; ++i) dot += (double)qr[i] * (double)yk[i];
+        z[t] = (double)sm_scale * dot;
+      }
+      double m = z[0];
+      for (int t = 1; t < len; ++t)
+        if (z[t] > m) m = z[t];
+      double l = 0.0;
+      for (int t = 0; t < len; ++t) {
+        z[t] = std::exp(z[t] - m);
+        l += z[t];
+      }
+      for (int i = 0; i < D; ++i) acc[i] = 0.0;
+      for (int t = 0; t < len; ++t) {
+        const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
+        dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());
+        const double w = z[t] / l;
+        for (int i = 0; i < D; ++i) acc[i] += w * (double)yv[i];
+      }
+      for (int i = 0; i < D; ++i) o32[i] = (float)acc[i];
+      srht_inverse_vec(o32.data(), s, D, o);
+    }
+  }
+  return st;
+}
+
+
+
 }  // namespace
 
 extern "C" {
@@ -336,51 +401,53 @@ int32_t oracle_decode_attention(int batch, int max_seq, int n_kv, int n_q, int D
                                 const uint8_t* k_codes, const uint16_t* k_scales,
                                 const uint8_t* v_codes, const uint16_t* v_scales,
                                 float sm_scale, const uint8_t* which, float* out) {
+  return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, k_codes, k_scales, nullptr, v_codes, v_scales,
+                     sm_scale, which, out);
+}
+
+// ---- asymmetric cache: K in binary16, V as int4 codes [MLX-modes] ----
+// Reading taken: K is stored as the binary16 (round to nearest even) of the
+// input element in the ORIGINAL domain (no rotation: nothing is quantised, so
+// the rotation has no job on K), layout [batch][max_seq][n_kv][D]; V is encoded
+// exactly as in oracle_quantize_append. A K element whose binary16 is not
+// finite raises ORC_STATUS_NONFINITE (its bits are stored as converted).
+int32_t oracle_quantize_append_kf16(int batch, int max_seq, int n_kv, int D, const float* s,
+                                    const float* k, const float* v, int n_new, const int32_t* start_pos,
+                                    uint16_t* k_f16, uint8_t* v_codes, uint16_t* v_scales) {
   int32_t st = 0;
-  const int G = n_q / n_kv;
   const int64_t cb = D / 2, sb = D / 32;
-  std::vector<float> qr(D), yk(D), yv(D), o32(D);
-  std::vector<double> z, acc(D);
   for (int b = 0; b < batch; ++b) {
-    const int len = seq_lens[b];
-    for (int hq = 0; hq < n_q; ++hq) {
-      if (which && !which[(int64_t)b * n_q + hq]) continue;
-      float* o = out + ((int64_t)b * n_q + hq) * D;
-      if (len <= 0 || len > max_seq) {
-        if (len > max_seq) st |= ORC_STATUS_CAPACITY;
-        for (int i = 0; i < D; ++i) o[i] = 0.0f;
-        continue;
+    const int64_t p0 = start_pos[b];
+    if (p0 < 0 || p0 + n_new > max_seq) {
+      st |= ORC_STATUS_CAPACITY;
+      continue;
+    }
+    for (int t = 0; t < n_new; ++t) {
+      for (int h = 0; h < n_kv; ++h) {
+        const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
+        const int64_t row = ((int64_t)b * max_seq + p0 + t) * n_kv + h;
+        for (int i = 0; i < D; ++i) {
+          const uint16_t hbits = f32_to_f16_rne(k[src + i]);
+          if ((hbits & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
+          k_f16[row * D + i] = hbits;
+        }
+        st |= oracle_encode(v + src, s, D, 1, v_codes + row * cb, v_scales + row * sb);
       }
-      const int kv = hq / G;
-      srht_forward_vec(q + ((int64_t)b * n_q + hq) * D, s, D, qr.data());
-      z.assign(len, 0.0);
-      for (int t = 0; t < len; ++t) {
-        const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
-        dequantize_rotated(k_codes + row * cb, k_scales + row * sb, D, yk.data());
-        double dot = 0.0;
-        for (int i = 0; i < D; ++i) dot += (double)qr[i] * (double)yk[i];
-        z[t] = (double)sm_scale * dot;
-      }
-      double m = z[0];
-      for (int t = 1; t < len; ++t)
-        if (z[t] > m) m = z[t];
-      double l = 0.0;
-      for (int t = 0; t < len; ++t) {
-        z[t] = std::exp(z[t] - m);
-        l += z[t];
-      }
-      for (int i = 0; i < D; ++i) acc[i] = 0.0;
-      for (int t = 0; t < len; ++t) {
-        const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
-        dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());
-        const double w = z[t] / l;
-        for (int i = 0; i < D; ++i) acc[i] += w * (double)yv[i];
-      }
-      for (int i = 0; i < D; ++i) o32[i] = (float)acc[i];
-      srht_inverse_vec(o32.data(), s, D, o);
     }
   }
   return st;
+}
+
+// Decode attention over the asymmetric cache: the same steps as
+// oracle_decode_attention, except that the scores pair q itself with the binary16
+// K values (both in the original domain); the values are still the
+// rotated-domain V, mapped back by SRHT^-1 after the weighted sum.
+int32_t oracle_decode_attention_kf16(int batch, int max_seq, int n_kv, int n_q, int D, const float* s,
+                                     const float* q, const int32_t* seq_lens, const uint16_t* k_f16,
+                                     const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale,
+                                     const uint8_t* which, float* out) {
+  return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, nullptr, nullptr, k_f16, v_codes, v_scales,
+                     sm_scale, which, out);
 }
 
 // Dequantise a whole cache: out [batch][max_seq][n_kv][D] binary32, rows t >= len_b

@@ -88,3 +88,47 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
     lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
     monkeypatch.setattr(oracle, "_lib", lib)
     assert failing_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"
+
+
+# Planted mistakes in the asymmetric (binary16 K) path, checked by its own pins.
+KF16_MUTATIONS = {
+    "kf16_k_index_reversed": ("k_f16[row * D + i] = hbits;", "k_f16[row * D + (D - 1 - i)] = hbits;"),
+    "kf16_q_rotated": ("std::memcpy(qr.data(), q + ((int64_t)b * n_q + hq) * D, sizeof(float) * D);",
+                       "srht_forward_vec(q + ((int64_t)b * n_q + hq) * D, s, D, qr.data());"),
+    "kf16_k_halved": ("for (int i = 0; i < D; ++i) yk[i] = f16_to_f32(k_f16[row * D + i]);",
+                      "for (int i = 0; i < D; ++i) yk[i] = 0.5f * f16_to_f32(k_f16[row * D + i]);"),
+}
+
+
+def kf16_pins(orc):
+    yield lambda: pins.test_kf16_append_stores_numpy_binary16_and_the_symmetric_v(orc, 128)
+    yield lambda: pins.test_kf16_attention_equals_fp64_original_domain(orc, 128, 16, 2, 33)
+    yield lambda: pins.test_kf16_attention_special_cases(orc)
+
+
+def failing_kf16_pins(orc):
+    failed = 0
+    for check in kf16_pins(orc):
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_kf16_pins_pass_on_committed_oracle(orc):
+    assert failing_kf16_pins(orc) == 0
+
+
+@pytest.mark.parametrize("name", sorted(KF16_MUTATIONS))
+def test_planted_kf16_mistake_is_caught(name, tmp_path, monkeypatch):
+    before, after = KF16_MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "tq_oracle_mut.cpp"
+    mutated.write_text(src.replace(before, after))
+    lib_path = tmp_path / f"libtq_oracle_{name}.so"
+    subprocess.run(["g++", *CXXFLAGS, "-o", str(lib_path), str(mutated)], check=True)
+    lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert failing_kf16_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"

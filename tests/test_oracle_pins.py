@@ -426,3 +426,111 @@ def test_dequantize_matches_independent(orc):
     assert np.array_equal(yr[0, :T].astype(np.float64), np_dequant_rotated(kc[0, :T], ks[0, :T], D))
     assert np.max(np.abs(xo[0, :T] - np_dequant_original(kc[0, :T], ks[0, :T], s))) < 1e-5
     assert np.all(yr[0, T:] == 0) and np.all(xo[0, T:] == 0)
+
+
+# ---------------------------------------------------------------- asymmetric cache (binary16 K, int4 V)
+# mlxcel "TurboQuant KV cache compression", §"Cache modes": the recommended
+# default keeps K in FP16 and compresses only V.
+
+def make_cache_kf16(orc, rng, B, T, Hkv, D, s, k=None, v=None):
+    if k is None:
+        k = np.stack([heavy_tailed(rng, T * Hkv, D).reshape(T, Hkv, D) for _ in range(B)])
+        v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    k16 = orc.new_k16_cache(B, T, Hkv, D)
+    vc, vs = orc.new_cache(B, T, Hkv, D)
+    st = orc.quantize_append_kf16(s, k, v, np.zeros(B, np.int32), k16, vc, vs)
+    return k, v, k16, vc, vs, st
+
+
+@pytest.mark.parametrize("D", DIMS)
+def test_kf16_append_stores_numpy_binary16_and_the_symmetric_v(orc, D):
+    rng = np.random.default_rng(D + 7)
+    s = orc.sign_vector(0, D)
+    k, v, k16, vc, vs, st = make_cache_kf16(orc, rng, 2, 9, 2, D, s)
+    assert st == 0
+    # K: numpy's own float32 -> float16 conversion (round to nearest even), bit for bit
+    assert np.array_equal(k16, k.astype(np.float16).view(np.uint16))
+    # V: the same bytes and scales as the symmetric append
+    kc2, ks2 = orc.new_cache(2, 9, 2, D)
+    vc2, vs2 = orc.new_cache(2, 9, 2, D)
+    orc.quantize_append(s, k, v, np.zeros(2, np.int32), kc2, ks2, vc2, vs2)
+    assert np.array_equal(vc, vc2) and np.array_equal(vs, vs2)
+
+
+def test_kf16_append_overflow_and_capacity(orc):
+    D = 32
+    s = orc.sign_vector(0, D)
+    k = np.zeros((1, 1, 1, D), np.float32)
+    k[0, 0, 0, 3] = 70000.0  # beyond the binary16 range -> inf
+    v = np.ones((1, 1, 1, D), np.float32)
+    k16 = orc.new_k16_cache(1, 1, 1, D)
+    vc, vs = orc.new_cache(1, 1, 1, D)
+    st = orc.quantize_append_kf16(s, k, v, np.zeros(1, np.int32), k16, vc, vs)
+    assert st & orc.STATUS_NONFINITE
+    assert k16[0, 0, 0, 3] == 0x7C00
+    st = orc.quantize_append_kf16(s, k, v, np.ones(1, np.int32), k16, vc, vs)  # position 1 of a 1-token cache
+    assert st & orc.STATUS_CAPACITY
+
+
+def brute_force_attention_kf16(q, lens, k16, vc, vs, s, sm_scale):
+    """softmax(q K^T * scale) V in fp64: K the binary16 values, V dequantised to the original domain."""
+    B, Hq, D = q.shape
+    Hkv = vc.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        L = lens[b]
+        if L == 0:
+            continue
+        for hq in range(Hq):
+            kv = hq // G
+            K = k16[b, :L, kv].view(np.float16).astype(np.float64)
+            V = np_dequant_original(vc[b, :L, kv], vs[b, :L, kv], s)
+            z = K @ q[b, hq].astype(np.float64) * sm_scale
+            w = np.exp(z - z.max())
+            out[b, hq] = (w / w.sum()) @ V
+    return out
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,T", [(32, 4, 1, 17), (128, 4, 1, 64), (128, 16, 2, 33), (64, 2, 2, 5),
+                                        (256, 4, 1, 40)])
+def test_kf16_attention_equals_fp64_original_domain(orc, D, Hq, Hkv, T):
+    rng = np.random.default_rng(D * 1000 + T + 1)
+    s = orc.sign_vector(0, D)
+    B = 2
+    _, _, k16, vc, vs, st = make_cache_kf16(orc, rng, B, T, Hkv, D, s)
+    assert st == 0
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    lens = np.array([T, max(1, T // 2)], np.int32)
+    scale = 1.0 / np.sqrt(D)
+    got, st = orc.decode_attention_kf16(s, q, lens, k16, vc, vs, scale)
+    assert st == 0
+    ref = brute_force_attention_kf16(q, lens, k16, vc, vs, s, scale)
+    assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_kf16_attention_special_cases(orc):
+    rng = np.random.default_rng(43)
+    D, Hkv, Hq, T = 128, 2, 4, 24
+    s = orc.sign_vector(0, D)
+    _, _, k16, vc, vs, _ = make_cache_kf16(orc, rng, 1, T, Hkv, D, s)
+    q = rng.standard_normal((1, Hq, D)).astype(np.float32)
+    # T = 1: the one dequantised V row (original domain)
+    out1, _ = orc.decode_attention_kf16(s, q, np.array([1], np.int32), k16, vc, vs, 0.1)
+    for hq in range(Hq):
+        ref = np_dequant_original(vc[0, 0, hq // 2], vs[0, 0, hq // 2], s)
+        assert np.max(np.abs(out1[0, hq] - ref)) < 1e-6 * max(1, np.abs(ref).max())
+    # all K rows identical: uniform weights for any q -> mean of V; equals q = 0
+    k2 = k16.copy()
+    k2[0, :] = k16[0, 0]
+    outk, _ = orc.decode_attention_kf16(s, q, np.array([T], np.int32), k2, vc, vs, 0.3)
+    out0, _ = orc.decode_attention_kf16(s, np.zeros_like(q), np.array([T], np.int32), k16, vc, vs, 0.3)
+    assert np.max(np.abs(outk - out0)) < 1e-6
+    for hq in range(Hq):
+        ref = np_dequant_original(vc[0, :T, hq // 2], vs[0, :T, hq // 2], s).mean(axis=0)
+        assert np.max(np.abs(out0[0, hq] - ref)) < 1e-6
+    # empty sequence and a length past max_seq
+    oute, st = orc.decode_attention_kf16(s, q, np.array([0], np.int32), k16, vc, vs, 0.1)
+    assert st == 0 and np.all(oute == 0)
+    outc, st = orc.decode_attention_kf16(s, q, np.array([T + 1], np.int32), k16, vc, vs, 0.1)
+    assert st & orc.STATUS_CAPACITY and np.all(outc == 0)
