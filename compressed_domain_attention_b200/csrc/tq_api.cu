@@ -99,11 +99,39 @@ int encode_codes_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::T
   return TQ_OK;
 }
 
+// 4-D view of a binary16 K buffer: (64 halves, D/64 lines, batch*max_seq tokens,
+// n_kv heads) with strides (128 B, token stride, 2D B), box (64, D/64, tile, n_kv):
+// the shared-memory image is [head][tile][D] binary16 in 128-byte lines with the
+// 128-byte swizzle (D = 32: one 64-byte line per row, 64-byte swizzle).
+int encode_k16_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::TensorMap128* out) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
+  const int D = L->head_dim;
+  const int inner = D < 64 ? D : 64;
+  const int lines = D / inner;
+  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)lines, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq,
+                        (cuuint64_t)L->n_kv_heads};
+  cuuint64_t strides[3] = {(cuuint64_t)inner * 2, (cuuint64_t)L->k_stride_tok, (cuuint64_t)D * 2};
+  cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)lines, (cuuint32_t)tile, (cuuint32_t)L->n_kv_heads};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUtensorMapSwizzle sw = inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap m;
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = (int)r;
+    return TQ_ERR_CUDA;
+  }
+  std::memcpy(out, &m, sizeof(m));
+  return TQ_OK;
+}
+
 int check_layout(const tq_layout_t* L) {
   if (L == nullptr) return TQ_ERR_INVALID_ARG;
   tq_layout_t chk;
-  const int r = tq_cache_layout(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
-                                L->sign_seed, &chk);
+  const int r = tq_cache_layout_kv(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
+                                   L->sign_seed, L->k_format, &chk);
   if (r != TQ_OK) return r;
   if (std::memcmp(&chk, L, sizeof(chk)) != 0) return TQ_ERR_INVALID_ARG;  // edited or stale layout
   return TQ_OK;
@@ -127,7 +155,13 @@ extern "C" {
 
 int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
                     uint64_t sign_seed, tq_layout_t* out) {
+  return tq_cache_layout_kv(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_K_INT4, out);
+}
+
+int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                       uint64_t sign_seed, int k_format, tq_layout_t* out) {
   if (out == nullptr) return TQ_ERR_INVALID_ARG;
+  if (k_format != TQ_K_INT4 && k_format != TQ_K_FP16) return TQ_ERR_INVALID_ARG;
   if (batch <= 0 || max_seq <= 0 || n_kv_heads <= 0 || n_q_heads <= 0) return TQ_ERR_INVALID_ARG;
   if (n_q_heads % n_kv_heads != 0) return TQ_ERR_INVALID_ARG;
   // mlxcel §"Known limitations / head dimension": power-of-two head dims only.
@@ -157,6 +191,16 @@ int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int h
   L.scales_bytes = (uint64_t)batch * (uint64_t)L.scale_stride_seq * 2ull + kMaxTileTokens * srow + 32ull;
   L.max_ctas = kMaxCtas;
   L.decode_workspace_bytes = workspace_bytes(batch, n_q_heads, head_dim, kMaxCtas);
+  L.k_format = k_format;
+  if (k_format == TQ_K_FP16) {
+    L.k_stride_tok = (int64_t)n_kv_heads * head_dim * 2;
+    L.k_stride_seq = (int64_t)max_seq * L.k_stride_tok;
+    L.k_bytes = (uint64_t)batch * (uint64_t)L.k_stride_seq;
+  } else {
+    L.k_stride_tok = L.code_stride_tok;
+    L.k_stride_seq = L.code_stride_seq;
+    L.k_bytes = L.codes_bytes;
+  }
   *out = L;
   return TQ_OK;
 }
@@ -170,7 +214,9 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
   if (n_new > layout->max_seq) return TQ_ERR_CAPACITY;
   if (in_dtype != TQ_F32 && in_dtype != TQ_BF16 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
   if (n_new == 0) return TQ_OK;
-  if (!k || !v || !d_start_pos || !k_codes || !k_scales || !v_codes || !v_scales) return TQ_ERR_INVALID_ARG;
+  const bool kf16 = layout->k_format == TQ_K_FP16;
+  if (!k || !v || !d_start_pos || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales)
+    return TQ_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes)) return TQ_ERR_INVALID_ARG;
   if ((int64_t)layout->batch * n_new * layout->n_kv_heads * layout->n_groups * 2 > (int64_t)INT32_MAX * 256)
     return TQ_ERR_UNSUPPORTED;
@@ -190,6 +236,7 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
   p.status = d_status;
   copy_signs(layout, p.sign_bits);
   p.c_d = layout->c_d;
+  p.k_f16 = kf16 ? 1 : 0;
   cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
@@ -205,9 +252,12 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
   if (layout->batch > kMaxBatchDecode) return TQ_ERR_UNSUPPORTED;
   if (!(Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) || G > 8) return TQ_ERR_UNSUPPORTED;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
-  if (!q || !d_seq_lens || !k_codes || !k_scales || !v_codes || !v_scales || !out || !workspace)
+  const bool kf16 = layout->k_format == TQ_K_FP16;
+  // binary16 K tiles: the stage ring holds them only up to head_dim 128
+  if (kf16 && D > 128) return TQ_ERR_UNSUPPORTED;
+  if (!q || !d_seq_lens || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales || !out || !workspace)
     return TQ_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) ||
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || (!kf16 && !aligned16(k_scales)) ||
       !aligned16(v_scales) || !aligned16(out) || !aligned16(workspace))
     return TQ_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return TQ_ERR_INVALID_ARG;
@@ -226,12 +276,13 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
   }
   if (grid > layout->max_ctas) grid = layout->max_ctas;
   if (ws_bytes < workspace_bytes(layout->batch, Hq, D, grid)) return TQ_ERR_INVALID_ARG;
-  if (tqk::decode_smem_bytes(D, Hkv) <= 0) return TQ_ERR_UNSUPPORTED;
+  if (tqk::decode_smem_bytes(D, Hkv, kf16 ? 1 : 0) <= 0) return TQ_ERR_UNSUPPORTED;
 
   tqk::TensorMap128 km, vm;
-  r = encode_codes_map(layout, k_codes, tqk::decode_tile_tokens(D, Hkv), &km);
+  const int tile = tqk::decode_tile_tokens(D, Hkv, kf16 ? 1 : 0);
+  r = kf16 ? encode_k16_map(layout, k_codes, tile, &km) : encode_codes_map(layout, k_codes, tile, &km);
   if (r != TQ_OK) return r;
-  r = encode_codes_map(layout, v_codes, tqk::decode_tile_tokens(D, Hkv), &vm);
+  r = encode_codes_map(layout, v_codes, tile, &vm);
   if (r != TQ_OK) return r;
 
   tqk::DecodeParams p;
@@ -256,6 +307,7 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
   p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
   p.c_d = layout->c_d;
   copy_signs(layout, p.sign_bits);
+  p.k_f16 = kf16 ? 1 : 0;
   cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }

@@ -58,40 +58,58 @@ constexpr int kMaxBatch = 1024;
 constexpr int kMergeThreads = 128;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every pipeline wait
 
-template <int D, int HKV>
+// KF16: K tiles are binary16 in the original domain (asymmetric cache), the V
+// side is unchanged; no K scales are copied or converted.
+template <int D, int HKV, bool KF16 = false>
 struct DecodeCfg {
   static constexpr int NG = D / 32;                  // groups per head vector
-  static constexpr int RB = D / 2;                   // code bytes per (token, head)
+  static constexpr int RB = D / 2;                   // V (and int4 K) code bytes per (token, head)
+  static constexpr int KRB = KF16 ? 2 * D : RB;      // K bytes per (token, head)
   static constexpr int WPH = kConsumerWarps / HKV;   // consumer warps per KV head
-  static constexpr int UNIT = D <= 128 ? 32 : 16;    // tokens per warp work unit
+  // tokens per warp work unit (16 where a 32-token binary16 K tile would not fit)
+  static constexpr int UNIT = (KF16 && D == 128) || D == 256 ? 16 : 32;
   static constexpr int NT = UNIT / 8;                // 8-token n-tiles per unit
   static constexpr int KSP = UNIT / 16;              // 16-token k-steps of P.V per unit
-  static constexpr int UPW_A = 2048 / (UNIT * RB) > 0 ? 2048 / (UNIT * RB) : 1;
+  // units per warp per stage: K tile of at most 16 KB (int4) or 32 KB (binary16)
+  static constexpr int UPW_A0 = KF16 ? 4096 / (UNIT * KRB) : 2048 / (UNIT * RB);
+  static constexpr int UPW_A = UPW_A0 > 0 ? UPW_A0 : 1;
   static constexpr int UPW_B = 256 / (UNIT * WPH) > 0 ? 256 / (UNIT * WPH) : 1;
-  static constexpr int UPW = UPW_A < UPW_B ? UPW_A : UPW_B;  // units per warp per stage
+  static constexpr int UPW = UPW_A < UPW_B ? UPW_A : UPW_B;
   static constexpr int T_TILE = UNIT * UPW * WPH;    // tokens per stage (<= 256)
   static constexpr int UNITS_TILE = T_TILE / UNIT;
-  static constexpr int CODE_BYTES = T_TILE * HKV * RB;
+  static constexpr int CODE_BYTES = T_TILE * HKV * RB;   // V tile
+  static constexpr int K_BYTES = T_TILE * HKV * KRB;     // K tile
   static constexpr int SROW = HKV * NG * 2;          // raw scale bytes per token (all heads)
   static constexpr int SCALE_SLAB = ((T_TILE * SROW + 15) / 16) * 16 + 16;
   static constexpr int SC_HEAD = T_TILE * NG + 4;    // fp32 scale floats per head (16 B pad)
   static constexpr int SC_KV = HKV * SC_HEAD;
-  static constexpr int OFF_SC32 = 2 * CODE_BYTES + 2 * SCALE_SLAB;  // within a stage
-  static constexpr int STAGE_BYTES = ((OFF_SC32 + 2 * SC_KV * 4 + 1023) / 1024) * 1024;
-  static constexpr uint32_t STAGE_TX = 2 * CODE_BYTES + 2 * SCALE_SLAB;
+  static constexpr int NSC = KF16 ? 1 : 2;           // scale sets in a stage (K and V, or V)
+  // stage: [K tile][V tile][raw scale slabs (K, V)][fp32 scales (K, V)]
+  static constexpr int OFF_VCODE = K_BYTES;
+  static constexpr int OFF_RAW = K_BYTES + CODE_BYTES;           // first raw slab
+  static constexpr int OFF_RAWV = OFF_RAW + (NSC - 1) * SCALE_SLAB;
+  static constexpr int OFF_SC32 = OFF_RAW + NSC * SCALE_SLAB;
+  static constexpr int OFF_SCV = OFF_SC32 + (NSC - 1) * SC_KV * 4;  // fp32 V scales
+  static constexpr int STAGE_BYTES = ((OFF_SC32 + NSC * SC_KV * 4 + 1023) / 1024) * 1024;
+  static constexpr uint32_t STAGE_TX = K_BYTES + CODE_BYTES + NSC * SCALE_SLAB;
   static constexpr int STAGES = D == 256 ? 3 : 4;
   static constexpr int QSTRIDE = D + 4;              // floats per staged q row (padded)
   static constexpr int SCRATCH = ((8 * QSTRIDE * 4 + 64 + 127) / 128) * 128;  // per consumer warp
   static constexpr int SWZ = RB == 128 ? 7 : RB == 64 ? 3 : RB == 32 ? 1 : 0;
+  // binary16 K: 128-byte lines (64 halves; one 64-byte line at D = 32), swizzled
+  static constexpr int KLINE = D < 64 ? 2 * D : 128;
+  static constexpr int KNCH = 2 * D / KLINE;         // lines per (token, head)
+  static constexpr int KSWZ = KLINE == 128 ? 7 : 3;
   static constexpr int OFF_SCRATCH = STAGES * STAGE_BYTES;
   static constexpr int OFF_BARS = OFF_SCRATCH + kConsumerWarps * SCRATCH;
   static constexpr int OFF_MISC = OFF_BARS + 3 * STAGES * 8;
   static constexpr int OFF_PREFIX = OFF_MISC + 64;
   static constexpr int SMEM_MAX = OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16;
   static_assert(T_TILE <= 256, "tensor-copy box limit");
-  static_assert(CODE_BYTES % 1024 == 0, "V block must stay swizzle-aligned");
+  static_assert(CODE_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "tiles must stay swizzle-aligned");
   static_assert((2 * NG * NT) % 4 == 0, "ldmatrix.x4 batches");
   static_assert(SMEM_MAX <= 232448, "shared memory per block");
+  static_assert(!KF16 || D <= 128, "binary16 K tiles up to head_dim 128");
 };
 
 // Workspace header: int64 prefix[batch + 1], int64 range_tokens.
@@ -198,11 +216,11 @@ struct TileWalker {
 // the query's binary16 hi/lo pieces of 4 heads in the 8 N columns, which halves
 // their count; otherwise the 8 heads' hi (rows 0-7) and lo (rows 8-15) pieces
 // are the M rows and the tokens the N columns.
-template <int D, int HKV, bool TOK_M>
+template <int D, int HKV, bool TOK_M, bool KF16>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap) {
-  using C = DecodeCfg<D, HKV>;
+  using C = DecodeCfg<D, HKV, KF16>;
   constexpr int NG = C::NG, RB = C::RB, T_TILE = C::T_TILE, UPW = C::UPW, NT = C::NT, KSP = C::KSP;
   constexpr int UNIT = C::UNIT, STAGES = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -273,12 +291,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* sb = smem + stage * C::STAGE_BYTES;
       mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
       const int row = (int)((int64_t)walk.b * p.max_seq + walk.t0);
-      tma_load_3d(sb, &kmap, &full[stage], 0, row, 0, pol);
-      tma_load_3d(sb + C::CODE_BYTES, &vmap, &full[stage], 0, row, 0, pol);
+      if constexpr (KF16)
+        tma_load_4d(sb, &kmap, &full[stage], 0, 0, row, 0, pol);
+      else
+        tma_load_3d(sb, &kmap, &full[stage], 0, row, 0, pol);
+      tma_load_3d(sb + C::OFF_VCODE, &vmap, &full[stage], 0, row, 0, pol);
       const int64_t soff = (int64_t)row * C::SROW;  // byte offset of the tile's first scale row
       const int64_t salign = soff & ~(int64_t)15;
-      bulk_load(sb + 2 * C::CODE_BYTES, ks_base + salign, C::SCALE_SLAB, &full[stage], pol);
-      bulk_load(sb + 2 * C::CODE_BYTES + C::SCALE_SLAB, vs_base + salign, C::SCALE_SLAB, &full[stage], pol);
+      if constexpr (!KF16) bulk_load(sb + C::OFF_RAW, ks_base + salign, C::SCALE_SLAB, &full[stage], pol);
+      bulk_load(sb + C::OFF_RAWV, vs_base + salign, C::SCALE_SLAB, &full[stage], pol);
       ++issued;
     }
     if (dead) {
@@ -336,10 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nv = min(T_TILE, walk.seg_hi - walk.t0);
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
 #pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
+        for (int kv = KF16 ? 1 : 0; kv < 2; ++kv) {  // binary16 K has no scales
           // plain (not volatile) shared loads: the compiler may issue a lane's loads together
-          const uint16_t* raw = reinterpret_cast<const uint16_t*>(sb + 2 * C::CODE_BYTES + kv * C::SCALE_SLAB + soff);
-          const uint32_t dst = sc + kv * C::SC_KV * 4;
+          const uint16_t* raw =
+              reinterpret_cast<const uint16_t*>(sb + (kv ? C::OFF_RAWV : C::OFF_RAW) + soff);
+          const uint32_t dst = kv ? smem_u32(sb + C::OFF_SCV) : sc;
 #pragma unroll
           for (int k = 0; k < ITEMS; ++k) {
             const int t = tok_of[k];
@@ -400,6 +422,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   static_assert((UNIT * RB) % 1024 == 0 || C::SWZ == 0 || (UNIT * RB) % ((C::SWZ + 1) * 128) == 0,
                 "unit rows must keep the swizzle phase");
+  // binary16 K: per-lane ldmatrix offsets of k-step kk inside the head's [tile][D]
+  // binary16 block, relative to the unit's first token (the unit and head offsets are
+  // whole multiples of the swizzle period). Row layout (K as B): matrix m = lane / 8
+  // is (8-token n-tile m / 2, dims + 8 (m % 2)); tokens-in-M (K as A): matrix m is
+  // (token rows 8 (m % 2) .., dims + 8 (m / 2)).
+  uint32_t k16_off[KF16 ? 2 * NG : 1];
+  if constexpr (KF16) {
+    const int m = lane >> 3, r = lane & 7;
+    const int tok = TOK_M ? (m & 1) * 8 + r : (m >> 1) * 8 + r;
+    const int dadd = TOK_M ? 8 * (m >> 1) : 8 * (m & 1);
+    constexpr int HPL = C::KLINE / 2;  // halves per line
+#pragma unroll
+    for (int kk = 0; kk < 2 * NG; ++kk) {
+      const int dims = 16 * kk + dadd;
+      const int ch = dims / HPL;
+      const int line = tok * C::KNCH + ch;
+      const int sw = ((line * C::KLINE) >> 7) & C::KSWZ;
+      k16_off[kk] = (uint32_t)(tok * C::KRB + ch * C::KLINE + ((((dims % HPL) >> 3) ^ sw) << 4));
+    }
+  }
+  static_assert(!KF16 || (UNIT % 16 == 0 && (T_TILE * C::KNCH) % 8 == 0), "binary16 K swizzle phase");
 
   uint32_t qA[NG][2][4];
   float biasK[NG];
@@ -417,7 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int HP = 32 / NG;  // heads rotated per pass
       const int part = lane % NG;
       const uint32_t sw = sign_word(p.sign_bits, part);
-      const float qs = p.c_d * p.sm_scale_log2;  // 1/sqrt(D) and the softmax scale in log2 units
+      // 1/sqrt(D) of the rotation and the softmax scale in log2 units; binary16 K is not
+      // rotated, so neither is q
+      const float qs = KF16 ? p.sm_scale_log2 : p.c_d * p.sm_scale_log2;
       for (int j0 = 0; j0 < 8 && j0 < G; j0 += HP) {  // rows j >= G are never read
         const int j = j0 + lane / NG;
         float u[32];
@@ -427,9 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) u[i] = 0.f;
         }
+        if constexpr (!KF16) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = flip_sign(u[i], sw, i);
-        fwht_group_x2<NG>(u, part);
+          for (int i = 0; i < 32; ++i) u[i] = flip_sign(u[i], sw, i);
+          fwht_group_x2<NG>(u, part);
+        }
         float mx = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -462,50 +509,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       // operand; otherwise head gid's hi (A rows 0-7) and lo (rows 8-15) pieces.
       const int qh = TOK_M ? (gid >> 1) : gid;
       const float* row = scratch + qh * C::QSTRIDE;
+      if constexpr (KF16) {
+        // binary16 K: natural k order, k-step kk covers dims 16 kk .. 16 kk + 15; the lane
+        // holds dims (2 tig, 2 tig + 1) and (8 + 2 tig, 9 + 2 tig) of it; no code offset
 #pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (qh < G) {
-          v0 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig);
-          v1 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig + 4);
-        }
-        const float qv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        // the code offset term -8 * sum(q) (the high-position pieces carry q / 16 against a
-        // 16x nibble, so every element enters with weight 1); q itself stands for its hi + lo
-        // pieces, which agree with it to 2^-22
-        float bsum = ((qv[0] + qv[1]) + (qv[2] + qv[3])) + ((qv[4] + qv[5]) + (qv[6] + qv[7]));
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const float2 lo = make_float2(qv[2 * ks], qv[2 * ks + 4]);
-          const float2 hi = __fmul2_rn(make_float2(qv[2 * ks + 1], qv[2 * ks + 5]), make_float2(0.0625f, 0.0625f));
-          const __half2 lo_h = __float22half2_rn(lo), hi_h = __float22half2_rn(hi);
-          // residual pieces: x - fp16(x) is exact in binary32, then rounded to binary16
-          const float2 lo_b = __half22float2(lo_h), hi_b = __half22float2(hi_h);
-          const __half2 lo_l = __float22half2_rn(make_float2(lo.x - lo_b.x, lo.y - lo_b.y));
-          const __half2 hi_l = __float22half2_rn(make_float2(hi.x - hi_b.x, hi.y - hi_b.y));
-          const uint32_t ah = *reinterpret_cast<const uint32_t*>(&lo_h);
-          const uint32_t al = *reinterpret_cast<const uint32_t*>(&lo_l);
-          const uint32_t ch = *reinterpret_cast<const uint32_t*>(&hi_h);
-          const uint32_t cl = *reinterpret_cast<const uint32_t*>(&hi_l);
+        for (int kk = 0; kk < 2 * NG; ++kk) {
+          float2 x0 = make_float2(0.f, 0.f), x1 = x0;
+          if (qh < G) {
+            x0 = *reinterpret_cast<const float2*>(row + 16 * kk + 2 * tig);
+            x1 = *reinterpret_cast<const float2*>(row + 16 * kk + 8 + 2 * tig);
+          }
+          const __half2 h0 = __float22half2_rn(x0), h1 = __float22half2_rn(x1);
+          const float2 b0f = __half22float2(h0), b1f = __half22float2(h1);
+          const __half2 l0 = __float22half2_rn(make_float2(x0.x - b0f.x, x0.y - b0f.y));
+          const __half2 l1 = __float22half2_rn(make_float2(x1.x - b1f.x, x1.y - b1f.y));
+          const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&h0), al0 = *reinterpret_cast<const uint32_t*>(&l0);
+          const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&h1), al1 = *reinterpret_cast<const uint32_t*>(&l1);
           if constexpr (TOK_M) {
-            qA[g][ks][0] = (gid & 1) ? al : ah;
-            qA[g][ks][1] = (gid & 1) ? cl : ch;
+            qA[kk / 2][kk % 2][0] = (gid & 1) ? al0 : ah0;
+            qA[kk / 2][kk % 2][1] = (gid & 1) ? al1 : ah1;
           } else {
-            qA[g][ks][0] = ah;
-            qA[g][ks][1] = al;
-            qA[g][ks][2] = ch;
-            qA[g][ks][3] = cl;
+            qA[kk / 2][kk % 2][0] = ah0;
+            qA[kk / 2][kk % 2][1] = al0;
+            qA[kk / 2][kk % 2][2] = ah1;
+            qA[kk / 2][kk % 2][3] = al1;
           }
         }
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
-        // TOK_M: the score lanes hold head tig, whose sum sits in lane 8 * tig (gid = 2 tig)
-        if constexpr (TOK_M) bsum = __shfl_sync(0xffffffffu, bsum, (8 * tig) & 31);
-        biasK[g] = -bsum * (8.0f * 5.9604644775390625e-08f);  // 8 * 2^-24
+#pragma unroll
+        for (int g = 0; g < NG; ++g) biasK[g] = 0.f;
+      } else {
+  #pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+          if (qh < G) {
+            v0 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig);
+            v1 = *reinterpret_cast<const float4*>(row + 32 * g + 8 * tig + 4);
+          }
+          const float qv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          // the code offset term -8 * sum(q) (the high-position pieces carry q / 16 against a
+          // 16x nibble, so every element enters with weight 1); q itself stands for its hi + lo
+          // pieces, which agree with it to 2^-22
+          float bsum = ((qv[0] + qv[1]) + (qv[2] + qv[3])) + ((qv[4] + qv[5]) + (qv[6] + qv[7]));
+  #pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const float2 lo = make_float2(qv[2 * ks], qv[2 * ks + 4]);
+            const float2 hi = __fmul2_rn(make_float2(qv[2 * ks + 1], qv[2 * ks + 5]), make_float2(0.0625f, 0.0625f));
+            const __half2 lo_h = __float22half2_rn(lo), hi_h = __float22half2_rn(hi);
+            // residual pieces: x - fp16(x) is exact in binary32, then rounded to binary16
+            const float2 lo_b = __half22float2(lo_h), hi_b = __half22float2(hi_h);
+            const __half2 lo_l = __float22half2_rn(make_float2(lo.x - lo_b.x, lo.y - lo_b.y));
+            const __half2 hi_l = __float22half2_rn(make_float2(hi.x - hi_b.x, hi.y - hi_b.y));
+            const uint32_t ah = *reinterpret_cast<const uint32_t*>(&lo_h);
+            const uint32_t al = *reinterpret_cast<const uint32_t*>(&lo_l);
+            const uint32_t ch = *reinterpret_cast<const uint32_t*>(&hi_h);
+            const uint32_t cl = *reinterpret_cast<const uint32_t*>(&hi_l);
+            if constexpr (TOK_M) {
+              qA[g][ks][0] = (gid & 1) ? al : ah;
+              qA[g][ks][1] = (gid & 1) ? cl : ch;
+            } else {
+              qA[g][ks][0] = ah;
+              qA[g][ks][1] = al;
+              qA[g][ks][2] = ch;
+              qA[g][ks][3] = cl;
+            }
+          }
+          bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
+          bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
+          // TOK_M: the score lanes hold head tig, whose sum sits in lane 8 * tig (gid = 2 tig)
+          if constexpr (TOK_M) bsum = __shfl_sync(0xffffffffu, bsum, (8 * tig) & 31);
+          biasK[g] = -bsum * (8.0f * 5.9604644775390625e-08f);  // 8 * 2^-24
+        }
       }
       const int sh_h = TOK_M ? tig : gid;  // the head of this lane's scores
       const int sh = (sh_h < G) ? reinterpret_cast<const int*>(scratch + 8 * C::QSTRIDE)[sh_h] : 0;
-      f_h = __int_as_float((127 + 24 - sh) << 23);  // 2^(24 - sh): MMA units -> log2 units
+      // MMA units -> log2 units: 2^(24 - sh) for the subnormal-coded nibbles, 2^-sh for binary16 K
+      f_h = __int_as_float((127 + (KF16 ? 0 : 24) - sh) << 23);
       __syncwarp();
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
@@ -533,10 +611,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!dead) {
         const uint32_t sbase = smem_base + stage * C::STAGE_BYTES;
-        const uint32_t kc = sbase + h * T_TILE * RB;
-        const uint32_t vc = sbase + C::CODE_BYTES + h * T_TILE * RB;
+        const uint32_t kc = sbase + h * T_TILE * C::KRB;
+        const uint32_t vc = sbase + C::OFF_VCODE + h * T_TILE * RB;
         const uint32_t sck = sbase + C::OFF_SC32 + 4 * h * C::SC_HEAD;
-        const uint32_t scv = sck + 4 * C::SC_KV;
+        const uint32_t scv = sbase + C::OFF_SCV + 4 * h * C::SC_HEAD;
         // tokens of the segment left in this tile, from this warp's first row on
         const int left = min(T_TILE, seg_hi - walk.t0) - sub * UPW * UNIT;
 #pragma unroll 1
@@ -557,48 +635,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             float2 s2[MT];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) s2[mt] = make_float2(0.f, 0.f);
+            if constexpr (KF16) {
+              // A = binary16 K rows (tokens) straight from ldmatrix, B = q pieces; no scales
 #pragma unroll
-            for (int g4 = 0; g4 < NG * NT; g4 += 4) {
-              uint32_t kw[4];
-              ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
-              float skm[4 / NT > 0 ? 4 / NT : 1][2 * MT];
+              for (int mt = 0; mt < MT; ++mt) {
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
-                const int g = g4 / NT + gi;
-                const uint32_t a0 = sck + 4 * (((uu * NG + g) * 8 + gid) * (2 * MT));
-                if constexpr (MT == 2) {
-                  const float4 v = lds_f4(a0);
-                  skm[gi][0] = v.x;
-                  skm[gi][1] = v.y;
-                  skm[gi][2] = v.z;
-                  skm[gi][3] = v.w;
-                } else {
-                  const float2 v = lds_f2(a0);
-                  skm[gi][0] = v.x;
-                  skm[gi][1] = v.y;
+                for (int kk = 0; kk < 2 * NG; ++kk) {
+                  uint32_t kw[4];
+                  ldmatrix_x4(kw, kc + (r0 + 16 * mt) * C::KRB + k16_off[kk]);
+                  mma_f16_16816_acc(c, kw, qA[kk / 2][kk % 2][0], qA[kk / 2][kk % 2][1]);
                 }
+                s2[mt] = make_float2(c[0] + c[1], c[2] + c[3]);  // hi + lo columns
               }
-#pragma unroll
-              for (int i = 0; i < 4; i += 2) {
-                const int g = (g4 + i) / NT, mt = ((g4 + i) % NT) >> 1;
-                const int gi = g - g4 / NT;
-                const uint32_t wa = kw[i], wb = kw[i + 1];  // tokens gid and gid + 8 of m-tile mt
-                float c[4];
-                uint32_t a[4];
-                a[0] = and_xor(wa, 0x000F000Fu, 0x00080008u);
-                a[1] = and_xor(wb, 0x000F000Fu, 0x00080008u);
-                a[2] = and_xor(wa, 0x00F000F0u, 0x00800080u);
-                a[3] = and_xor(wb, 0x00F000F0u, 0x00800080u);
-                mma_f16_16816_c(c, a, qA[g][0][0], qA[g][0][1], 0.f, 0.f, 0.f, 0.f);
-                const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
-                a[0] = and_xor(wa8, 0x000F000Fu, 0x00080008u);
-                a[1] = and_xor(wb8, 0x000F000Fu, 0x00080008u);
-                a[2] = and_xor(wa8, 0x00F000F0u, 0x00800080u);
-                a[3] = and_xor(wb8, 0x00F000F0u, 0x00800080u);
-                mma_f16_16816_acc(c, a, qA[g][1][0], qA[g][1][1]);
-                // hi + lo columns, plus the offset term -8 * sum(q) of the offset-binary code
-                const float2 x = __fadd2_rn(make_float2(c[0] + c[1], c[2] + c[3]), make_float2(biasK[g], biasK[g]));
-                s2[mt] = __ffma2_rn(make_float2(skm[gi][2 * mt], skm[gi][2 * mt + 1]), x, s2[mt]);
+            } else {
+
+  #pragma unroll
+              for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+                uint32_t kw[4];
+                ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
+                float skm[4 / NT > 0 ? 4 / NT : 1][2 * MT];
+  #pragma unroll
+                for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
+                  const int g = g4 / NT + gi;
+                  const uint32_t a0 = sck + 4 * (((uu * NG + g) * 8 + gid) * (2 * MT));
+                  if constexpr (MT == 2) {
+                    const float4 v = lds_f4(a0);
+                    skm[gi][0] = v.x;
+                    skm[gi][1] = v.y;
+                    skm[gi][2] = v.z;
+                    skm[gi][3] = v.w;
+                  } else {
+                    const float2 v = lds_f2(a0);
+                    skm[gi][0] = v.x;
+                    skm[gi][1] = v.y;
+                  }
+                }
+  #pragma unroll
+                for (int i = 0; i < 4; i += 2) {
+                  const int g = (g4 + i) / NT, mt = ((g4 + i) % NT) >> 1;
+                  const int gi = g - g4 / NT;
+                  const uint32_t wa = kw[i], wb = kw[i + 1];  // tokens gid and gid + 8 of m-tile mt
+                  float c[4];
+                  uint32_t a[4];
+                  a[0] = and_xor(wa, 0x000F000Fu, 0x00080008u);
+                  a[1] = and_xor(wb, 0x000F000Fu, 0x00080008u);
+                  a[2] = and_xor(wa, 0x00F000F0u, 0x00800080u);
+                  a[3] = and_xor(wb, 0x00F000F0u, 0x00800080u);
+                  mma_f16_16816_c(c, a, qA[g][0][0], qA[g][0][1], 0.f, 0.f, 0.f, 0.f);
+                  const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+                  a[0] = and_xor(wa8, 0x000F000Fu, 0x00080008u);
+                  a[1] = and_xor(wb8, 0x000F000Fu, 0x00080008u);
+                  a[2] = and_xor(wa8, 0x00F000F0u, 0x00800080u);
+                  a[3] = and_xor(wb8, 0x00F000F0u, 0x00800080u);
+                  mma_f16_16816_acc(c, a, qA[g][1][0], qA[g][1][1]);
+                  // hi + lo columns, plus the offset term -8 * sum(q) of the offset-binary code
+                  const float2 x = __fadd2_rn(make_float2(c[0] + c[1], c[2] + c[3]), make_float2(biasK[g], biasK[g]));
+                  s2[mt] = __ffma2_rn(make_float2(skm[gi][2 * mt], skm[gi][2 * mt + 1]), x, s2[mt]);
+                }
               }
             }
             if (nv < UNIT) {
@@ -663,44 +757,66 @@ __global__ void __launch_bounds__(kThreads, 1)
               s2[nt] = make_float2(0.f, 0.f);
               s2b[nt] = make_float2(0.f, 0.f);
             }
-  #pragma unroll
-            for (int g4 = 0; g4 < NG * NT; g4 += 4) {
-              uint32_t kw[4];
-              ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
-              // this lane's K scales for the groups of this batch: (n-tile, e) pairs
-              float skv[4 / NT > 0 ? 4 / NT : 1][2 * NT];
-  #pragma unroll
-              for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
-                const int g = g4 / NT + gi;
-                const uint32_t a0 = sck + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT));
-  #pragma unroll
-                for (int q4 = 0; q4 < 2 * NT; q4 += 4) {
-                  const float4 v = lds_f4(a0 + 4 * q4);
-                  skv[gi][q4] = v.x;
-                  skv[gi][q4 + 1] = v.y;
-                  skv[gi][q4 + 2] = v.z;
-                  skv[gi][q4 + 3] = v.w;
+            if constexpr (KF16) {
+              // B = binary16 K (8 tokens x 16 dims per n-tile and k-step) straight from
+              // ldmatrix; one accumulator per n-tile over all k-steps; no scales
+              static_assert(NT % 2 == 0, "binary16 K row layout: n-tile pairs");
+              float c[NT][4];
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+#pragma unroll
+              for (int kk = 0; kk < 2 * NG; ++kk) {
+#pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                  uint32_t kw[4];
+                  ldmatrix_x4(kw, kc + (r0 + 16 * np) * C::KRB + k16_off[kk]);
+                  mma_f16_16816_acc(c[2 * np], qA[kk / 2][kk % 2], kw[0], kw[1]);
+                  mma_f16_16816_acc(c[2 * np + 1], qA[kk / 2][kk % 2], kw[2], kw[3]);
                 }
               }
-  #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int g = (g4 + i) / NT, nt = (g4 + i) % NT;
-                const int gi = g - g4 / NT;
-                const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
-                float c[4];
-                const uint32_t w = kw[i];
-                mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
-                                0.f, 0.f, 0.f, 0.f);
-                const uint32_t w8 = w >> 8;
-                mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
-                                  and_xor(w8, 0x00F000F0u, 0x00800080u));
-                // hi + lo rows, plus the offset term -8 * sum(q) of the offset-binary code
-                const float2 x = __fadd2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
-                                            make_float2(biasK[g], biasK[g]));
-                if (g & 1)
-                  s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
-                else
-                  s2[nt] = __ffma2_rn(sk, x, s2[nt]);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)  // hi + lo rows
+                s2[nt] = __fadd2_rn(make_float2(c[nt][0], c[nt][1]), make_float2(c[nt][2], c[nt][3]));
+            } else {
+    #pragma unroll
+              for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+                uint32_t kw[4];
+                ldmatrix_x4(kw, kc + r0 * RB + k_off[g4 / 4]);
+                // this lane's K scales for the groups of this batch: (n-tile, e) pairs
+                float skv[4 / NT > 0 ? 4 / NT : 1][2 * NT];
+    #pragma unroll
+                for (int gi = 0; gi < (4 / NT > 0 ? 4 / NT : 1); ++gi) {
+                  const int g = g4 / NT + gi;
+                  const uint32_t a0 = sck + 4 * (((uu * NG + g) * 4 + tig) * (2 * NT));
+    #pragma unroll
+                  for (int q4 = 0; q4 < 2 * NT; q4 += 4) {
+                    const float4 v = lds_f4(a0 + 4 * q4);
+                    skv[gi][q4] = v.x;
+                    skv[gi][q4 + 1] = v.y;
+                    skv[gi][q4 + 2] = v.z;
+                    skv[gi][q4 + 3] = v.w;
+                  }
+                }
+    #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int g = (g4 + i) / NT, nt = (g4 + i) % NT;
+                  const int gi = g - g4 / NT;
+                  const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
+                  float c[4];
+                  const uint32_t w = kw[i];
+                  mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
+                                  0.f, 0.f, 0.f, 0.f);
+                  const uint32_t w8 = w >> 8;
+                  mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
+                                    and_xor(w8, 0x00F000F0u, 0x00800080u));
+                  // hi + lo rows, plus the offset term -8 * sum(q) of the offset-binary code
+                  const float2 x = __fadd2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
+                                              make_float2(biasK[g], biasK[g]));
+                  if (g & 1)
+                    s2b[nt] = __ffma2_rn(sk, x, s2b[nt]);
+                  else
+                    s2[nt] = __ffma2_rn(sk, x, s2[nt]);
+                }
               }
             }
   #pragma unroll
@@ -1044,14 +1160,14 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   }
 }
 
-template <int D, int HKV, bool TOK_M>
+template <int D, int HKV, bool TOK_M, bool KF16>
 static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
                                     cudaStream_t s, cudaEvent_t ev) {
-  using C = DecodeCfg<D, HKV>;
+  using C = DecodeCfg<D, HKV, KF16>;
   const int smem = C::OFF_PREFIX + 8 * (p.batch + 1) + 8 * 16;
   static bool attr_set = false;  // per instantiation; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV, TOK_M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV, TOK_M, KF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_MAX);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -1068,7 +1184,7 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   kattr[0].val.programmaticStreamSerializationAllowed = 1;
   kcfg.attrs = kattr;
   kcfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M>, p, kmap, vmap);
+  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M, KF16>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
   const bool few = (int64_t)p.batch * p.n_q < 2 * (int64_t)p.grid;  // merge blocks vs SMs
   if (ev != nullptr) {  // timing split: plain stream order between the two kernels
@@ -1099,8 +1215,16 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
 template <int D, int HKV>
 static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
                                     cudaStream_t s, cudaEvent_t ev) {
-  if (p.group <= 4) return launch_decode_dht<D, HKV, true>(p, km, vm, s, ev);
-  return launch_decode_dht<D, HKV, false>(p, km, vm, s, ev);
+  if constexpr (D <= 128) {
+    if (p.k_f16) {
+      if (p.group <= 4) return launch_decode_dht<D, HKV, true, true>(p, km, vm, s, ev);
+      return launch_decode_dht<D, HKV, false, true>(p, km, vm, s, ev);
+    }
+  } else {
+    if (p.k_f16) return cudaErrorInvalidValue;  // binary16 K tiles: head_dim <= 128
+  }
+  if (p.group <= 4) return launch_decode_dht<D, HKV, true, false>(p, km, vm, s, ev);
+  return launch_decode_dht<D, HKV, false, false>(p, km, vm, s, ev);
 }
 
 template <int D>
@@ -1126,9 +1250,12 @@ cudaError_t launch_decode(const DecodeParams& p, const TensorMap128& km, const T
   return cudaErrorInvalidValue;
 }
 
-int decode_tile_tokens(int D, int n_kv) {
-#define TQ_TT(DD, HH) \
-  if (D == DD && n_kv == HH) return DecodeCfg<DD, HH>::T_TILE;
+int decode_tile_tokens(int D, int n_kv, int k_f16) {
+#define TQ_TT(DD, HH)                                                          \
+  if (D == DD && n_kv == HH) {                                                 \
+    if (k_f16) return DD <= 128 ? DecodeCfg<(DD <= 128 ? DD : 128), HH, true>::T_TILE : 0; \
+    return DecodeCfg<DD, HH>::T_TILE;                                          \
+  }
   TQ_TT(32, 1) TQ_TT(32, 2) TQ_TT(32, 4) TQ_TT(32, 8)
   TQ_TT(64, 1) TQ_TT(64, 2) TQ_TT(64, 4) TQ_TT(64, 8)
   TQ_TT(128, 1) TQ_TT(128, 2) TQ_TT(128, 4) TQ_TT(128, 8)
@@ -1137,9 +1264,14 @@ int decode_tile_tokens(int D, int n_kv) {
   return 0;
 }
 
-int decode_smem_bytes(int D, int n_kv) {
-#define TQ_SM(DD, HH) \
-  if (D == DD && n_kv == HH) return DecodeCfg<DD, HH>::OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16;
+int decode_smem_bytes(int D, int n_kv, int k_f16) {
+#define TQ_SM(DD, HH)                                                                                     \
+  if (D == DD && n_kv == HH) {                                                                            \
+    if (k_f16)                                                                                            \
+      return DD <= 128 ? DecodeCfg<(DD <= 128 ? DD : 128), HH, true>::OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16 \
+                       : 0;                                                                               \
+    return DecodeCfg<DD, HH>::OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16;                                  \
+  }
   TQ_SM(32, 1) TQ_SM(32, 2) TQ_SM(32, 4) TQ_SM(32, 8)
   TQ_SM(64, 1) TQ_SM(64, 2) TQ_SM(64, 4) TQ_SM(64, 8)
   TQ_SM(128, 1) TQ_SM(128, 2) TQ_SM(128, 4) TQ_SM(128, 8)

@@ -19,6 +19,7 @@ struct QuantizeParams {
   int32_t* status;
   uint64_t sign_bits[4];
   float c_d;
+  int k_f16;  // 1: K is stored as binary16 of the input (k_codes is that buffer), k_scales unused
 };
 
 struct DequantParams {
@@ -53,13 +54,14 @@ struct DecodeParams {
   float sm_scale_log2; // sm_scale * log2(e)
   float c_d;
   uint64_t sign_bits[4];
+  int k_f16;  // 1: K tiles are binary16 (original domain), no K scales
 };
 
 cudaError_t launch_quantize(const QuantizeParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, const TensorMap128& kmap, const TensorMap128& vmap, int head_dim,
                           cudaStream_t s, cudaEvent_t after_split);
-int decode_smem_bytes(int head_dim, int n_kv);
-int decode_tile_tokens(int head_dim, int n_kv);
+int decode_smem_bytes(int head_dim, int n_kv, int k_f16);
+int decode_tile_tokens(int head_dim, int n_kv, int k_f16);
 
 }  // namespace tqk

@@ -23,6 +23,39 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
+// Asymmetric cache (mlxcel guide, cache modes: K kept in FP16): thread kt stores
+// the binary16 (round to nearest even) of 32 consecutive K elements.
+template <int D>
+__device__ __forceinline__ void copy_k_f16(const QuantizeParams& p, int64_t kt) {
+  constexpr int NG = D / 32;
+  const int64_t r = kt / NG;
+  const int part = (int)(kt % NG);
+  const int h = (int)(r % p.n_kv);
+  const int64_t bt = r / p.n_kv;
+  const int t = (int)(bt % p.n_new);
+  const int b = (int)(bt / p.n_new);
+  float u[32];
+  load32(u, p.k, r * D + part * 32, p.in_dtype);
+  const int64_t pos = p.start_pos[b];
+  if (pos < 0 || pos + p.n_new > p.max_seq) {
+    if (t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
+    return;
+  }
+  uint32_t w[16];
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const __half2 hv = __floats2half2_rn(u[2 * i], u[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    finite = finite && ((w[i] & 0x7C00u) != 0x7C00u) && ((w[i] & 0x7C000000u) != 0x7C000000u);
+  }
+  if (!finite) status_or(p.status, TQ_STATUS_NONFINITE);
+  const int64_t row = ((int64_t)b * p.max_seq + pos + t) * p.n_kv + h;
+  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.k_codes) + row * D + part * 32);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantizeParams p) {
   // Launched as a programmatic dependent of the previous kernel on the stream:
@@ -33,8 +66,19 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
   constexpr int NG = D / 32;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t vecs_per_tensor = (int64_t)p.batch * p.n_new * p.n_kv;
-  const int64_t vec = gt / NG;
+  const int64_t thr_per_tensor = vecs_per_tensor * NG;
+  int64_t vec = gt / NG;
   const int part = (int)(gt % NG);
+  if (p.k_f16) {
+    // V threads first, then the K copies from the next warp boundary on, so that a
+    // warp is all V (its lanes exchange butterflies) or all K.
+    const int64_t kbase = (thr_per_tensor + 31) / 32 * 32;
+    if (gt >= kbase) {
+      if (gt - kbase < thr_per_tensor) copy_k_f16<D>(p, gt - kbase);
+      return;
+    }
+    vec = gt < thr_per_tensor ? vecs_per_tensor + vec : 2 * vecs_per_tensor;  // V; the rest pads the warp
+  }
   const bool in_range = vec < 2 * vecs_per_tensor;
   const int which = in_range ? (int)(vec / vecs_per_tensor) : 0;  // 0 = K, 1 = V
   const int64_t r = in_range ? vec % vecs_per_tensor : 0;
@@ -177,7 +221,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__
 
 template <int D>
 static cudaError_t launch_quantize_d(const QuantizeParams& p, cudaStream_t s) {
-  const int64_t threads = 2LL * p.batch * p.n_new * p.n_kv * (D / 32);
+  const int64_t per_tensor = (int64_t)p.batch * p.n_new * p.n_kv * (D / 32);
+  const int64_t threads = p.k_f16 ? (per_tensor + 31) / 32 * 32 + per_tensor : 2 * per_tensor;
   const int64_t blocks = (threads + 255) / 256;
   // programmatic dependent launch: set-up overlaps the previous kernel's tail,
   // griddepcontrol.wait in the kernel orders the reads

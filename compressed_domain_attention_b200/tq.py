@@ -24,8 +24,10 @@ TQ_STATUS_TIMEOUT = 4
 
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
+TQ_K_INT4, TQ_K_FP16 = 0, 1  # K storage format (V is always int4 codes + binary16 scales)
+
 # C symbols declared in include/tq.h
-EXPORTS = ("tq_cache_layout", "tq_quantize_append", "tq_decode_attention", "tq_decode_attention_ex",
+EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_quantize_append", "tq_decode_attention", "tq_decode_attention_ex",
            "tq_decode_attention_noalloc", "tq_dequantize_debug", "tq_status_string", "tq_last_cuda_error")
 
 TQ_NOALLOC_WORKSPACE_BYTES = 8 << 20
@@ -41,7 +43,8 @@ class TqLayout(ctypes.Structure):
         ("scale_stride_tok", ctypes.c_int64), ("scale_stride_seq", ctypes.c_int64),
         ("codes_bytes", ctypes.c_uint64), ("scales_bytes", ctypes.c_uint64),
         ("decode_workspace_bytes", ctypes.c_uint64),
-        ("max_ctas", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("max_ctas", ctypes.c_int32), ("k_format", ctypes.c_int32),
+        ("k_bytes", ctypes.c_uint64), ("k_stride_tok", ctypes.c_int64), ("k_stride_seq", ctypes.c_int64),
     ]
 
 
@@ -72,6 +75,8 @@ def _lib():
         P, I, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
         lib.tq_cache_layout.argtypes = [I, I, I, I, I, I, U64, ctypes.POINTER(TqLayout)]
         lib.tq_cache_layout.restype = I
+        lib.tq_cache_layout_kv.argtypes = [I, I, I, I, I, I, U64, I, ctypes.POINTER(TqLayout)]
+        lib.tq_cache_layout_kv.restype = I
         lib.tq_quantize_append.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
         lib.tq_quantize_append.restype = I
         lib.tq_decode_attention.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float, P, P,
@@ -123,6 +128,16 @@ def tq_cache_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size=
     return out
 
 
+def tq_cache_layout_kv(batch, max_seq, n_kv_heads, n_q_heads, head_dim, k_format, group_size=32,
+                       sign_seed=0) -> TqLayout:
+    """Layout with the K storage format: TQ_K_INT4 (symmetric) or TQ_K_FP16 (binary16 K, int4 V)."""
+    out = TqLayout()
+    _check("tq_cache_layout_kv", _lib().tq_cache_layout_kv(batch, max_seq, n_kv_heads, n_q_heads, head_dim,
+                                                           group_size, ctypes.c_uint64(sign_seed), int(k_format),
+                                                           ctypes.byref(out)))
+    return out
+
+
 def tq_cache_layout_status(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size=32, sign_seed=0):
     """Raw status code variant (for callers that test rejection paths)."""
     out = TqLayout()
@@ -135,7 +150,7 @@ def tq_quantize_append(layout, k, v, n_new, start_pos, k_codes, k_scales, v_code
                        stream=None):
     """k, v: [batch][n_new][Hkv][D] (f32/bf16/f16, CUDA, contiguous); start_pos: int32 [batch] on the device."""
     for t in (k, v, start_pos, k_codes, k_scales, v_codes, v_scales):
-        assert t.is_contiguous()
+        assert t is None or t.is_contiguous()
     code = _lib().tq_quantize_append(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
                                      _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
                                      _ptr(v_scales), _ptr(status), _stream(stream))
@@ -146,7 +161,7 @@ def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scale
                         status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None):
     """q: [batch][Hq][D]; out: float32 [batch][Hq][D]; workspace: >= layout.decode_workspace_bytes bytes."""
     for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out, workspace):
-        assert t.is_contiguous()
+        assert t is None or t.is_contiguous()
     ws_bytes = workspace.numel() * workspace.element_size()
     lib = _lib()
     if min_split_tokens or max_ctas or after_split_event is not None:
@@ -175,7 +190,7 @@ def tq_decode_attention_noalloc(layout, q, seq_lens, k_codes, k_scales, v_codes,
     scratch than the array holds.
     """
     for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out):
-        assert t.is_contiguous()
+        assert t is None or t.is_contiguous()
     code = _lib().tq_decode_attention_noalloc(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
                                               _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
                                               ctypes.c_float(sm_scale), _ptr(out), _ptr(status), _stream(stream))
@@ -194,13 +209,20 @@ def sign_vector(layout):
 
 
 def alloc_cache(layout, device="cuda"):
-    """Allocate (k_codes, k_scales, v_codes, v_scales) with the layout's sizes (zero-filled)."""
+    """Allocate (k_codes, k_scales, v_codes, v_scales) with the layout's sizes (zero-filled).
+
+    With layout.k_format == TQ_K_FP16, k_codes is the binary16 K buffer (k_bytes) and
+    k_scales is None.
+    """
     import torch
     cb = int(layout.codes_bytes)
     sb = int(layout.scales_bytes)
-    k_codes = torch.zeros(cb, dtype=torch.uint8, device=device)
+    k_codes = torch.zeros(int(layout.k_bytes), dtype=torch.uint8, device=device)
     v_codes = torch.zeros(cb, dtype=torch.uint8, device=device)
-    k_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
+    if layout.k_format == TQ_K_FP16:
+        k_scales = None
+    else:
+        k_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
     v_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
     return k_codes, k_scales, v_codes, v_scales
 

@@ -17,6 +17,9 @@
  *    rejected when the cache is created).
  *  - "TurboQuant on AMD GPUs", §4: the Walsh-Hadamard transform is used as the
  *    rotation because it spreads energy evenly and suits GPU kernels.
+ *  - the mlxcel guide, §"Cache modes": the recommended default mode keeps K in
+ *    FP16 and compresses only V (K decides where attention looks, V is mixed
+ *    after); that asymmetric cache is TQ_K_FP16 below.
  *
  * Conventions fixed by this library where the pages are silent:
  *  - rotation: y = c_D * H * (s o x), H the Sylvester Hadamard matrix applied
@@ -31,6 +34,9 @@
  * and keeps no state between calls):
  *  - codes  [batch][max_seq][n_kv_heads][head_dim/2]  uint8   (one buffer for K, one for V)
  *  - scales [batch][max_seq][n_kv_heads][head_dim/32] binary16 bits (one for K, one for V)
+ *  - with k_format TQ_K_FP16, K is instead one binary16 buffer
+ *    [batch][max_seq][n_kv_heads][head_dim] (k_bytes) in the original domain and
+ *    has no scales; V keeps its codes and scales.
  *    Allocate `scales_bytes` (slightly more than the array): decode reads
  *    scale rows in tile-sized blocks that may run past the last valid token.
  *  - every device buffer must be 16-byte aligned (cudaMalloc gives 256).
@@ -67,6 +73,12 @@ typedef enum {
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 
+/* How K is stored (V is always rotated int4 codes + binary16 group scales). */
+typedef enum {
+  TQ_K_INT4 = 0, /* K encoded like V (the symmetric cache) */
+  TQ_K_FP16 = 1  /* K as binary16 (round to nearest even) of the input, original domain */
+} tq_k_format;
+
 /* Filled by tq_cache_layout; plain data, caller-owned, never modified by the library. */
 typedef struct {
   int32_t batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size;
@@ -82,7 +94,10 @@ typedef struct {
   uint64_t scales_bytes;       /* allocation size of ONE scales buffer, including read-ahead padding */
   uint64_t decode_workspace_bytes; /* workspace tq_decode_attention needs with default options */
   int32_t max_ctas;            /* largest split-K grid the workspace size allows */
-  int32_t reserved;
+  int32_t k_format;            /* tq_k_format */
+  uint64_t k_bytes;            /* allocation size of the K buffer (codes_bytes for TQ_K_INT4) */
+  int64_t k_stride_tok;        /* bytes between tokens of one sequence in the K buffer */
+  int64_t k_stride_seq;        /* bytes between sequences in the K buffer */
 } tq_layout_t;
 
 /* Optional knobs for tq_decode_attention_ex (NULL = defaults). */
@@ -103,6 +118,16 @@ int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int h
                     int group_size, uint64_t sign_seed, tq_layout_t* out);
 
 /*
+ * As tq_cache_layout, with the K storage format (tq_k_format). TQ_K_FP16 is the
+ * asymmetric cache of the mlxcel guide's recommended mode: K kept as binary16
+ * (an input beyond the binary16 range is stored as +-inf and sets
+ * TQ_STATUS_NONFINITE), V compressed. tq_cache_layout(...) equals
+ * tq_cache_layout_kv(..., TQ_K_INT4, out). Unknown formats: TQ_ERR_INVALID_ARG.
+ */
+int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim,
+                       int group_size, uint64_t sign_seed, int k_format, tq_layout_t* out);
+
+/*
  * Quantise and append n_new tokens to every sequence (Open-TQ-Metal abstract:
  * the fused sign-randomised transform + per-group abs-max + int4 nibble pack,
  * run when the cache is appended to).
@@ -111,7 +136,9 @@ int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int h
  *                position d_start_pos[b] + t. A sequence whose append would
  *                pass max_seq (or a negative start) is skipped and sets
  *                TQ_STATUS_CAPACITY.
- *   k_codes, v_codes, k_scales, v_scales   device caches (layout above).
+ *   k_codes, v_codes, k_scales, v_scales   device caches (layout above). With
+ *                layout->k_format == TQ_K_FP16, k_codes is the binary16 K buffer
+ *                and k_scales is not used (may be NULL).
  * n_new == 0 is a no-op. Codes and scales are bit-exact with the reference
  * definition (IEEE binary32 steps, no contraction, round-half-even).
  */
@@ -134,7 +161,10 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
  *                ever written)
  * The query is rotated by the same transform, K and V nibbles are unpacked in
  * registers, softmax runs online over split-K token ranges, the partials are
- * merged, and one inverse transform produces the output.
+ * merged, and one inverse transform produces the output. With
+ * layout->k_format == TQ_K_FP16, k_codes is the binary16 K buffer (k_scales
+ * unused, may be NULL): the scores use the unrotated query against it, the V
+ * side is unchanged.
  * Limits: batch <= 1024; n_kv_heads in {1, 2, 4, 8}; n_q_heads / n_kv_heads <= 8
  * (otherwise TQ_ERR_UNSUPPORTED).
  */

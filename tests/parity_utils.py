@@ -17,17 +17,18 @@ def np_f32(t):
 class GpuCache:
     """A packed K/V cache in device memory laid out by tq_cache_layout."""
 
-    def __init__(self, batch, max_seq, n_kv, n_q, D, sign_seed=0, device="cuda"):
-        self.layout = tq.tq_cache_layout(batch, max_seq, n_kv, n_q, D, 32, sign_seed)
+    def __init__(self, batch, max_seq, n_kv, n_q, D, sign_seed=0, device="cuda", k_format=tq.TQ_K_INT4):
+        self.layout = tq.tq_cache_layout_kv(batch, max_seq, n_kv, n_q, D, k_format, 32, sign_seed)
         self.k_codes, self.k_scales, self.v_codes, self.v_scales = tq.alloc_cache(self.layout, device)
         self.device = device
+        self.kf16 = k_format == tq.TQ_K_FP16
 
     def seq_view(self, b):
         """(layout, k_codes, k_scales, v_codes, v_scales) for sequence b alone (a batch-1 view)."""
         L = self.layout
-        l1 = tq.tq_cache_layout(1, L.max_seq, L.n_kv_heads, L.n_q_heads, L.head_dim, 32, L.sign_seed)
-        cs, ss = int(L.code_stride_seq), int(L.scale_stride_seq)
-        return (l1, self.k_codes[b * cs:(b + 1) * cs], self.k_scales[b * ss:],
+        l1 = tq.tq_cache_layout_kv(1, L.max_seq, L.n_kv_heads, L.n_q_heads, L.head_dim, L.k_format, 32, L.sign_seed)
+        cs, ss, ks_ = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
+        return (l1, self.k_codes[b * ks_:(b + 1) * ks_], None if self.kf16 else self.k_scales[b * ss:],
                 self.v_codes[b * cs:(b + 1) * cs], self.v_scales[b * ss:])
 
     def append_seq(self, b, k, v, start, status=None):
@@ -47,9 +48,13 @@ class GpuCache:
         L = self.layout
         B, S, H, D = L.batch, L.max_seq, L.n_kv_heads, L.head_dim
         n_s = B * S * H * (D // 32)
-        kc = self.k_codes.cpu().numpy().reshape(B, S, H, D // 2)
         vc = self.v_codes.cpu().numpy().reshape(B, S, H, D // 2)
-        ks = self.k_scales[:n_s].cpu().numpy().view(np.uint16).reshape(B, S, H, D // 32)
+        if self.kf16:  # binary16 K bits [B][S][H][D], no K scales
+            kc = self.k_codes.cpu().numpy().view(np.uint16).reshape(B, S, H, D)
+            ks = None
+        else:
+            kc = self.k_codes.cpu().numpy().reshape(B, S, H, D // 2)
+            ks = self.k_scales[:n_s].cpu().numpy().view(np.uint16).reshape(B, S, H, D // 32)
         vs = self.v_scales[:n_s].cpu().numpy().view(np.uint16).reshape(B, S, H, D // 32)
         return kc, ks, vc, vs
 
@@ -64,19 +69,32 @@ class GpuCache:
 
 
 class OracleCache:
-    def __init__(self, batch, max_seq, n_kv, D, sign_seed=0):
+    def __init__(self, batch, max_seq, n_kv, D, sign_seed=0, kf16=False):
         self.signs = oracle.sign_vector(sign_seed, D)
-        self.kc, self.ks = oracle.new_cache(batch, max_seq, n_kv, D)
+        self.kf16 = kf16
+        if kf16:
+            self.kc, self.ks = oracle.new_k16_cache(batch, max_seq, n_kv, D), None
+        else:
+            self.kc, self.ks = oracle.new_cache(batch, max_seq, n_kv, D)
         self.vc, self.vs = oracle.new_cache(batch, max_seq, n_kv, D)
 
     def append_seq(self, b, k, v, start):
-        st = oracle.quantize_append(self.signs, np_f32(k)[None], np_f32(v)[None], np.array([start], np.int32),
-                                    self.kc[b:b + 1], self.ks[b:b + 1], self.vc[b:b + 1], self.vs[b:b + 1])
+        sp = np.array([start], np.int32)
+        if self.kf16:
+            st = oracle.quantize_append_kf16(self.signs, np_f32(k)[None], np_f32(v)[None], sp, self.kc[b:b + 1],
+                                             self.vc[b:b + 1], self.vs[b:b + 1])
+        else:
+            st = oracle.quantize_append(self.signs, np_f32(k)[None], np_f32(v)[None], sp, self.kc[b:b + 1],
+                                        self.ks[b:b + 1], self.vc[b:b + 1], self.vs[b:b + 1])
         assert st == 0
 
     def decode(self, q, seq_lens, sm_scale, which=None):
-        out, st = oracle.decode_attention(self.signs, np_f32(q), np.asarray(seq_lens, np.int32), self.kc, self.ks,
-                                          self.vc, self.vs, sm_scale, which)
+        lens = np.asarray(seq_lens, np.int32)
+        if self.kf16:
+            return oracle.decode_attention_kf16(self.signs, np_f32(q), lens, self.kc, self.vc, self.vs, sm_scale,
+                                                which)
+        out, st = oracle.decode_attention(self.signs, np_f32(q), lens, self.kc, self.ks, self.vc, self.vs, sm_scale,
+                                          which)
         return out, st
 
 

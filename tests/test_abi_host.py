@@ -157,3 +157,22 @@ def test_status_strings(lib):
     for code in (0, -1, -2, -3, -4, 99):
         assert isinstance(lib.tq_status_string(code), bytes)
     assert lib.tq_status_string(-2) == b"unsupported shape"
+
+
+def test_layout_kv_formats():
+    L4 = tq.tq_cache_layout(3, 100, 8, 32, 128)
+    Lk = tq.tq_cache_layout_kv(3, 100, 8, 32, 128, tq.TQ_K_INT4)
+    assert bytes(L4) == bytes(Lk)
+    assert L4.k_format == tq.TQ_K_INT4 and L4.k_bytes == L4.codes_bytes and L4.k_stride_tok == L4.code_stride_tok
+    L16 = tq.tq_cache_layout_kv(3, 100, 8, 32, 128, tq.TQ_K_FP16)
+    assert L16.k_format == tq.TQ_K_FP16
+    assert L16.k_stride_tok == 8 * 128 * 2 and L16.k_stride_seq == 100 * 8 * 128 * 2
+    assert L16.k_bytes == 3 * 100 * 8 * 128 * 2
+    # V side unchanged
+    assert (L16.codes_bytes, L16.scales_bytes, L16.code_stride_tok) == (L4.codes_bytes, L4.scales_bytes,
+                                                                        L4.code_stride_tok)
+    code, _ = tq.tq_cache_layout_status(3, 100, 8, 32, 128)
+    assert code == tq.TQ_OK
+    with pytest.raises(tq.TqError) as exc:
+        tq.tq_cache_layout_kv(3, 100, 8, 32, 128, 7)
+    assert exc.value.code == tq.TQ_ERR_INVALID_ARG
