@@ -46,6 +46,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
     ap.add_argument("--no-references", action="store_true",
                     help="skip the quantise-throughput, bf16 dense-KV and dequantise-then-attend reference points")
+    ap.add_argument("--k-format", choices=["int4", "fp16"], default="int4",
+                    help="K storage: int4 codes like V (symmetric cache), or binary16 in the original domain "
+                         "(the asymmetric cache of the mlxcel guide's recommended mode)")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report instead of the step benchmark: decode and prefill-quantise "
                          "times (median, p10, p90; cold L2, and warm L2 where the cache fits) for every workload "
@@ -61,17 +64,20 @@ def get_workload(name):
 
 # ----------------------------------------------------------------------------- algorithmic bytes
 
-def decode_bytes(w, lens):
-    """Packed K + V codes and binary16 scales the decode must read: (D/2 + D/16) * 2 bytes per token.kv-head."""
-    per = 2 * (w.head_dim // 2 + 2 * (w.head_dim // 32))
-    return sum(lens) * w.n_kv_heads * per
-
-
-def append_bytes(w, in_bytes=2):
-    """Quantise-append traffic: raw K/V in + packed codes and scales out, per appended token."""
+def decode_bytes(w, lens, kf16=False):
+    """Cache bytes the decode must read per token.kv-head: packed V codes + binary16 scales
+    (D/2 + D/16), and the same again for int4 K or 2D for binary16 K."""
     D = w.head_dim
-    per_vec = D * in_bytes + D // 2 + 2 * (D // 32)
-    return 2 * w.batch * w.n_append * w.n_kv_heads * per_vec
+    v = D // 2 + 2 * (D // 32)
+    return sum(lens) * w.n_kv_heads * (v + (2 * D if kf16 else v))
+
+
+def append_bytes(w, in_bytes=2, kf16=False):
+    """Quantise-append traffic: raw K/V in + packed codes and scales (or binary16 K) out, per appended token."""
+    D = w.head_dim
+    v_vec = D * in_bytes + D // 2 + 2 * (D // 32)
+    k_vec = D * in_bytes + 2 * D if kf16 else v_vec
+    return w.batch * w.n_append * w.n_kv_heads * (v_vec + k_vec)
 
 
 def load_peaks():
@@ -238,35 +244,53 @@ class OracleStep:
     re-appends the new token at position len_b and decodes over len_b + 1.
     """
 
-    def __init__(self, w, tensors, seqs):
+    def __init__(self, w, tensors, seqs, kf16=False):
         import numpy as np
         import oracle
         from compressed_domain_attention_b200 import synthetic as syn
         self.oracle, self.np = oracle, np
         D, H = w.head_dim, w.n_kv_heads
-        self.w, self.seqs = w, seqs
+        self.w, self.seqs, self.kf16 = w, seqs, kf16
         self.s = oracle.sign_vector(0, D)
         n = len(seqs)
         cap = max(w.seq_lens[b] for b in seqs) + 1
-        self.kc, self.ks = oracle.new_cache(n, cap, H, D)
+        if kf16:
+            self.kc, self.ks = oracle.new_k16_cache(n, cap, H, D), None
+        else:
+            self.kc, self.ks = oracle.new_cache(n, cap, H, D)
         self.vc, self.vs = oracle.new_cache(n, cap, H, D)
         for i, b in enumerate(seqs):
             k = tensors.k[b].float().cpu().numpy()[None]
             v = tensors.v[b].float().cpu().numpy()[None]
-            oracle.quantize_append(self.s, k, v, np.zeros(1, np.int32), self.kc[i:i + 1], self.ks[i:i + 1],
-                                   self.vc[i:i + 1], self.vs[i:i + 1])
+            self._append(i, i + 1, k, v, np.zeros(1, np.int32))
         self.q = np.ascontiguousarray(tensors.q[seqs].float().cpu().numpy())
         self.kn = np.ascontiguousarray(tensors.k_new[seqs].float().cpu().numpy())
         self.vn = np.ascontiguousarray(tensors.v_new[seqs].float().cpu().numpy())
         self.lens = np.array([w.seq_lens[b] for b in seqs], np.int32)
         sub = syn.Workload(w.name, n, w.n_q_heads, H, D, [w.seq_lens[b] for b in seqs], w.dtype, w.seed, n_append=1)
-        self.nbytes = decode_bytes(sub, [L + 1 for L in sub.seq_lens]) + append_bytes(sub)
+        self.nbytes = decode_bytes(sub, [L + 1 for L in sub.seq_lens], kf16) + append_bytes(sub, kf16=kf16)
         self.ntok = int(self.lens.sum()) + n
 
+    def _append(self, i0, i1, k, v, start):
+        sl = slice(i0, i1)
+        if self.kf16:
+            self.oracle.quantize_append_kf16(self.s, k, v, start, self.kc[sl], self.vc[sl], self.vs[sl])
+        else:
+            self.oracle.quantize_append(self.s, k, v, start, self.kc[sl], self.ks[sl], self.vc[sl], self.vs[sl])
+
+    def _decode(self, i0, i1, q, lens):
+        sl = slice(i0, i1)
+        if self.kf16:
+            self.oracle.decode_attention_kf16(self.s, q, lens, self.kc[sl], self.vc[sl], self.vs[sl], self.w.scale)
+        else:
+            self.oracle.decode_attention(self.s, q, lens, self.kc[sl], self.ks[sl], self.vc[sl], self.vs[sl],
+                                         self.w.scale)
+
     def run(self):
+        n = len(self.seqs)
         t0 = time.perf_counter()
-        self.oracle.quantize_append(self.s, self.kn, self.vn, self.lens, self.kc, self.ks, self.vc, self.vs)
-        self.oracle.decode_attention(self.s, self.q, self.lens + 1, self.kc, self.ks, self.vc, self.vs, self.w.scale)
+        self._append(0, n, self.kn, self.vn, self.lens)
+        self._decode(0, n, self.q, self.lens + 1)
         return time.perf_counter() - t0
 
     def run_parallel(self, threads):
@@ -280,10 +304,8 @@ class OracleStep:
 
         def one(i):
             sl = slice(i, i + 1)
-            o.quantize_append(self.s, self.kn[sl], self.vn[sl], self.lens[sl], self.kc[sl], self.ks[sl],
-                              self.vc[sl], self.vs[sl])
-            o.decode_attention(self.s, self.q[sl], self.lens[sl] + 1, self.kc[sl], self.ks[sl], self.vc[sl],
-                               self.vs[sl], self.w.scale)
+            self._append(i, i + 1, self.kn[sl], self.vn[sl], self.lens[sl])
+            self._decode(i, i + 1, self.q[sl], self.lens[sl] + 1)
 
         with ThreadPoolExecutor(max_workers=threads) as ex:
             t0 = time.perf_counter()
@@ -298,9 +320,9 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, tensors, target_tokens):
+def cpu_baseline(w, tensors, target_tokens, kf16=False):
     seqs = oracle_sample(w, target_tokens)
-    o = OracleStep(w, tensors, seqs)
+    o = OracleStep(w, tensors, seqs, kf16)
     dt = o.run()
     line = {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
@@ -333,7 +355,7 @@ def _time_cold(fn, reps, flush, stream):
     return statistics.median(ts)
 
 
-def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args):
+def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, kf16=False):
     """Quantise throughput, the bf16 dense-KV decode and dequantise-then-attend, on this GPU and workload."""
     import torch
     import torch.nn.functional as F
@@ -393,7 +415,7 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args):
         torch.cuda.empty_cache()
     # 3. dequantise-then-attend (the comparison category of the Open-TQ-Metal abstract):
     #    tq_dequantize_debug to dense fp32 K/V in the original domain, then SDPA per sequence
-    if not args.no_references and w.batch * L.max_seq * w.n_kv_heads * w.head_dim * 4 * 2 < 24e9:
+    if not args.no_references and not kf16 and w.batch * L.max_seq * w.n_kv_heads * w.head_dim * 4 * 2 < 24e9:
         Kd = torch.empty((w.batch, L.max_seq, w.n_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
         Vd = torch.empty_like(Kd)
         qf = q.float().view(w.batch, w.n_q_heads, 1, w.head_dim)
@@ -458,27 +480,32 @@ def run_sweep(args):
     stream = torch.cuda.current_stream()
     flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)  # 256 MB > 126 MB L2
     peak, peak_kind = load_peaks()
-    cfgs = [("c0", syn.tiny_single_head()), ("c1", syn.llama3_8b_layer())]
-    cfgs += [("c2", syn.gemma3_1b_sweep(T)) for T in (256, 512, 1024, 2048, 4096)]
-    cfgs += [("c3", syn.llama31_70b_long()), ("c4", syn.ragged_serving())]
-    for tag, w in cfgs:
+    cfgs = [("c0", syn.tiny_single_head, False), ("c1", syn.llama3_8b_layer, False)]
+    cfgs += [("c2", (lambda T=T: syn.gemma3_1b_sweep(T)), False) for T in (256, 512, 1024, 2048, 4096)]
+    cfgs += [("c3", syn.llama31_70b_long, False), ("c4", syn.ragged_serving, False)]
+    # the asymmetric cache (binary16 K, int4 V) on the head_dim-128 shapes
+    cfgs += [("c1", syn.llama3_8b_layer, True), ("c3", syn.llama31_70b_long, True), ("c4", syn.ragged_serving, True)]
+    for tag, make, kf16 in cfgs:
+        w = make()
         t = syn.generate(w, device="cuda")
         n_app = max(w.n_append, 1)
         cap = max(w.seq_lens) + n_app
-        L = tq.tq_cache_layout(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+        kfmt = tq.TQ_K_FP16 if kf16 else tq.TQ_K_INT4
+        L = tq.tq_cache_layout_kv(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
         kc, ks, vc, vs = tq.alloc_cache(L, dev)
         wsp = tq.alloc_workspace(L, dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        l1 = tq.tq_cache_layout(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+        l1 = tq.tq_cache_layout_kv(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
         zero = torch.zeros(1, dtype=torch.int32, device=dev)
-        cs, ss = int(L.code_stride_seq), int(L.scale_stride_seq)
+        cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
         kb = [t.k[b][None].contiguous() for b in range(w.batch)]
         vb = [t.v[b][None].contiguous() for b in range(w.batch)]
 
         def prefill():
             for b in range(w.batch):
-                tq.tq_quantize_append(l1, kb[b], vb[b], w.seq_lens[b], zero, kc[b * cs:(b + 1) * cs], ks[b * ss:],
-                                      vc[b * cs:(b + 1) * cs], vs[b * ss:], status, stream)
+                tq.tq_quantize_append(l1, kb[b], vb[b], w.seq_lens[b], zero, kc[b * kst:(b + 1) * kst],
+                                      None if kf16 else ks[b * ss:], vc[b * cs:(b + 1) * cs], vs[b * ss:], status,
+                                      stream)
 
         prefill()
         pre = _time_reps(prefill, 5, flush, stream)
@@ -494,7 +521,7 @@ def run_sweep(args):
             decode()
         reps = 20 if sum(w.seq_lens) * w.n_kv_heads >= 1 << 20 else 100
         cold = _time_reps(decode, reps, flush, stream)
-        nbytes = decode_bytes(w, w.seq_lens)
+        nbytes = decode_bytes(w, w.seq_lens, kf16)
         warm = _time_reps(decode, reps, None, stream) if nbytes < 64e6 else None
         kn, vn = t.k_new.contiguous() if w.n_append else None, t.v_new.contiguous() if w.n_append else None
         app = None
@@ -522,7 +549,8 @@ def run_sweep(args):
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the sweep ({w.name})")
         ms = cold["median"]
-        line = {"sweep": tag, "workload": w.name, "batch": w.batch, "tokens": sum(w.seq_lens),
+        line = {"sweep": tag, "workload": w.name, "k_format": "fp16" if kf16 else "int4", "batch": w.batch,
+                "tokens": sum(w.seq_lens), "cache_bytes_read": nbytes,
                 "decode_ms_cold_l2": cold, "decode_gbs": round(nbytes / ms / 1e6, 1),
                 "pct_of_8_tbs": round(nbytes / ms / 1e6 / 80.0, 2),
                 "pct_of_measured_hbm": round(nbytes / ms / 1e6 / peak * 100.0, 2), "peak_kind": peak_kind,
@@ -552,7 +580,8 @@ def run_reference(args):
         w.n_append = 1
     seqs = oracle_sample(w, 8192)
     t = syn.generate(w, device="cpu", seq_subset=seqs)
-    o = OracleStep(w, t, seqs)
+    kf16 = getattr(args, "k_format", "int4") == "fp16"
+    o = OracleStep(w, t, seqs, kf16)
     for _ in range(args.warmup):
         o.run()
     tot_t = sum(o.run() for _ in range(args.steps))
@@ -562,7 +591,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode / f64 attention",
-            "data": "synthetic (seeded)", "config": {"workload": w.name, "global_batch": w.batch},
+            "data": "synthetic (seeded)", "config": {"workload": w.name, "global_batch": w.batch,
+                                                     "k_format": getattr(args, "k_format", "int4")},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -584,18 +614,20 @@ def run_tq(args):
         w.n_append = 1
     cap = max(w.seq_lens) + w.n_append
     t = syn.generate(w, device="cuda")
-    L = tq.tq_cache_layout(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+    kf16 = args.k_format == "fp16"
+    kfmt = tq.TQ_K_FP16 if kf16 else tq.TQ_K_INT4
+    L = tq.tq_cache_layout_kv(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
     kc, ks, vc, vs = tq.alloc_cache(L, dev)
     wsp = tq.alloc_workspace(L, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     # prefill (untimed): one append per sequence through a batch-1 view of the cache
-    l1 = tq.tq_cache_layout(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+    l1 = tq.tq_cache_layout_kv(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
     zero = torch.zeros(1, dtype=torch.int32, device=dev)
-    cs, ss = int(L.code_stride_seq), int(L.scale_stride_seq)
+    cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
     for b in range(w.batch):
         n = w.seq_lens[b]
-        tq.tq_quantize_append(l1, t.k[b][None], t.v[b][None], n, zero, kc[b * cs:(b + 1) * cs], ks[b * ss:],
-                              vc[b * cs:(b + 1) * cs], vs[b * ss:], status)
+        tq.tq_quantize_append(l1, t.k[b][None], t.v[b][None], n, zero, kc[b * kst:(b + 1) * kst],
+                              None if kf16 else ks[b * ss:], vc[b * cs:(b + 1) * cs], vs[b * ss:], status)
     torch.cuda.synchronize()
     lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
     lens1 = lens + w.n_append
@@ -735,11 +767,12 @@ def run_tq(args):
     if not torch.equal(h_out[(args.steps - 1) % 2], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-timed output")
 
-    refs = {} if args.no_references else reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args)
+    refs = {} if args.no_references else reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args,
+                                                          kf16=kf16)
 
     lens_step = [x + w.n_append for x in w.seq_lens]
-    bytes_decode = decode_bytes(w, lens_step)
-    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4)
+    bytes_decode = decode_bytes(w, lens_step, kf16)
+    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4, kf16)
     max_t = max_over_ranks(elapsed, dev)
     max_e2e = max_over_ranks(e2e_s, dev)
     split_avg = max_over_ranks(statistics.mean(split_ms), dev)
@@ -747,8 +780,9 @@ def run_tq(args):
 
     peak, peak_kind = load_peaks()
     achieved = bytes_decode / (split_avg / 1e3) / 1e9
-    traffic = load_traffic(f"decode_split_kernel/{w.name}")
+    traffic = load_traffic(f"decode_split_kernel/{w.name}" + ("/k_fp16" if kf16 else ""))
     kv_tokens = sum(lens_step) * w.n_kv_heads
+    cache_bytes = int(L.k_bytes + L.codes_bytes + L.scales_bytes * (1 if kf16 else 2))
     extra = {
         "tokens_per_s": round(ws * w.batch * w.n_append * args.steps / max_t, 1),
         "kv_tokens_per_s": round(ws * sum(lens_step) * args.steps / max_t, 1),
@@ -776,13 +810,13 @@ def run_tq(args):
     cfg = {"workload": w.name, "global_batch": w.batch * ws, "kv_tokens_per_seq_step": lens_step if w.batch <= 4
            else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+           "k_format": args.k_format,
            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-           "l2": f"inputs larger than L2 (packed cache {2 * int(L.codes_bytes + L.scales_bytes) / 1e9:.2f} GB "
-                 "per replica > 126 MB), no flush",
+           "l2": f"inputs larger than L2 (cache {cache_bytes / 1e9:.2f} GB per replica > 126 MB), no flush",
            "algorithmic_bytes_per_step": bytes_step}
     total_bytes = sum_over_ranks(bytes_step * args.steps, dev)  # every rank takes part
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        extra["cpu_baseline"] = cpu_baseline(w, t, 300000)
+        extra["cpu_baseline"] = cpu_baseline(w, t, 300000, kf16)
     if rank == 0:
         line = assemble_line(n_gpus=ws, steps=args.steps, warmup=args.warmup, total_bytes_all_ranks=total_bytes,
                              max_time_s=max_t, workload=cfg, extra=extra)
