@@ -99,20 +99,21 @@ int encode_codes_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::T
   return TQ_OK;
 }
 
-// 4-D view of a binary16 K buffer: (64 halves, D/64 lines, batch*max_seq tokens,
-// n_kv heads) with strides (128 B, token stride, 2D B), box (64, D/64, tile, n_kv):
-// the shared-memory image is [head][tile][D] binary16 in 128-byte lines with the
-// 128-byte swizzle (D = 32: one 64-byte line per row, 64-byte swizzle).
+// 4-D view of a binary16 K buffer: (64 halves, batch*max_seq tokens, D/64 lines,
+// n_kv heads) with strides (token stride, 128 B, 2D B), box (64, tile, D/64, n_kv):
+// the shared-memory image is [head][line][tile][64] binary16 with the 128-byte
+// swizzle, so 8 consecutive tokens of one line fall on 8 swizzle phases
+// (D = 32: one 64-byte line per token, 64-byte swizzle).
 int encode_k16_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::TensorMap128* out) {
   auto enc = get_encode_fn();
   if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
   const int D = L->head_dim;
   const int inner = D < 64 ? D : 64;
   const int lines = D / inner;
-  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)lines, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq,
+  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq, (cuuint64_t)lines,
                         (cuuint64_t)L->n_kv_heads};
-  cuuint64_t strides[3] = {(cuuint64_t)inner * 2, (cuuint64_t)L->k_stride_tok, (cuuint64_t)D * 2};
-  cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)lines, (cuuint32_t)tile, (cuuint32_t)L->n_kv_heads};
+  cuuint64_t strides[3] = {(cuuint64_t)L->k_stride_tok, (cuuint64_t)inner * 2, (cuuint64_t)D * 2};
+  cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)tile, (cuuint32_t)lines, (cuuint32_t)L->n_kv_heads};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUtensorMapSwizzle sw = inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap m;

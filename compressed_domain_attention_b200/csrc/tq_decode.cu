@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
       const int row = (int)((int64_t)walk.b * p.max_seq + walk.t0);
       if constexpr (KF16)
-        tma_load_4d(sb, &kmap, &full[stage], 0, 0, row, 0, pol);
+        tma_load_4d(sb, &kmap, &full[stage], 0, row, 0, 0, pol);
       else
         tma_load_3d(sb, &kmap, &full[stage], 0, row, 0, pol);
       tma_load_3d(sb + C::OFF_VCODE, &vmap, &full[stage], 0, row, 0, pol);
@@ -422,9 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   static_assert((UNIT * RB) % 1024 == 0 || C::SWZ == 0 || (UNIT * RB) % ((C::SWZ + 1) * 128) == 0,
                 "unit rows must keep the swizzle phase");
-  // binary16 K: per-lane ldmatrix offsets of k-step kk inside the head's [tile][D]
-  // binary16 block, relative to the unit's first token (the unit and head offsets are
-  // whole multiples of the swizzle period). Row layout (K as B): matrix m = lane / 8
+  // binary16 K: per-lane ldmatrix offsets of k-step kk inside the head's
+  // [line][tile][64] binary16 block, relative to the unit's first token (unit and head
+  // offsets are whole multiples of the swizzle period). Row layout (K as B): matrix m = lane / 8
   // is (8-token n-tile m / 2, dims + 8 (m % 2)); tokens-in-M (K as A): matrix m is
   // (token rows 8 (m % 2) .., dims + 8 (m / 2)).
   uint32_t k16_off[KF16 ? 2 * NG : 1];
@@ -437,12 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kk = 0; kk < 2 * NG; ++kk) {
       const int dims = 16 * kk + dadd;
       const int ch = dims / HPL;
-      const int line = tok * C::KNCH + ch;
+      const int line = ch * T_TILE + tok;
       const int sw = ((line * C::KLINE) >> 7) & C::KSWZ;
-      k16_off[kk] = (uint32_t)(tok * C::KRB + ch * C::KLINE + ((((dims % HPL) >> 3) ^ sw) << 4));
+      k16_off[kk] = (uint32_t)(line * C::KLINE + ((((dims % HPL) >> 3) ^ sw) << 4));
     }
   }
-  static_assert(!KF16 || (UNIT % 16 == 0 && (T_TILE * C::KNCH) % 8 == 0), "binary16 K swizzle phase");
+  static_assert(!KF16 || (UNIT % 16 == 0 && T_TILE % 8 == 0), "binary16 K swizzle phase");
 
   uint32_t qA[NG][2][4];
   float biasK[NG];
@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 2 * NG; ++kk) {
                   uint32_t kw[4];
-                  ldmatrix_x4(kw, kc + (r0 + 16 * mt) * C::KRB + k16_off[kk]);
+                  ldmatrix_x4(kw, kc + (r0 + 16 * mt) * C::KLINE + k16_off[kk]);
                   mma_f16_16816_acc(c, kw, qA[kk / 2][kk % 2][0], qA[kk / 2][kk % 2][1]);
                 }
                 s2[mt] = make_float2(c[0] + c[1], c[2] + c[3]);  // hi + lo columns
@@ -769,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int np = 0; np < NT / 2; ++np) {
                   uint32_t kw[4];
-                  ldmatrix_x4(kw, kc + (r0 + 16 * np) * C::KRB + k16_off[kk]);
+                  ldmatrix_x4(kw, kc + (r0 + 16 * np) * C::KLINE + k16_off[kk]);
                   mma_f16_16816_acc(c[2 * np], qA[kk / 2][kk % 2], kw[0], kw[1]);
                   mma_f16_16816_acc(c[2 * np + 1], qA[kk / 2][kk % 2], kw[2], kw[3]);
                 }
