@@ -47,6 +47,11 @@ def _signatures():
         "oracle_dequantize": ([ctypes.c_int] * 4 + [P, P, P, P, ctypes.c_int, P], i32),
         "oracle_quantize_append_kf16": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P, P, P], i32),
         "oracle_decode_attention_kf16": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, f32, P, P], i32),
+        "oracle_cold_length": ([i64, ctypes.c_int, ctypes.c_int], i64),
+        "oracle_append_delegated": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
+                                                          P, P, P, P], i32),
+        "oracle_decode_attention_delegated": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                                                    f32, P, P], i32),
     }
 
 
@@ -242,6 +247,49 @@ def decode_attention_kf16(signs, q, seq_lens, k_f16, v_codes, v_scales, sm_scale
         B, max_seq, n_kv, n_q, D, _p(s), _p(q), _p(sl), _p(_c(k_f16, np.uint16)),
         _p(_c(v_codes, np.uint8)), _p(_c(v_scales, np.uint16)), ctypes.c_float(sm_scale),
         None if w is None else _p(w), _p(out))
+    return out, int(st)
+
+
+def cold_length(length: int, window: int, fold: int) -> int:
+    """Tokens of a delegated-cache sequence of `length` tokens that sit in the int4 body."""
+    return int(_load().oracle_cold_length(length, window, fold))
+
+
+def new_tail(batch, window, n_kv, D):
+    """Zeroed binary16 V hot tail [B][W][Hkv][D] (bits, uint16) for the delegated cache."""
+    return np.zeros((batch, window, n_kv, D), np.uint16)
+
+
+def append_delegated(signs, k, v, start_pos, window, fold, k_f16, v_codes, v_scales, v_tail) -> int:
+    """Delegated append (binary16 K; V into the binary16 hot tail, folded into int4 codes). In place."""
+    k = _c(k, np.float32)
+    v = _c(v, np.float32)
+    B, n_new, n_kv, D = k.shape
+    max_seq = v_codes.shape[1]
+    assert k_f16.dtype == np.uint16 and k_f16.flags.c_contiguous and k_f16.shape[1] == max_seq
+    assert v_tail.dtype == np.uint16 and v_tail.flags.c_contiguous and v_tail.shape == (B, window, n_kv, D)
+    for a, dt in ((v_codes, np.uint8), (v_scales, np.uint16)):
+        assert a.dtype == dt and a.flags.c_contiguous
+    sp = _c(start_pos, np.int32)
+    s = _c(signs, np.float32)
+    return int(_load().oracle_append_delegated(B, max_seq, n_kv, D, _p(s), _p(k), _p(v), n_new, _p(sp),
+                                               window, fold, _p(k_f16), _p(v_codes), _p(v_scales), _p(v_tail)))
+
+
+def decode_attention_delegated(signs, q, seq_lens, k_f16, v_codes, v_scales, v_tail, window, fold, sm_scale,
+                               which=None):
+    """Decode attention on the delegated cache. -> (out [B][Hq][D] float32, status)."""
+    q = _c(q, np.float32)
+    B, n_q, D = q.shape
+    max_seq, n_kv = v_codes.shape[1], v_codes.shape[2]
+    sl = _c(seq_lens, np.int32)
+    s = _c(signs, np.float32)
+    out = np.zeros((B, n_q, D), np.float32)
+    w = None if which is None else _c(which, np.uint8)
+    st = _load().oracle_decode_attention_delegated(
+        B, max_seq, n_kv, n_q, D, _p(s), _p(q), _p(sl), _p(_c(k_f16, np.uint16)),
+        _p(_c(v_codes, np.uint8)), _p(_c(v_scales, np.uint16)), _p(_c(v_tail, np.uint16)), window, fold,
+        ctypes.c_float(sm_scale), None if w is None else _p(w), _p(out))
     return out, int(st)
 
 

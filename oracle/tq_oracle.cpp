@@ -25,6 +25,10 @@
 //  [MLX-modes] the same guide, §"Cache modes" and §"What TurboQuant changes":
 //          the recommended default mode (fp16+turbo4) keeps K in FP16 and
 //          compresses only V, because K decides where attention looks.
+//  [MLX-deleg] the same guide, §"Cache modes" (turbo4-delegated row: K in FP16,
+//          V as an FP16 hot tail plus a Turbo4 cold body) and §"Delegated cache
+//          variant" (recent tokens stay FP16, older V tokens are stored in the
+//          4-bit form; the FP16 sidecars are folded into it).
 //  [AMD]   "TurboQuant on AMD GPUs" (oracore.dev), §4: Walsh-Hadamard spreads
 //          energy evenly and suits kernels better than a dense random rotation.
 //
@@ -222,17 +226,34 @@ void dequantize_rotated(const uint8_t* bytes, const uint16_t* scales, int D, flo
   for (int i = 0; i < D; ++i) yhat[i] = (float)codes[i] * f16_to_f32(scales[i / 32]);
 }
 
+// ---- delegated hot/cold cache [MLX-deleg] ----
+// Reading taken (the guide names the parts, not the policy): the hot tail holds
+// the most recent tokens' V in binary16, at most W of them, in a ring of W slots
+// per (sequence, kv head), token t in slot t mod W. Tokens leave it oldest first,
+// F at a time: a sequence of len tokens has cold_length(len) tokens in the int4
+// body, so that W - F < len - cold_length(len) <= W once len > W.
+int64_t cold_length(int64_t len, int W, int F) {
+  if (len <= W) return 0;
+  return (len - W + F - 1) / F * F;
+}
+
+// The decode steps shared by the three cache formats. k_f16 == nullptr: int4 K
+// (scores against SRHT(q)); otherwise binary16 K (scores against q). v_tail ==
+// nullptr: every V token is int4; otherwise tokens t >= cold_length(len_b)
+// take their binary16 tail value, mapped to the rotated domain by the forward
+// SRHT so that the weighted sum stays in one domain (the transform is linear).
 int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const float* s, const float* q,
                     const int32_t* seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
-                    const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale,
-                    const uint8_t* which, float* out) {
+                    const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales,
+                    const uint16_t* v_tail, int W, int F, float sm_scale, const uint8_t* which, float* out) {
   int32_t st = 0;
   const int G = n_q / n_kv;
   const int64_t cb = D / 2, sb = D / 32;
-  std::vector<float> qr(D), yk(D), yv(D), o32(D);
+  std::vector<float> qr(D), yk(D), yv(D), xv(D), o32(D);
   std::vector<double> z, acc(D);
   for (int b = 0; b < batch; ++b) {
     const int len = seq_lens[b];
+    const int64_t n_cold = v_tail ? cold_length(len, W, F) : len;
     for (int hq = 0; hq < n_q; ++hq) {
       if (which && !which[(int64_t)b * n_q + hq]) continue;
       float* o = out + ((int64_t)b * n_q + hq) * D;
@@ -271,7 +292,13 @@ int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const floa
       for (int i = 0; i < D; ++i) acc[i] = 0.0;
       for (int t = 0; t < len; ++t) {
         const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
-        dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());
+        if (t < n_cold) {
+          dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());
+        } else {
+          const uint16_t* hot = v_tail + (((int64_t)b * W + t % W) * n_kv + kv) * D;
+          for (int i = 0; i < D; ++i) xv[i] = f16_to_f32(hot[i]);
+          srht_forward_vec(xv.data(), s, D, yv.data());
+        }
         const double w = z[t] / l;
         for (int i = 0; i < D; ++i) acc[i] += w * (double)yv[i];
       }
@@ -402,7 +429,7 @@ int32_t oracle_decode_attention(int batch, int max_seq, int n_kv, int n_q, int D
                                 const uint8_t* v_codes, const uint16_t* v_scales,
                                 float sm_scale, const uint8_t* which, float* out) {
   return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, k_codes, k_scales, nullptr, v_codes, v_scales,
-                     sm_scale, which, out);
+                     nullptr, 0, 0, sm_scale, which, out);
 }
 
 // ---- asymmetric cache: K in binary16, V as int4 codes [MLX-modes] ----
@@ -447,8 +474,69 @@ int32_t oracle_decode_attention_kf16(int batch, int max_seq, int n_kv, int n_q, 
                                      const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale,
                                      const uint8_t* which, float* out) {
   return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, nullptr, nullptr, k_f16, v_codes, v_scales,
-                     sm_scale, which, out);
+                     nullptr, 0, 0, sm_scale, which, out);
 }
+
+// Delegated hot/cold cache [MLX-deleg]: K as binary16 for every token (as in
+// the asymmetric cache), V as binary16 in the hot tail v_tail [batch][W][n_kv][D]
+// and as int4 codes in the cold body (the usual V caches, at the token's own
+// position). Tokens are taken one at a time, in order: when the sequence grows
+// from P to P + 1 tokens, every token that cold_length moves out of the tail is
+// folded first (its binary16 tail value encoded exactly as a fresh V vector),
+// then token P enters the tail. A V element whose binary16 is not finite raises
+// ORC_STATUS_NONFINITE. Tail slots of tokens already folded keep stale values.
+int32_t oracle_append_delegated(int batch, int max_seq, int n_kv, int D, const float* s, const float* k,
+                                const float* v, int n_new, const int32_t* start_pos, int W, int F,
+                                uint16_t* k_f16, uint8_t* v_codes, uint16_t* v_scales, uint16_t* v_tail) {
+  int32_t st = 0;
+  const int64_t cb = D / 2, sb = D / 32;
+  std::vector<float> x(D);
+  for (int b = 0; b < batch; ++b) {
+    const int64_t p0 = start_pos[b];
+    if (p0 < 0 || p0 + n_new > max_seq) {
+      st |= ORC_STATUS_CAPACITY;
+      continue;
+    }
+    for (int t = 0; t < n_new; ++t) {
+      const int64_t P = p0 + t;
+      for (int64_t T = cold_length(P, W, F); T < cold_length(P + 1, W, F); ++T) {
+        for (int h = 0; h < n_kv; ++h) {
+          const uint16_t* hot = v_tail + (((int64_t)b * W + T % W) * n_kv + h) * D;
+          for (int i = 0; i < D; ++i) x[i] = f16_to_f32(hot[i]);
+          const int64_t row = ((int64_t)b * max_seq + T) * n_kv + h;
+          st |= oracle_encode(x.data(), s, D, 1, v_codes + row * cb, v_scales + row * sb);
+        }
+      }
+      for (int h = 0; h < n_kv; ++h) {
+        const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
+        const int64_t row = ((int64_t)b * max_seq + P) * n_kv + h;
+        uint16_t* hot = v_tail + (((int64_t)b * W + P % W) * n_kv + h) * D;
+        for (int i = 0; i < D; ++i) {
+          const uint16_t kb = f32_to_f16_rne(k[src + i]);
+          const uint16_t vb = f32_to_f16_rne(v[src + i]);
+          if ((kb & 0x7C00u) == 0x7C00u || (vb & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
+          k_f16[row * D + i] = kb;
+          hot[i] = vb;
+        }
+      }
+    }
+  }
+  return st;
+}
+
+// Decode attention over the delegated cache: the asymmetric decode's steps
+// (binary16 K against q), with V_t = code * sigma for t < cold_length(len_b)
+// and SRHT(binary16 tail value) otherwise, then SRHT^-1 of the weighted sum.
+int32_t oracle_decode_attention_delegated(int batch, int max_seq, int n_kv, int n_q, int D, const float* s,
+                                          const float* q, const int32_t* seq_lens, const uint16_t* k_f16,
+                                          const uint8_t* v_codes, const uint16_t* v_scales,
+                                          const uint16_t* v_tail, int W, int F, float sm_scale,
+                                          const uint8_t* which, float* out) {
+  return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, nullptr, nullptr, k_f16, v_codes, v_scales,
+                     v_tail, W, F, sm_scale, which, out);
+}
+
+int64_t oracle_cold_length(int64_t len, int W, int F) { return cold_length(len, W, F); }
 
 // Dequantise a whole cache: out [batch][max_seq][n_kv][D] binary32, rows t >= len_b
 // set to 0. original_domain = 0 gives yhat = code * sigma (rotated domain);

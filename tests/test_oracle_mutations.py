@@ -132,3 +132,53 @@ def test_planted_kf16_mistake_is_caught(name, tmp_path, monkeypatch):
     lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
     monkeypatch.setattr(oracle, "_lib", lib)
     assert failing_kf16_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"
+
+
+DELEGATED_MUTATIONS = {
+    "deleg_cold_length_floor": ("return (len - W + F - 1) / F * F;", "return (len - W) / F * F;"),
+    "deleg_fold_reads_next_slot": ("const uint16_t* hot = v_tail + (((int64_t)b * W + T % W) * n_kv + h) * D;",
+                                   "const uint16_t* hot = v_tail + (((int64_t)b * W + (T + 1) % W) * n_kv + h) * D;"),
+    "deleg_tail_written_one_slot_late": ("uint16_t* hot = v_tail + (((int64_t)b * W + P % W) * n_kv + h) * D;",
+                                         "uint16_t* hot = v_tail + (((int64_t)b * W + (P + 1) % W) * n_kv + h) * D;"),
+    "deleg_hot_v_not_rotated": ("srht_forward_vec(xv.data(), s, D, yv.data());",
+                                "std::memcpy(yv.data(), xv.data(), sizeof(float) * D);"),
+    "deleg_tail_holds_k": ("hot[i] = vb;", "hot[i] = kb;"),
+    "deleg_boundary_token_read_cold": ("if (t < n_cold) {", "if (t <= n_cold) {"),
+}
+
+
+def delegated_pins(orc):
+    yield lambda: pins.test_delegated_cold_length_worked_values_and_invariants(orc)
+    yield lambda: pins.test_delegated_append_holds_binary16_tail_and_encoded_body(orc, 128, 8, 4, 13)
+    yield lambda: pins.test_delegated_append_is_chunking_invariant(orc)
+    yield lambda: pins.test_delegated_attention_equals_fp64(orc, 128, 8, 1, 16, 8, 50)
+    yield lambda: pins.test_delegated_all_hot_is_binary16_attention_of_the_inputs(orc)
+    yield lambda: pins.test_delegated_special_cases(orc)
+
+
+def failing_delegated_pins(orc):
+    failed = 0
+    for check in delegated_pins(orc):
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_delegated_pins_pass_on_committed_oracle(orc):
+    assert failing_delegated_pins(orc) == 0
+
+
+@pytest.mark.parametrize("name", sorted(DELEGATED_MUTATIONS))
+def test_planted_delegated_mistake_is_caught(name, tmp_path, monkeypatch):
+    before, after = DELEGATED_MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "tq_oracle_mut.cpp"
+    mutated.write_text(src.replace(before, after))
+    lib_path = tmp_path / f"libtq_oracle_{name}.so"
+    subprocess.run(["g++", *CXXFLAGS, "-o", str(lib_path), str(mutated)], check=True)
+    lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert failing_delegated_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"

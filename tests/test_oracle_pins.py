@@ -534,3 +534,170 @@ def test_kf16_attention_special_cases(orc):
     assert st == 0 and np.all(oute == 0)
     outc, st = orc.decode_attention_kf16(s, q, np.array([T + 1], np.int32), k16, vc, vs, 0.1)
     assert st & orc.STATUS_CAPACITY and np.all(outc == 0)
+
+
+# ---------------------------------------------------------------- delegated hot/cold cache
+# mlxcel "TurboQuant KV cache compression", §"Cache modes" (turbo4-delegated: K in
+# FP16, V as an FP16 hot tail plus a 4-bit cold body) and §"Delegated cache variant".
+
+# cold_length(len) for W = 8, F = 4 and W = 6, F = 3, worked by hand from the
+# reading "at most W hot tokens, folded F at a time, oldest first"
+COLD_W8_F4 = [0] * 9 + [4] * 4 + [8] * 4 + [12] * 4          # len 0..20
+COLD_W6_F3 = [0] * 7 + [3] * 3 + [6] * 3 + [9] * 3           # len 0..15
+
+
+def test_delegated_cold_length_worked_values_and_invariants(orc):
+    assert [orc.cold_length(n, 8, 4) for n in range(21)] == COLD_W8_F4
+    assert [orc.cold_length(n, 6, 3) for n in range(16)] == COLD_W6_F3
+    for W, F in ((1, 1), (16, 16), (64, 16), (256, 64), (100, 7)):
+        prev = 0
+        for n in range(0, 5 * W + 3):
+            c = orc.cold_length(n, W, F)
+            assert c % F == 0 and c >= prev and c - prev in (0, F)
+            hot = n - c
+            assert (hot == n) if n <= W else (W - F < hot <= W)
+            prev = c
+
+
+def make_delegated(orc, s, k, v, W, F, chunks=None, max_seq=None):
+    """Append k, v [B][T][Hkv][D] into a fresh delegated cache, in one call or in the given chunk sizes."""
+    B, T, Hkv, D = k.shape
+    S = max_seq or T
+    k16 = orc.new_k16_cache(B, S, Hkv, D)
+    vc, vs = orc.new_cache(B, S, Hkv, D)
+    tail = orc.new_tail(B, W, Hkv, D)
+    st = 0
+    pos = 0
+    for c in (chunks or [T]):
+        st |= orc.append_delegated(s, k[:, pos:pos + c], v[:, pos:pos + c], np.full(B, pos, np.int32), W, F,
+                                   k16, vc, vs, tail)
+        pos += c
+    assert pos == T
+    return k16, vc, vs, tail, st
+
+
+@pytest.mark.parametrize("D,W,F,T", [(32, 8, 4, 21), (128, 8, 4, 13), (64, 6, 3, 6), (128, 16, 16, 40)])
+def test_delegated_append_holds_binary16_tail_and_encoded_body(orc, D, W, F, T):
+    rng = np.random.default_rng(D + W + T)
+    s = orc.sign_vector(0, D)
+    B, Hkv = 2, 2
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    v = np.stack([heavy_tailed(rng, T * Hkv, D).reshape(T, Hkv, D) for _ in range(B)])
+    k16, vc, vs, tail, st = make_delegated(orc, s, k, v, W, F)
+    assert st == 0
+    # K: numpy's binary16 of every token
+    assert np.array_equal(k16, k.astype(np.float16).view(np.uint16))
+    nc = orc.cold_length(T, W, F)
+    v16 = v.astype(np.float16)
+    # hot tokens: numpy's binary16 of V, at slot t mod W
+    for t in range(nc, T):
+        assert np.array_equal(tail[:, t % W], v16[:, t].view(np.uint16))
+    # cold tokens: the symmetric encoding of the binary16-rounded V, bit for bit
+    kc2, ks2 = orc.new_cache(B, T, Hkv, D)
+    vc2, vs2 = orc.new_cache(B, T, Hkv, D)
+    orc.quantize_append(s, k, v16.astype(np.float32), np.zeros(B, np.int32), kc2, ks2, vc2, vs2)
+    assert np.array_equal(vc[:, :nc], vc2[:, :nc]) and np.array_equal(vs[:, :nc], vs2[:, :nc])
+
+
+def test_delegated_append_is_chunking_invariant(orc):
+    rng = np.random.default_rng(99)
+    D, W, F, T, B, Hkv = 64, 8, 4, 37, 2, 2
+    s = orc.sign_vector(5, D)
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    ref = make_delegated(orc, s, k, v, W, F)
+    nc = orc.cold_length(T, W, F)
+    live = sorted({t % W for t in range(nc, T)})
+    for chunks in ([1] * T, [3, 9, 1, 1, 20, 3], [8, 8, 8, 8, 5], [30, 7]):
+        got = make_delegated(orc, s, k, v, W, F, chunks)
+        assert np.array_equal(got[0], ref[0])
+        assert np.array_equal(got[1][:, :nc], ref[1][:, :nc]) and np.array_equal(got[2][:, :nc], ref[2][:, :nc])
+        assert np.array_equal(got[3][:, live], ref[3][:, live])
+
+
+def brute_force_attention_delegated(q, lens, k16, vc, vs, tail, s, W, F, cold_len, sm_scale):
+    """softmax(q K^T * scale) V in fp64 with the cache's own values: binary16 K; V the dequantised
+    original-domain body below cold_len(len), the binary16 tail value above."""
+    B, Hq, D = q.shape
+    Hkv = vc.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        L = lens[b]
+        if L == 0:
+            continue
+        nc = cold_len(L)
+        for hq in range(Hq):
+            kv = hq // G
+            K = k16[b, :L, kv].view(np.float16).astype(np.float64)
+            V = np.empty((L, D))
+            if nc:
+                V[:nc] = np_dequant_original(vc[b, :nc, kv], vs[b, :nc, kv], s)
+            for t in range(nc, L):
+                V[t] = tail[b, t % W, kv].view(np.float16).astype(np.float64)
+            z = K @ q[b, hq].astype(np.float64) * sm_scale
+            w = np.exp(z - z.max())
+            out[b, hq] = (w / w.sum()) @ V
+    return out
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,W,F,T", [(32, 4, 1, 8, 4, 21), (128, 8, 1, 16, 8, 50), (64, 4, 2, 6, 3, 6),
+                                            (128, 16, 2, 32, 32, 33)])
+def test_delegated_attention_equals_fp64(orc, D, Hq, Hkv, W, F, T):
+    rng = np.random.default_rng(D + Hq + W + T)
+    s = orc.sign_vector(0, D)
+    B = 3
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    k16, vc, vs, tail, st = make_delegated(orc, s, k, v, W, F)
+    assert st == 0
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    scale = 1.0 / np.sqrt(D)
+    # decode at the full length only: shorter lengths would read tail slots a later token overwrote
+    lens = np.array([T, T, T], np.int32)
+    got, st = orc.decode_attention_delegated(s, q, lens, k16, vc, vs, tail, W, F, scale)
+    assert st == 0
+    # cold_length restated from the worked tables' rule, not through the oracle
+    cold = lambda n: 0 if n <= W else -(-(n - W) // F) * F
+    ref = brute_force_attention_delegated(q, lens, k16, vc, vs, tail, s, W, F, cold, scale)
+    assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_delegated_all_hot_is_binary16_attention_of_the_inputs(orc):
+    # len <= W: nothing is quantised; the output is softmax attention over the
+    # binary16-rounded inputs themselves (no cache values read here)
+    rng = np.random.default_rng(7)
+    D, Hq, Hkv, W, F, T, B = 128, 4, 1, 32, 8, 32, 1
+    s = orc.sign_vector(0, D)
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    k16, vc, vs, tail, _ = make_delegated(orc, s, k, v, W, F)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float32)
+    for L in (1, 17, 32):
+        got, _ = orc.decode_attention_delegated(s, q, np.array([L], np.int32), k16, vc, vs, tail, W, F, 0.2)
+        K = k[0, :L, 0].astype(np.float16).astype(np.float64)
+        V = v[0, :L, 0].astype(np.float16).astype(np.float64)
+        for hq in range(Hq):
+            z = K @ q[0, hq].astype(np.float64) * 0.2
+            w = np.exp(z - z.max())
+            ref = (w / w.sum()) @ V
+            assert np.max(np.abs(got[0, hq] - ref)) < 1e-6
+
+
+def test_delegated_special_cases(orc):
+    rng = np.random.default_rng(3)
+    D, W, F = 32, 4, 2
+    s = orc.sign_vector(0, D)
+    k = rng.standard_normal((1, 6, 1, D)).astype(np.float32)
+    v = rng.standard_normal((1, 6, 1, D)).astype(np.float32)
+    v[0, 5, 0, 1] = 1.0e5  # beyond binary16
+    k16, vc, vs, tail, st = make_delegated(orc, s, k, v, W, F)
+    assert st & orc.STATUS_NONFINITE
+    assert tail[0, 5 % W, 0, 1] == 0x7C00
+    q = rng.standard_normal((1, 2, D)).astype(np.float32)
+    out, st = orc.decode_attention_delegated(s, q, np.array([0], np.int32), k16, vc, vs, tail, W, F, 0.1)
+    assert st == 0 and np.all(out == 0)
+    out, st = orc.decode_attention_delegated(s, q, np.array([7], np.int32), k16, vc, vs, tail, W, F, 0.1)
+    assert st & orc.STATUS_CAPACITY and np.all(out == 0)
+    st = orc.append_delegated(s, k[:, :1], v[:, :1], np.array([6], np.int32), W, F, k16, vc, vs, tail)
+    assert st & orc.STATUS_CAPACITY
