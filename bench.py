@@ -46,9 +46,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
     ap.add_argument("--no-references", action="store_true",
                     help="skip the quantise-throughput, bf16 dense-KV and dequantise-then-attend reference points")
-    ap.add_argument("--k-format", choices=["int4", "fp16"], default="int4",
-                    help="K storage: int4 codes like V (symmetric cache), or binary16 in the original domain "
-                         "(the asymmetric cache of the mlxcel guide's recommended mode)")
+    ap.add_argument("--k-format", choices=list(FORMATS), default="int4",
+                    help="cache format: int4 K and V (symmetric cache); binary16 K in the original domain with "
+                         "int4 V (the asymmetric cache of the mlxcel guide's recommended mode); or 'delegated', "
+                         "binary16 K with a binary16 V hot tail folded into int4 V (the guide's delegated mode)")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report instead of the step benchmark: decode and prefill-quantise "
                          "times (median, p10, p90; cold L2, and warm L2 where the cache fits) for every workload "
@@ -64,20 +65,53 @@ def get_workload(name):
 
 # ----------------------------------------------------------------------------- algorithmic bytes
 
-def decode_bytes(w, lens, kf16=False):
-    """Cache bytes the decode must read per token.kv-head: packed V codes + binary16 scales
+FORMATS = ("int4", "fp16", "delegated")
+
+
+def delegated_window():
+    from compressed_domain_attention_b200 import synthetic as syn
+    return syn.DELEGATED_WINDOW, syn.DELEGATED_FOLD
+
+
+def cold_count(n, fmt):
+    """Tokens of an n-token sequence held as int4 V codes: all of them, except in the delegated cache,
+    whose most recent tokens (between W - F + 1 and W once n > W) stay binary16 in the hot tail."""
+    if fmt != "delegated":
+        return n
+    W, F = delegated_window()
+    return 0 if n <= W else (n - W + F - 1) // F * F
+
+
+def split_bytes(w, lens, fmt="int4"):
+    """Cache bytes the split-K kernel reads: per cold token.kv-head, packed V codes + binary16 scales
     (D/2 + D/16), and the same again for int4 K or 2D for binary16 K."""
     D = w.head_dim
     v = D // 2 + 2 * (D // 32)
-    return sum(lens) * w.n_kv_heads * (v + (2 * D if kf16 else v))
+    k = v if fmt == "int4" else 2 * D
+    return sum(cold_count(n, fmt) for n in lens) * w.n_kv_heads * (v + k)
 
 
-def append_bytes(w, in_bytes=2, kf16=False):
-    """Quantise-append traffic: raw K/V in + packed codes and scales (or binary16 K) out, per appended token."""
+def decode_bytes(w, lens, fmt="int4"):
+    """Cache bytes the decode reads per step: the split-K kernel's, plus (delegated cache) the hot
+    tokens' binary16 K and V rows, which the merge kernel reads."""
     D = w.head_dim
-    v_vec = D * in_bytes + D // 2 + 2 * (D // 32)
-    k_vec = D * in_bytes + 2 * D if kf16 else v_vec
-    return w.batch * w.n_append * w.n_kv_heads * (v_vec + k_vec)
+    hot = sum(n - cold_count(n, fmt) for n in lens)
+    return split_bytes(w, lens, fmt) + hot * w.n_kv_heads * 4 * D
+
+
+def append_bytes(w, in_bytes=2, fmt="int4", lens0=None):
+    """Append traffic per step: raw K/V in, packed codes and scales (or binary16 K / binary16 V tail) out;
+    for the delegated cache also the tokens that fold out of the tail (binary16 in, codes and scales out)."""
+    D = w.head_dim
+    code = D // 2 + 2 * (D // 32)
+    v_vec = D * in_bytes + (2 * D if fmt == "delegated" else code)
+    k_vec = D * in_bytes + (code if fmt == "int4" else 2 * D)
+    total = w.batch * w.n_append * w.n_kv_heads * (v_vec + k_vec)
+    if fmt == "delegated":
+        lens0 = w.seq_lens if lens0 is None else lens0
+        folds = sum(cold_count(n + w.n_append, fmt) - cold_count(n, fmt) for n in lens0)
+        total += folds * w.n_kv_heads * (2 * D + code)
+    return total
 
 
 def load_peaks():
@@ -244,21 +278,23 @@ class OracleStep:
     re-appends the new token at position len_b and decodes over len_b + 1.
     """
 
-    def __init__(self, w, tensors, seqs, kf16=False):
+    def __init__(self, w, tensors, seqs, fmt="int4"):
         import numpy as np
         import oracle
         from compressed_domain_attention_b200 import synthetic as syn
         self.oracle, self.np = oracle, np
         D, H = w.head_dim, w.n_kv_heads
-        self.w, self.seqs, self.kf16 = w, seqs, kf16
+        self.w, self.seqs, self.fmt = w, seqs, fmt
         self.s = oracle.sign_vector(0, D)
         n = len(seqs)
         cap = max(w.seq_lens[b] for b in seqs) + 1
-        if kf16:
-            self.kc, self.ks = oracle.new_k16_cache(n, cap, H, D), None
-        else:
+        if fmt == "int4":
             self.kc, self.ks = oracle.new_cache(n, cap, H, D)
+        else:
+            self.kc, self.ks = oracle.new_k16_cache(n, cap, H, D), None
         self.vc, self.vs = oracle.new_cache(n, cap, H, D)
+        self.W, self.F = delegated_window() if fmt == "delegated" else (0, 0)
+        self.tail = oracle.new_tail(n, self.W, H, D) if fmt == "delegated" else None
         for i, b in enumerate(seqs):
             k = tensors.k[b].float().cpu().numpy()[None]
             v = tensors.v[b].float().cpu().numpy()[None]
@@ -268,19 +304,25 @@ class OracleStep:
         self.vn = np.ascontiguousarray(tensors.v_new[seqs].float().cpu().numpy())
         self.lens = np.array([w.seq_lens[b] for b in seqs], np.int32)
         sub = syn.Workload(w.name, n, w.n_q_heads, H, D, [w.seq_lens[b] for b in seqs], w.dtype, w.seed, n_append=1)
-        self.nbytes = decode_bytes(sub, [L + 1 for L in sub.seq_lens], kf16) + append_bytes(sub, kf16=kf16)
+        self.nbytes = decode_bytes(sub, [L + 1 for L in sub.seq_lens], fmt) + append_bytes(sub, fmt=fmt)
         self.ntok = int(self.lens.sum()) + n
 
     def _append(self, i0, i1, k, v, start):
         sl = slice(i0, i1)
-        if self.kf16:
+        if self.fmt == "delegated":
+            self.oracle.append_delegated(self.s, k, v, start, self.W, self.F, self.kc[sl], self.vc[sl], self.vs[sl],
+                                         self.tail[sl])
+        elif self.fmt == "fp16":
             self.oracle.quantize_append_kf16(self.s, k, v, start, self.kc[sl], self.vc[sl], self.vs[sl])
         else:
             self.oracle.quantize_append(self.s, k, v, start, self.kc[sl], self.ks[sl], self.vc[sl], self.vs[sl])
 
     def _decode(self, i0, i1, q, lens):
         sl = slice(i0, i1)
-        if self.kf16:
+        if self.fmt == "delegated":
+            self.oracle.decode_attention_delegated(self.s, q, lens, self.kc[sl], self.vc[sl], self.vs[sl],
+                                                   self.tail[sl], self.W, self.F, self.w.scale)
+        elif self.fmt == "fp16":
             self.oracle.decode_attention_kf16(self.s, q, lens, self.kc[sl], self.vc[sl], self.vs[sl], self.w.scale)
         else:
             self.oracle.decode_attention(self.s, q, lens, self.kc[sl], self.ks[sl], self.vc[sl], self.vs[sl],
@@ -320,9 +362,9 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, tensors, target_tokens, kf16=False):
+def cpu_baseline(w, tensors, target_tokens, fmt="int4"):
     seqs = oracle_sample(w, target_tokens)
-    o = OracleStep(w, tensors, seqs, kf16)
+    o = OracleStep(w, tensors, seqs, fmt)
     dt = o.run()
     line = {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
@@ -355,7 +397,7 @@ def _time_cold(fn, reps, flush, stream):
     return statistics.median(ts)
 
 
-def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, kf16=False):
+def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, fmt="int4"):
     """Quantise throughput, the bf16 dense-KV decode and dequantise-then-attend, on this GPU and workload."""
     import torch
     import torch.nn.functional as F
@@ -415,7 +457,8 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, kf16=
         torch.cuda.empty_cache()
     # 3. dequantise-then-attend (the comparison category of the Open-TQ-Metal abstract):
     #    tq_dequantize_debug to dense fp32 K/V in the original domain, then SDPA per sequence
-    if not args.no_references and not kf16 and w.batch * L.max_seq * w.n_kv_heads * w.head_dim * 4 * 2 < 24e9:
+    if (not args.no_references and fmt == "int4"
+            and w.batch * L.max_seq * w.n_kv_heads * w.head_dim * 4 * 2 < 24e9):
         Kd = torch.empty((w.batch, L.max_seq, w.n_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
         Vd = torch.empty_like(Kd)
         qf = q.float().view(w.batch, w.n_q_heads, 1, w.head_dim)
@@ -441,6 +484,59 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, kf16=
         torch.cuda.empty_cache()
     return out
 
+
+
+# ----------------------------------------------------------------------------- the cache on the device
+
+class DeviceCache:
+    """One cache format in device memory, driven through the library's C ABI (tq.py)."""
+
+    def __init__(self, w, cap, fmt, dev):
+        from compressed_domain_attention_b200 import tq
+        self.tq, self.fmt = tq, fmt
+        shape = (cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
+        if fmt == "delegated":
+            W, F = delegated_window()
+            self.L = tq.tq_cache_layout_delegated(w.batch, *shape, W, F)
+            self.l1 = tq.tq_cache_layout_delegated(1, *shape, W, F)
+        else:
+            kfmt = tq.TQ_K_INT4 if fmt == "int4" else tq.TQ_K_FP16
+            self.L = tq.tq_cache_layout_kv(w.batch, *shape, kfmt)
+            self.l1 = tq.tq_cache_layout_kv(1, *shape, kfmt)
+        self.kc, self.ks, self.vc, self.vs = tq.alloc_cache(self.L, dev)
+        self.tail = tq.alloc_tail(self.L, dev) if fmt == "delegated" else None
+        self.wsp = tq.alloc_workspace(self.L, dev)
+
+    def nbytes(self):
+        L = self.L
+        return int(L.k_bytes + L.codes_bytes + L.scales_bytes * (2 if self.fmt == "int4" else 1) + L.tail_bytes)
+
+    def append_seq(self, b, k, v, n, zero, status, stream):
+        """Prefill of sequence b alone (n tokens at position 0) through a batch-1 view."""
+        L, tq = self.L, self.tq
+        cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
+        kc, vc, vs = self.kc[b * kst:(b + 1) * kst], self.vc[b * cs:(b + 1) * cs], self.vs[b * ss:]
+        if self.fmt == "delegated":
+            ts = int(L.tail_stride_seq) // 2
+            tq.tq_append_delegated(self.l1, k, v, n, zero, kc, vc, vs, self.tail[b * ts:(b + 1) * ts], status,
+                                   stream)
+        else:
+            tq.tq_quantize_append(self.l1, k, v, n, zero, kc, None if self.ks is None else self.ks[b * ss:], vc, vs,
+                                  status, stream)
+
+    def append(self, k, v, n, start, status, stream):
+        if self.fmt == "delegated":
+            self.tq.tq_append_delegated(self.L, k, v, n, start, self.kc, self.vc, self.vs, self.tail, status, stream)
+        else:
+            self.tq.tq_quantize_append(self.L, k, v, n, start, self.kc, self.ks, self.vc, self.vs, status, stream)
+
+    def decode(self, q, lens, scale, out, status, stream, after_split_event=None):
+        if self.fmt == "delegated":
+            self.tq.tq_decode_attention_delegated(self.L, q, lens, self.kc, self.vc, self.vs, self.tail, scale, out,
+                                                  self.wsp, status, stream, after_split_event=after_split_event)
+        else:
+            self.tq.tq_decode_attention(self.L, q, lens, self.kc, self.ks, self.vc, self.vs, scale, out, self.wsp,
+                                        status, stream, after_split_event=after_split_event)
 
 
 # ----------------------------------------------------------------------------- per-configuration sweep
@@ -483,29 +579,25 @@ def run_sweep(args):
     cfgs = [("c0", syn.tiny_single_head, False), ("c1", syn.llama3_8b_layer, False)]
     cfgs += [("c2", (lambda T=T: syn.gemma3_1b_sweep(T)), False) for T in (256, 512, 1024, 2048, 4096)]
     cfgs += [("c3", syn.llama31_70b_long, False), ("c4", syn.ragged_serving, False)]
-    # the asymmetric cache (binary16 K, int4 V) on the head_dim-128 shapes
-    cfgs += [("c1", syn.llama3_8b_layer, True), ("c3", syn.llama31_70b_long, True), ("c4", syn.ragged_serving, True)]
-    for tag, make, kf16 in cfgs:
+    # the asymmetric (binary16 K, int4 V) and delegated caches on the head_dim-128 shapes
+    for fmt in ("fp16", "delegated"):
+        cfgs += [("c1", syn.llama3_8b_layer, fmt), ("c3", syn.llama31_70b_long, fmt),
+                 ("c4", syn.ragged_serving, fmt)]
+    for tag, make, fmt in cfgs:
+        fmt = fmt or "int4"
         w = make()
         t = syn.generate(w, device="cuda")
         n_app = max(w.n_append, 1)
         cap = max(w.seq_lens) + n_app
-        kfmt = tq.TQ_K_FP16 if kf16 else tq.TQ_K_INT4
-        L = tq.tq_cache_layout_kv(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
-        kc, ks, vc, vs = tq.alloc_cache(L, dev)
-        wsp = tq.alloc_workspace(L, dev)
+        cache = DeviceCache(w, cap, fmt, dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        l1 = tq.tq_cache_layout_kv(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
         zero = torch.zeros(1, dtype=torch.int32, device=dev)
-        cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
         kb = [t.k[b][None].contiguous() for b in range(w.batch)]
         vb = [t.v[b][None].contiguous() for b in range(w.batch)]
 
         def prefill():
             for b in range(w.batch):
-                tq.tq_quantize_append(l1, kb[b], vb[b], w.seq_lens[b], zero, kc[b * kst:(b + 1) * kst],
-                                      None if kf16 else ks[b * ss:], vc[b * cs:(b + 1) * cs], vs[b * ss:], status,
-                                      stream)
+                cache.append_seq(b, kb[b], vb[b], w.seq_lens[b], zero, status, stream)
 
         prefill()
         pre = _time_reps(prefill, 5, flush, stream)
@@ -515,19 +607,19 @@ def run_sweep(args):
         out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
 
         def decode():
-            tq.tq_decode_attention(L, q, lens, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
+            cache.decode(q, lens, w.scale, out, status, stream)
 
         for _ in range(10):
             decode()
         reps = 20 if sum(w.seq_lens) * w.n_kv_heads >= 1 << 20 else 100
         cold = _time_reps(decode, reps, flush, stream)
-        nbytes = decode_bytes(w, w.seq_lens, kf16)
+        nbytes = decode_bytes(w, w.seq_lens, fmt)
         warm = _time_reps(decode, reps, None, stream) if nbytes < 64e6 else None
         kn, vn = t.k_new.contiguous() if w.n_append else None, t.v_new.contiguous() if w.n_append else None
         app = None
         if w.n_append:
             def append():
-                tq.tq_quantize_append(L, kn, vn, w.n_append, lens, kc, ks, vc, vs, status, stream)
+                cache.append(kn, vn, w.n_append, lens, status, stream)
             app = _time_reps(append, 50, flush, stream)
         dense = None
         if w.dtype != torch.float32:
@@ -549,7 +641,7 @@ def run_sweep(args):
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the sweep ({w.name})")
         ms = cold["median"]
-        line = {"sweep": tag, "workload": w.name, "k_format": "fp16" if kf16 else "int4", "batch": w.batch,
+        line = {"sweep": tag, "workload": w.name, "k_format": fmt, "batch": w.batch,
                 "tokens": sum(w.seq_lens), "cache_bytes_read": nbytes,
                 "decode_ms_cold_l2": cold, "decode_gbs": round(nbytes / ms / 1e6, 1),
                 "pct_of_8_tbs": round(nbytes / ms / 1e6 / 80.0, 2),
@@ -563,7 +655,7 @@ def run_sweep(args):
                 "bf16_dense_sdpa_ms_cold_l2": dense,
                 "speedup_vs_bf16_dense": round(dense["median"] / ms, 2) if dense else None}
         print(json.dumps(line), flush=True)
-        del kc, ks, vc, vs, wsp, t, kb, vb
+        del cache, t, kb, vb
         torch.cuda.empty_cache()
     return 0
 
@@ -580,8 +672,7 @@ def run_reference(args):
         w.n_append = 1
     seqs = oracle_sample(w, 8192)
     t = syn.generate(w, device="cpu", seq_subset=seqs)
-    kf16 = getattr(args, "k_format", "int4") == "fp16"
-    o = OracleStep(w, t, seqs, kf16)
+    o = OracleStep(w, t, seqs, getattr(args, "k_format", "int4"))
     for _ in range(args.warmup):
         o.run()
     tot_t = sum(o.run() for _ in range(args.steps))
@@ -614,42 +705,40 @@ def run_tq(args):
         w.n_append = 1
     cap = max(w.seq_lens) + w.n_append
     t = syn.generate(w, device="cuda")
-    kf16 = args.k_format == "fp16"
-    kfmt = tq.TQ_K_FP16 if kf16 else tq.TQ_K_INT4
-    L = tq.tq_cache_layout_kv(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
-    kc, ks, vc, vs = tq.alloc_cache(L, dev)
-    wsp = tq.alloc_workspace(L, dev)
+    fmt = args.k_format
+    cache = DeviceCache(w, cap, fmt, dev)
+    L = cache.L
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
     # prefill (untimed): one append per sequence through a batch-1 view of the cache
-    l1 = tq.tq_cache_layout_kv(1, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, kfmt)
     zero = torch.zeros(1, dtype=torch.int32, device=dev)
-    cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
     for b in range(w.batch):
-        n = w.seq_lens[b]
-        tq.tq_quantize_append(l1, t.k[b][None], t.v[b][None], n, zero, kc[b * kst:(b + 1) * kst],
-                              None if kf16 else ks[b * ss:], vc[b * cs:(b + 1) * cs], vs[b * ss:], status)
+        cache.append_seq(b, t.k[b][None].contiguous(), t.v[b][None].contiguous(), w.seq_lens[b], zero, status,
+                         stream)
     torch.cuda.synchronize()
     lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
     lens1 = lens + w.n_append
     q = t.q.contiguous()
     k_new, v_new = t.k_new.contiguous(), t.v_new.contiguous()
     out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
 
     n_ev = args.steps
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
 
+    # One step appends each sequence's new token at its prefix length and decodes over
+    # prefix + 1, so every step repeats the same work (with the delegated cache, the
+    # same fold of the tail into the int4 body where a sequence's length crosses a
+    # fold boundary).
     def step(i=None):
-        tq.tq_quantize_append(L, k_new, v_new, w.n_append, lens, kc, ks, vc, vs, status, stream)
+        cache.append(k_new, v_new, w.n_append, lens, status, stream)
         if i is not None:
             ev_a[i].record(stream)
-            tq.tq_decode_attention(L, q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream,
-                                   after_split_event=ev_s[i])
+            cache.decode(q, lens1, w.scale, out, status, stream, after_split_event=ev_s[i])
             ev_b[i].record(stream)
         else:
-            tq.tq_decode_attention(L, q, lens1, kc, ks, vc, vs, w.scale, out, wsp, status, stream)
+            cache.decode(q, lens1, w.scale, out, status, stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -723,8 +812,8 @@ def run_tq(args):
             cs.wait_event(ev_in[j])
             if i >= 2:
                 cs.wait_event(ev_out[j])  # step i-2's output was copied out of d_out[j]
-            tq.tq_quantize_append(L, d_k[j], d_v[j], w.n_append, lens, kc, ks, vc, vs, status, cs)
-            tq.tq_decode_attention(L, d_q[j], lens1, kc, ks, vc, vs, w.scale, d_out[j], wsp, status, cs)
+            cache.append(d_k[j], d_v[j], w.n_append, lens, status, cs)
+            cache.decode(d_q[j], lens1, w.scale, d_out[j], status, cs)
             ev_done[j].record(cs)
             with torch.cuda.stream(cstream):
                 cstream.wait_event(ev_done[j])
@@ -767,22 +856,23 @@ def run_tq(args):
     if not torch.equal(h_out[(args.steps - 1) % 2], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-timed output")
 
-    refs = {} if args.no_references else reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args,
-                                                          kf16=kf16)
+    refs = {} if args.no_references else reference_points(w, t, L, cache.kc, cache.ks, cache.vc, cache.vs, lens1,
+                                                          q, dev, stream, args, fmt=fmt)
 
     lens_step = [x + w.n_append for x in w.seq_lens]
-    bytes_decode = decode_bytes(w, lens_step, kf16)
-    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4, kf16)
+    bytes_decode = decode_bytes(w, lens_step, fmt)
+    bytes_split = split_bytes(w, lens_step, fmt)
+    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4, fmt)
     max_t = max_over_ranks(elapsed, dev)
     max_e2e = max_over_ranks(e2e_s, dev)
     split_avg = max_over_ranks(statistics.mean(split_ms), dev)
     merge_avg = max_over_ranks(statistics.mean(merge_ms), dev)
 
     peak, peak_kind = load_peaks()
-    achieved = bytes_decode / (split_avg / 1e3) / 1e9
-    traffic = load_traffic(f"decode_split_kernel/{w.name}" + ("/k_fp16" if kf16 else ""))
-    kv_tokens = sum(lens_step) * w.n_kv_heads
-    cache_bytes = int(L.k_bytes + L.codes_bytes + L.scales_bytes * (1 if kf16 else 2))
+    achieved = bytes_split / (split_avg / 1e3) / 1e9
+    traffic = load_traffic(f"decode_split_kernel/{w.name}" + {"int4": "", "fp16": "/k_fp16",
+                                                                "delegated": "/delegated"}[fmt])
+    cache_bytes = cache.nbytes()
     extra = {
         "tokens_per_s": round(ws * w.batch * w.n_append * args.steps / max_t, 1),
         "kv_tokens_per_s": round(ws * sum(lens_step) * args.steps / max_t, 1),
@@ -792,7 +882,7 @@ def run_tq(args):
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": bytes_decode, "avg_launch_ms": round(split_avg, 4),
+                     "algorithmic_bytes_per_launch": bytes_split, "avg_launch_ms": round(split_avg, 4),
                      "merge_avg_ms": round(merge_avg, 4)},
         "e2e": {"value": round(ws * bytes_step * args.steps / max_e2e / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(k_new.numel() * k_new.element_size() * 2 + q.numel() * q.element_size()),
@@ -816,7 +906,7 @@ def run_tq(args):
            "algorithmic_bytes_per_step": bytes_step}
     total_bytes = sum_over_ranks(bytes_step * args.steps, dev)  # every rank takes part
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        extra["cpu_baseline"] = cpu_baseline(w, t, 300000, kf16)
+        extra["cpu_baseline"] = cpu_baseline(w, t, 300000, fmt)
     if rank == 0:
         line = assemble_line(n_gpus=ws, steps=args.steps, warmup=args.warmup, total_bytes_all_ranks=total_bytes,
                              max_time_s=max_t, workload=cfg, extra=extra)

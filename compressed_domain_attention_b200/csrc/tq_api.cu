@@ -128,11 +128,14 @@ int encode_k16_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::Ten
   return TQ_OK;
 }
 
+int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, tq_layout_t* out);
+
 int check_layout(const tq_layout_t* L) {
   if (L == nullptr) return TQ_ERR_INVALID_ARG;
   tq_layout_t chk;
-  const int r = tq_cache_layout_kv(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
-                                   L->sign_seed, L->k_format, &chk);
+  const int r = build_layout(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
+                             L->sign_seed, L->k_format, L->tail_window, L->fold_chunk, &chk);
   if (r != TQ_OK) return r;
   if (std::memcmp(&chk, L, sizeof(chk)) != 0) return TQ_ERR_INVALID_ARG;  // edited or stale layout
   return TQ_OK;
@@ -142,27 +145,29 @@ void copy_signs(const tq_layout_t* L, uint64_t (&dst)[4]) {
   for (int i = 0; i < 4; ++i) dst[i] = L->sign_bits[i];
 }
 
-uint64_t workspace_bytes(int batch, int n_q, int D, int max_ctas) {
-  const uint64_t slots = (uint64_t)max_ctas + (uint64_t)batch;
+// Split-K partial slots (one per CTA plus one per sequence for ranges that
+// straddle sequences) and, for the delegated cache, the hot-tail partials.
+uint64_t workspace_bytes(int batch, int n_q, int D, int max_ctas, int tail_window = 0) {
+  const uint64_t slots =
+      (uint64_t)max_ctas + (uint64_t)batch + (uint64_t)batch * (uint64_t)tqk::tail_chunk_count(tail_window);
   const uint64_t header = 8ull * (uint64_t)(batch + 2);
   const uint64_t ml = slots * (uint64_t)n_q * 2ull * 4ull;
   const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
   return ((header + ml + 255) / 256) * 256 + acc;
 }
 
-}  // namespace
+constexpr int kMaxTailWindow = 1024;  // the merge kernel keeps one score per hot token in shared memory
 
-extern "C" {
-
-int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
-                    uint64_t sign_seed, tq_layout_t* out) {
-  return tq_cache_layout_kv(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_K_INT4, out);
-}
-
-int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
-                       uint64_t sign_seed, int k_format, tq_layout_t* out) {
+int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, tq_layout_t* out) {
   if (out == nullptr) return TQ_ERR_INVALID_ARG;
-  if (k_format != TQ_K_INT4 && k_format != TQ_K_FP16) return TQ_ERR_INVALID_ARG;
+  if (k_format != TQ_K_INT4 && k_format != TQ_K_FP16 && k_format != TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  if (k_format == TQ_KV_DELEGATED) {
+    if (tail_window < 1 || tail_window > kMaxTailWindow || fold_chunk < 1 || fold_chunk > tail_window)
+      return TQ_ERR_INVALID_ARG;
+  } else if (tail_window != 0 || fold_chunk != 0) {
+    return TQ_ERR_INVALID_ARG;
+  }
   if (batch <= 0 || max_seq <= 0 || n_kv_heads <= 0 || n_q_heads <= 0) return TQ_ERR_INVALID_ARG;
   if (n_q_heads % n_kv_heads != 0) return TQ_ERR_INVALID_ARG;
   // mlxcel §"Known limitations / head dimension": power-of-two head dims only.
@@ -191,9 +196,10 @@ int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, in
   const uint64_t srow = (uint64_t)L.scale_stride_tok * 2ull;
   L.scales_bytes = (uint64_t)batch * (uint64_t)L.scale_stride_seq * 2ull + kMaxTileTokens * srow + 32ull;
   L.max_ctas = kMaxCtas;
-  L.decode_workspace_bytes = workspace_bytes(batch, n_q_heads, head_dim, kMaxCtas);
+  L.decode_workspace_bytes =
+      workspace_bytes(batch, n_q_heads, head_dim, kMaxCtas, k_format == TQ_KV_DELEGATED ? tail_window : 0);
   L.k_format = k_format;
-  if (k_format == TQ_K_FP16) {
+  if (k_format != TQ_K_INT4) {
     L.k_stride_tok = (int64_t)n_kv_heads * head_dim * 2;
     L.k_stride_seq = (int64_t)max_seq * L.k_stride_tok;
     L.k_bytes = (uint64_t)batch * (uint64_t)L.k_stride_seq;
@@ -202,24 +208,60 @@ int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, in
     L.k_stride_seq = L.code_stride_seq;
     L.k_bytes = L.codes_bytes;
   }
+  if (k_format == TQ_KV_DELEGATED) {
+    L.tail_window = tail_window;
+    L.fold_chunk = fold_chunk;
+    L.tail_stride_tok = (int64_t)n_kv_heads * head_dim * 2;
+    L.tail_stride_seq = (int64_t)tail_window * L.tail_stride_tok;
+    L.tail_bytes = (uint64_t)batch * (uint64_t)L.tail_stride_seq;
+  }
   *out = L;
   return TQ_OK;
 }
 
-int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
-                       const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
-                       uint16_t* v_scales, int32_t* d_status, void* stream) {
-  int r = check_layout(layout);
-  if (r != TQ_OK) return r;
+}  // namespace
+
+extern "C" {
+
+int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                    uint64_t sign_seed, tq_layout_t* out) {
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_K_INT4, 0, 0, out);
+}
+
+int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                       uint64_t sign_seed, int k_format, tq_layout_t* out) {
+  if (k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;  // needs the window sizes
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, k_format, 0, 0, out);
+}
+
+int tq_cache_layout_delegated(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                              uint64_t sign_seed, int tail_window, int fold_chunk, tq_layout_t* out) {
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_KV_DELEGATED,
+                      tail_window, fold_chunk, out);
+}
+
+int64_t tq_cold_length(const tq_layout_t* layout, int64_t len) {
+  if (layout == nullptr || len < 0) return -1;
+  return tqk::cold_tokens(len, layout->tail_window, layout->fold_chunk);
+}
+
+namespace {
+
+int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
+                uint16_t* v_scales, uint16_t* v_tail, int32_t* d_status, void* stream) {
   if (n_new < 0) return TQ_ERR_INVALID_ARG;
   if (n_new > layout->max_seq) return TQ_ERR_CAPACITY;
   if (in_dtype != TQ_F32 && in_dtype != TQ_BF16 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
   if (n_new == 0) return TQ_OK;
-  const bool kf16 = layout->k_format == TQ_K_FP16;
-  if (!k || !v || !d_start_pos || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales)
+  const bool kf16 = layout->k_format != TQ_K_INT4;
+  const bool deleg = layout->k_format == TQ_KV_DELEGATED;
+  if (!k || !v || !d_start_pos || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales || (deleg && !v_tail))
     return TQ_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes)) return TQ_ERR_INVALID_ARG;
-  if ((int64_t)layout->batch * n_new * layout->n_kv_heads * layout->n_groups * 2 > (int64_t)INT32_MAX * 256)
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes) || (deleg && !aligned16(v_tail)))
+    return TQ_ERR_INVALID_ARG;
+  const int64_t v_rows = (int64_t)n_new + (deleg ? layout->tail_window : 0);
+  if ((int64_t)layout->batch * v_rows * layout->n_kv_heads * layout->n_groups * 2 > (int64_t)INT32_MAX * 256)
     return TQ_ERR_UNSUPPORTED;
   tqk::QuantizeParams p;
   p.k = k;
@@ -238,28 +280,56 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
   copy_signs(layout, p.sign_bits);
   p.c_d = layout->c_d;
   p.k_f16 = kf16 ? 1 : 0;
+  p.v_tail = v_tail;
+  p.tail_window = layout->tail_window;
+  p.fold_chunk = layout->fold_chunk;
   cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
 
-int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
-                           const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes,
-                           const uint16_t* v_scales, float sm_scale, float* out, void* workspace, size_t ws_bytes,
-                           int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+}  // namespace
+
+int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                       const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
+                       uint16_t* v_scales, int32_t* d_status, void* stream) {
   int r = check_layout(layout);
   if (r != TQ_OK) return r;
+  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
+                     d_status, stream);
+}
+
+int tq_append_delegated(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                        const int32_t* d_start_pos, uint16_t* k_f16, uint8_t* v_codes, uint16_t* v_scales,
+                        uint16_t* v_tail, int32_t* d_status, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->k_format != TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, reinterpret_cast<uint8_t*>(k_f16), nullptr,
+                     v_codes, v_scales, v_tail, d_status, stream);
+}
+
+namespace {
+
+int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes, const uint16_t* v_scales,
+                const uint16_t* v_tail, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+  int r = TQ_OK;
   const int D = layout->head_dim, Hkv = layout->n_kv_heads, Hq = layout->n_q_heads;
   const int G = Hq / Hkv;
   if (layout->batch > kMaxBatchDecode) return TQ_ERR_UNSUPPORTED;
   if (!(Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) || G > 8) return TQ_ERR_UNSUPPORTED;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
-  const bool kf16 = layout->k_format == TQ_K_FP16;
+  const bool kf16 = layout->k_format != TQ_K_INT4;
+  const bool deleg = layout->k_format == TQ_KV_DELEGATED;
   // binary16 K tiles: the stage ring holds them only up to head_dim 128
   if (kf16 && D > 128) return TQ_ERR_UNSUPPORTED;
-  if (!q || !d_seq_lens || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales || !out || !workspace)
+  if (!q || !d_seq_lens || !k_codes || (!kf16 && !k_scales) || !v_codes || !v_scales || !out || !workspace ||
+      (deleg && !v_tail))
     return TQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || (!kf16 && !aligned16(k_scales)) ||
-      !aligned16(v_scales) || !aligned16(out) || !aligned16(workspace))
+      !aligned16(v_scales) || !aligned16(out) || !aligned16(workspace) || (deleg && !aligned16(v_tail)))
     return TQ_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return TQ_ERR_INVALID_ARG;
   int sms = 0;
@@ -276,7 +346,8 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
     ev = reinterpret_cast<cudaEvent_t>(opts->after_split_event);
   }
   if (grid > layout->max_ctas) grid = layout->max_ctas;
-  if (ws_bytes < workspace_bytes(layout->batch, Hq, D, grid)) return TQ_ERR_INVALID_ARG;
+  const int W = deleg ? layout->tail_window : 0;
+  if (ws_bytes < workspace_bytes(layout->batch, Hq, D, grid, W)) return TQ_ERR_INVALID_ARG;
   if (tqk::decode_smem_bytes(D, Hkv, kf16 ? 1 : 0) <= 0) return TQ_ERR_UNSUPPORTED;
 
   tqk::TensorMap128 km, vm;
@@ -292,8 +363,9 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
   p.seq_lens = d_seq_lens;
   p.k_scales = k_scales;
   p.v_scales = v_scales;
-  const uint64_t header_ml =
-      ((8ull * (uint64_t)(layout->batch + 2) + (uint64_t)(grid + layout->batch) * Hq * 8ull + 255) / 256) * 256;
+  const uint64_t slots =
+      (uint64_t)grid + (uint64_t)layout->batch + (uint64_t)layout->batch * (uint64_t)tqk::tail_chunk_count(W);
+  const uint64_t header_ml = ((8ull * (uint64_t)(layout->batch + 2) + slots * Hq * 8ull + 255) / 256) * 256;
   p.ws_ml = reinterpret_cast<float*>(workspace);
   p.ws_acc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + header_ml);
   p.out = out;
@@ -309,8 +381,38 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
   p.c_d = layout->c_d;
   copy_signs(layout, p.sign_bits);
   p.k_f16 = kf16 ? 1 : 0;
+  p.k16 = kf16 ? reinterpret_cast<const uint16_t*>(k_codes) : nullptr;
+  p.v_tail = v_tail;
+  p.tail_window = layout->tail_window;
+  p.fold_chunk = layout->fold_chunk;
+  p.tail_chunks = tqk::tail_chunk_count(W);
+  p.tail_slot0 = grid + layout->batch;
   cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                           const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes,
+                           const uint16_t* v_scales, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                           int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  return decode_impl(layout, q, q_dtype, d_seq_lens, k_codes, k_scales, v_codes, v_scales, nullptr, sm_scale, out,
+                     workspace, ws_bytes, d_status, opts, stream);
+}
+
+int tq_decode_attention_delegated(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                                  const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales,
+                                  const uint16_t* v_tail, float sm_scale, float* out, void* workspace,
+                                  size_t ws_bytes, int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->k_format != TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  return decode_impl(layout, q, q_dtype, d_seq_lens, reinterpret_cast<const uint8_t*>(k_f16), nullptr, v_codes,
+                     v_scales, v_tail, sm_scale, out, workspace, ws_bytes, d_status, opts, stream);
 }
 
 int tq_decode_attention(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,

@@ -129,7 +129,7 @@ __device__ void block_prefix_lengths(const DecodeParams& p, int64_t* prefix, int
     int64_t L = 0;
     if (b < p.batch) {
       const int x = p.seq_lens[b];
-      if (x < 0 || x > p.max_seq) bad = true; else L = x;
+      if (x < 0 || x > p.max_seq) bad = true; else L = cold_tokens(x, p.tail_window, p.fold_chunk);
     }
     v[i] = L;
     local += L;
@@ -1017,6 +1017,290 @@ __global__ void __launch_bounds__(kThreads, 1)
 // NTH = 128 threads (8 blocks per SM) when there are many (sequence, head)
 // pairs, 1024 when there are fewer than twice the SMs: a long sequence then has
 // up to one partial per SM, and its loads should all be in flight at once.
+// Kernel 1b (decode_tail_kernel, delegated cache only): attention partials over
+// the hot tail (mlxcel guide, delegated cache variant: the recent tokens keep
+// binary16 K and V). One block per (sequence, kv head, chunk of kTailTokens hot
+// tokens) computes the partial (running max in log2 units, sum, accumulator) of
+// every q head of the group, so each binary16 K and V row is read once per kv
+// head: the chunk's K and V rows are staged in shared memory by cp.async (all
+// copies in flight together, 16-byte pieces XOR-swizzled by row so that
+// ldmatrix is conflict-free), then each of the 4 warps takes 16 tokens on the
+// tensor cores (mma.m16n8k16, f16 in, f32 accumulate), as in the split-K kernel:
+//   Q.K^T  A rows 0-7 = the binary16 hi piece of q head 0-7 (scaled by 2^sh so
+//          that its largest element is below 2^14), rows 8-15 = the lo piece;
+//          B = K rows (exact); the score is the sum of the two rows times 2^-sh;
+//   P.V    A rows 0-7 = binary16 of the weights p = 2^(s - m), rows 8-15 = the
+//          binary16 of their residual; B = V rows through a transposing ldmatrix.
+// The warps' partials share the block's running max and are summed in shared
+// memory. The accumulator is mapped into the rotated domain by the forward SRHT
+// (c_D H (s o x); the transform is linear), so the merge kernel combines it like
+// any split-K partial and its single inverse SRHT brings the output back.
+// Chunks past a sequence's hot tokens write empty partials (m = -inf, l = 0).
+// The inputs were complete before the split-K grid started, so the work runs
+// before the dependency wait; the wait comes last, so that this grid completes
+// only after the split-K grid, and the merge kernel's wait covers both.
+constexpr int kTailTokens = 64;  // tail_chunk_count() in tq_kernels.h uses the same 64
+constexpr int kTailThreads = 128;
+constexpr int kMaxTailChunks = 16;  // tail windows up to 1024 tokens
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// 16-byte piece c of row j of a [rows][D] binary16 tile, XOR-swizzled so that 8
+// consecutive rows at one piece index fall in 8 different bank groups.
+template <int D>
+__device__ __forceinline__ int tile_piece(int j, int c) {
+  return (D >= 64) ? (c ^ (j & 7)) : (c ^ ((j >> 1) & 3));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTailThreads) decode_tail_kernel(const __grid_constant__ DecodeParams p) {
+  static_assert(D <= 128, "binary16 K rows up to head_dim 128");
+  constexpr int CPR = D / 8;  // 16-byte pieces per row
+  constexpr int KS = D / 16;  // k-steps of the scores
+  constexpr int NT = D / 8;   // n-tiles (8 dims) of P.V
+  constexpr int NW = kTailThreads / 32;
+  constexpr int PP = D + 8;   // padded row of the warp partials (floats)
+  __shared__ __align__(128) uint16_t tiles[2 * kTailTokens * D];  // K rows, then V rows
+  __shared__ float mred[NW][8];
+  __shared__ float lred[NW][8];
+  uint16_t* ks = tiles;
+  uint16_t* vsm = tiles + kTailTokens * D;
+  float* part = reinterpret_cast<float*>(tiles);  // [NW][8][PP] after P.V
+  static_assert(NW * 8 * PP * 4 <= (int)sizeof(tiles), "warp partials fit in the K and V tiles");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int nch = p.tail_chunks;
+  const int chunk = blockIdx.x % nch;
+  const int bh = blockIdx.x / nch;
+  const int kvh = bh % p.n_kv, b = bh / p.n_kv;
+  const int G = p.group, W = p.tail_window;
+  int len = p.seq_lens[b];
+  if (len < 0 || len > p.max_seq) len = 0;
+  const int t_lo = (int)cold_tokens(len, W, p.fold_chunk) + chunk * kTailTokens;
+  const int n = max(0, min(len, t_lo + kTailTokens) - t_lo);
+  const int64_t slot = (int64_t)p.tail_slot0 + (int64_t)b * nch + chunk;
+  float* ml = p.ws_ml + 2 * (p.batch + 2) + (slot * p.n_q + (int64_t)kvh * G) * 2;
+  float* acc_out = p.ws_acc + (slot * p.n_q + (int64_t)kvh * G) * D;
+  if (n == 0) {
+    for (int i = tid; i < G; i += kTailThreads) {
+      ml[2 * i] = -INFINITY;
+      ml[2 * i + 1] = 0.f;
+    }
+    for (int i = tid; i < G * D; i += kTailThreads) acc_out[i] = 0.f;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
+  // stage the chunk's K rows and V tail rows; V rows past n are zeroed (their
+  // weights are 0, but 0 * NaN would not be)
+  {
+    const int64_t rstride = (int64_t)p.n_kv * D;  // binary16 elements between tokens (K) or slots (V)
+    const uint16_t* kg = p.k16 + (((int64_t)b * p.max_seq + t_lo) * p.n_kv + kvh) * D;
+    const uint16_t* vg = p.v_tail + ((int64_t)b * W * p.n_kv + kvh) * D;
+    const int c = tid % CPR;
+    constexpr int RSTEP = kTailThreads / CPR;
+    int j = tid / CPR;
+    int slot_v = (t_lo + j) % W;
+    for (; j < kTailTokens; j += RSTEP) {
+      const int pc = tile_piece<D>(j, c);
+      if (j < n) {
+        cp_async16(smem_u32(&ks[j * D + pc * 8]), kg + (int64_t)j * rstride + c * 8);
+        cp_async16(smem_u32(&vsm[j * D + pc * 8]), vg + (int64_t)slot_v * rstride + c * 8);
+      } else {
+        *reinterpret_cast<uint4*>(&vsm[j * D + pc * 8]) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      slot_v += RSTEP;
+      while (slot_v >= W) slot_v -= W;
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  // A fragments of the scores: head gid's hi (rows 0-7) and lo (rows 8-15) pieces,
+  // dims 16 kk + 2 tig + {0, 1} (a0, a1) and 16 kk + 8 + 2 tig + {0, 1} (a2, a3)
+  uint32_t qa[KS][4];
+  float f_h = 1.f;
+  {
+    float x[KS][4];
+    float mx = 0.f;
+    const bool has = gid < G;
+    const int64_t qoff = ((int64_t)b * p.n_q + (int64_t)kvh * G + gid) * D;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int d = 16 * kk + 8 * (e >> 1) + 2 * tig + (e & 1);
+        x[kk][e] = has ? load_scalar(p.q, qoff + d, p.q_dtype) * p.sm_scale_log2 : 0.f;
+        mx = fmaxf(mx, fabsf(x[kk][e]));
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    int ex = 0;
+    if (mx > 0.f) (void)frexpf(mx, &ex);
+    const int sh = min(100, max(-100, 14 - ex));  // scaled max < 2^14
+    const float sc = __int_as_float((127 + sh) << 23);
+    f_h = __int_as_float((127 - sh) << 23);
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 v = make_float2(x[kk][2 * h] * sc, x[kk][2 * h + 1] * sc);
+        const __half2 hi = __float22half2_rn(v);
+        const float2 hf = __half22float2(hi);
+        const __half2 lo = __float22half2_rn(make_float2(v.x - hf.x, v.y - hf.y));
+        qa[kk][2 * h] = *reinterpret_cast<const uint32_t*>(&hi);
+        qa[kk][2 * h + 1] = *reinterpret_cast<const uint32_t*>(&lo);
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // scores of this warp's 16 tokens: two n-tiles of 8
+  const int tok0 = wp * 16;
+  float c[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+  {
+    const int mi = lane >> 3, r = lane & 7;
+    const int row = tok0 + 8 * (mi >> 1) + r;  // matrices: (n-tile 0, piece 2kk), (0, 2kk+1), (1, 2kk), (1, 2kk+1)
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t bf[4];
+      ldmatrix_x4(bf, smem_u32(&ks[row * D + tile_piece<D>(row, 2 * kk + (mi & 1)) * 8]));
+      mma_f16_16816_acc(c[0], qa[kk], bf[0], bf[1]);
+      mma_f16_16816_acc(c[1], qa[kk], bf[2], bf[3]);
+    }
+  }
+  // s for head gid at tokens tok0 + 8 nt + 2 tig + e; masked past n
+  float sv[2][2];
+  float mloc = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = tok0 + 8 * nt + 2 * tig + e;
+      const float v = (c[nt][e] + c[nt][2 + e]) * f_h;
+      sv[nt][e] = t < n ? v : -INFINITY;
+      mloc = fmaxf(mloc, sv[nt][e]);
+    }
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  if (tig == 0) mred[wp][gid] = mloc;
+  __syncthreads();
+  float m = mred[0][gid];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) m = fmaxf(m, mred[w][gid]);
+  // weights, their sum, and the A fragments (hi rows 0-7, residual rows 8-15)
+  float lsum = 0.f;
+  uint32_t pa[4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const float p0 = (sv[nt][0] == -INFINITY) ? 0.f : exp2f(sv[nt][0] - m);
+    const float p1 = (sv[nt][1] == -INFINITY) ? 0.f : exp2f(sv[nt][1] - m);
+    lsum += p0 + p1;
+    const __half2 hi = __float22half2_rn(make_float2(p0, p1));
+    const float2 hf = __half22float2(hi);
+    const __half2 lo = __float22half2_rn(make_float2(p0 - hf.x, p1 - hf.y));
+    pa[2 * nt] = *reinterpret_cast<const uint32_t*>(&hi);
+    pa[2 * nt + 1] = *reinterpret_cast<const uint32_t*>(&lo);
+  }
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+  if (tig == 0) lred[wp][gid] = lsum;
+  // P.V over this warp's 16 tokens: B = V rows (k = tokens, n = dims) via ldmatrix.trans
+  float o[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  {
+    const int mi = lane >> 3, r = lane & 7;
+    const int row = tok0 + 8 * (mi & 1) + r;  // matrices: (tokens 0-7, piece dn), (8-15, dn), (0-7, dn+1), (8-15, dn+1)
+#pragma unroll
+    for (int dn = 0; dn < NT; dn += 2) {
+      uint32_t bf[4];
+      ldmatrix_x4_trans(bf, smem_u32(&vsm[row * D + tile_piece<D>(row, dn + (mi >> 1)) * 8]));
+      mma_f16_16816_acc(o[dn], pa, bf[0], bf[1]);
+      mma_f16_16816_acc(o[dn + 1], pa, bf[2], bf[3]);
+    }
+  }
+  __syncthreads();  // every warp is done with the K and V tiles: part[] may overwrite them
+  // head gid, dims 8 dn + 2 tig + {0, 1}: hi row plus residual row
+#pragma unroll
+  for (int dn = 0; dn < NT; ++dn)
+    *reinterpret_cast<float2*>(part + (wp * 8 + gid) * PP + 8 * dn + 2 * tig) =
+        make_float2(o[dn][0] + o[dn][2], o[dn][1] + o[dn][3]);
+  __syncthreads();
+  // sum the warps and apply the signs (in place in warp 0's rows)
+  for (int i = tid; i < G * D; i += kTailThreads) {
+    const int g = i / D, d = i % D;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) sum += part[(w * 8 + g) * PP + d];
+    part[g * PP + d] = apply_sign(sum, p.sign_bits, d);
+  }
+  if (tid < G) {
+    float mt = mred[0][tid], l = 0.f;
+#pragma unroll
+    for (int w = 1; w < NW; ++w) mt = fmaxf(mt, mred[w][tid]);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) l += lred[w][tid];
+    ml[2 * tid] = mt;
+    ml[2 * tid + 1] = l;
+  }
+  __syncthreads();
+  // forward SRHT, one warp per q head
+  constexpr int EPL = D / 32;  // elements per lane, consecutive
+  for (int g = wp; g < G; g += NW) {
+    float u[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) u[i] = part[g * PP + lane * EPL + i];
+    // butterflies of stride < EPL inside the lane, then across lanes
+#pragma unroll
+    for (int h = 1; h < EPL; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        if ((i & h) == 0) {
+          const float a = u[i], bb = u[i + h];
+          u[i] = a + bb;
+          u[i + h] = a - bb;
+        }
+      }
+    }
+#pragma unroll
+    for (int lm = 1; lm < 32; lm <<= 1) {
+      const bool upper = (lane & lm) != 0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, u[i], lm);
+        u[i] = upper ? other - u[i] : u[i] + other;
+      }
+    }
+    float* dst = acc_out + (int64_t)g * D + lane * EPL;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) dst[i] = u[i] * p.c_d;
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <int D>
+static cudaError_t launch_tail(const DecodeParams& p, cudaStream_t s, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.batch * p.n_kv * p.tail_chunks));
+  cfg.blockDim = dim3(kTailThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_tail_kernel<D>, p);
+}
+
 template <int D, int NTH>
 __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NG = D / 32;
@@ -1024,8 +1308,8 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   constexpr int PH = NTH / F4;         // slot phases
   constexpr int PF = 8;                // loads in flight per thread
   constexpr int MAX_SLOTS = 1024;      // a sequence meets at most one partial per split-K CTA
-  __shared__ float wts[MAX_SLOTS];
-  __shared__ float lsv[MAX_SLOTS];
+  __shared__ float wts[MAX_SLOTS + kMaxTailChunks];
+  __shared__ float lsv[MAX_SLOTS + kMaxTailChunks];
   __shared__ float red[NTH / 32];
   __shared__ __align__(16) float accs[PH][D];
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
@@ -1034,13 +1318,16 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   // split-K kernel's rules (lengths outside [0, max_seq] count as 0). The lengths are
   // read before the dependency wait: this grid is launched only once every split-K
   // block has passed its own wait, so whatever wrote them has completed.
+  // With a hot tail (delegated cache) the split-K kernel covered only each sequence's
+  // cold tokens, and so do these ranges.
   __shared__ long long red64[2][NTH / 32];
   long long before = 0, total = 0;
   for (int i = tid; i < p.batch; i += NTH) {
     int x = p.seq_lens[i];
     if (x < 0 || x > p.max_seq) x = 0;
-    total += x;
-    if (i < b) before += x;
+    const long long c = cold_tokens(x, p.tail_window, p.fold_chunk);
+    total += c;
+    if (i < b) before += c;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -1059,38 +1346,49 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
     before += red64[0][w];
     total += red64[1][w];
   }
-  int len_b = p.seq_lens[b];
-  if (len_b < 0 || len_b > p.max_seq) len_b = 0;
+  int len_all = p.seq_lens[b];
+  if (len_all < 0 || len_all > p.max_seq) len_all = 0;
+  const int64_t len_b = cold_tokens(len_all, p.tail_window, p.fold_chunk);
   int64_t R = (total + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
   R = ((R + 15) / 16) * 16;
   const int64_t P0 = before, P1 = before + len_b;
+  // Delegated cache: the hot tail's partials (one per chunk of hot tokens, in the
+  // rotated domain like the rest) follow in slots tail_slot0 + b * tail_chunks + k.
+  const int n_tail = (p.tail_window > 0 && len_all > 0) ? p.tail_chunks : 0;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
-  if (P1 <= P0) {  // empty sequence
+  if (P1 <= P0 && n_tail == 0) {  // empty sequence
     for (int d = tid; d < D; d += NTH) out[d] = 0.f;
     return;
   }
-  const int c0 = (int)(P0 / R), c1 = (int)((P1 - 1) / R);
-  const int ns = min(c1 - c0 + 1, MAX_SLOTS);
+  const int c0 = P1 > P0 ? (int)(P0 / R) : 0, c1 = P1 > P0 ? (int)((P1 - 1) / R) : -1;
+  const int ns_cold = min(c1 - c0 + 1, MAX_SLOTS);
+  const int ns = ns_cold + n_tail;
+  const int64_t tail_first = (int64_t)p.tail_slot0 + (int64_t)b * p.tail_chunks;
   const float* mlb = ml + ((int64_t)(b + c0) * p.n_q + hq) * 2;
+  const float* mlt = ml + (tail_first * p.n_q + hq) * 2;
   const int64_t mls = (int64_t)p.n_q * 2;
   const int col = tid % F4, ph = tid / F4;
   const float4* base = reinterpret_cast<const float4*>(p.ws_acc) + ((int64_t)(b + c0) * p.n_q + hq) * F4 + col;
+  const float4* tbase = reinterpret_cast<const float4*>(p.ws_acc) + (tail_first * p.n_q + hq) * F4 + col;
   const int64_t stride = (int64_t)p.n_q * F4;
+  auto acc_at = [&](int i) {  // partial i: the cold run first, then the tail run
+    return i < ns_cold ? base + (int64_t)i * stride : tbase + (int64_t)(i - ns_cold) * stride;
+  };
   // The accumulator loads of the first chunk do not depend on the weights: issue them
   // together with the (m, l) loads, so the merge costs about one memory round trip.
   float4 v[PF];
 #pragma unroll
   for (int k = 0; k < PF; ++k) {
     const int i = ph + k * PH;
-    v[k] = i < ns ? __ldcg(base + (int64_t)i * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[k] = i < ns ? __ldcg(acc_at(i)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l
   float m = -INFINITY;
   for (int i = tid; i < ns; i += NTH) {
-    const float2 e = __ldcg(reinterpret_cast<const float2*>(mlb + i * mls));
+    const float2 e = __ldcg(reinterpret_cast<const float2*>(i < ns_cold ? mlb + i * mls : mlt + (i - ns_cold) * mls));
     wts[i] = e.x;
     lsv[i] = e.y;
     m = fmaxf(m, e.x);
@@ -1133,7 +1431,7 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
 #pragma unroll
     for (int k = 0; k < PF; ++k) {
       const int i = i0 + PH * PF + k * PH;
-      v[k] = i < ns ? __ldcg(base + (int64_t)i * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[k] = i < ns ? __ldcg(acc_at(i)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   reinterpret_cast<float4*>(accs[ph])[col] = a;
@@ -1187,9 +1485,15 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M, KF16>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
   const bool few = (int64_t)p.batch * p.n_q < 2 * (int64_t)p.grid;  // merge blocks vs SMs
-  if (ev != nullptr) {  // timing split: plain stream order between the two kernels
+  if (ev != nullptr) {  // timing split: plain stream order between the kernels
     e = cudaEventRecord(ev, s);
     if (e != cudaSuccess) return e;
+    if constexpr (D <= 128) {
+      if (p.tail_window > 0) {
+        e = launch_tail<D>(p, s, false);
+        if (e != cudaSuccess) return e;
+      }
+    }
     if (few)
       decode_merge_kernel<D, 1024><<<p.batch * p.n_q, 1024, 0, s>>>(p);
     else
@@ -1197,7 +1501,15 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
     return cudaGetLastError();
   }
   // programmatic dependent launch: the merge grid is set up while the split-K
-  // grid drains; griddepcontrol.wait in the merge kernel orders the reads.
+  // grid drains; griddepcontrol.wait in the merge kernel orders the reads. With a
+  // hot tail its kernel sits in between: it starts as split-K blocks finish, and
+  // completes only after the split-K grid (its own wait comes last).
+  if constexpr (D <= 128) {
+    if (p.tail_window > 0) {
+      e = launch_tail<D>(p, s, true);
+      if (e != cudaSuccess) return e;
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.batch * p.n_q));
   cfg.blockDim = dim3(few ? 1024 : kMergeThreads);

@@ -20,6 +20,9 @@ struct QuantizeParams {
   uint64_t sign_bits[4];
   float c_d;
   int k_f16;  // 1: K is stored as binary16 of the input (k_codes is that buffer), k_scales unused
+  // delegated cache (tail_window > 0, with k_f16): binary16 V hot tail [batch][W][n_kv][D]
+  uint16_t* v_tail;
+  int tail_window, fold_chunk;
 };
 
 struct DequantParams {
@@ -55,7 +58,24 @@ struct DecodeParams {
   float c_d;
   uint64_t sign_bits[4];
   int k_f16;  // 1: K tiles are binary16 (original domain), no K scales
+  // delegated cache (tail_window > 0, with k_f16): the split-K kernel covers the cold
+  // tokens; the merge kernel attends to the hot ones (binary16 K rows and V tail)
+  const uint16_t* k16;
+  const uint16_t* v_tail;
+  int tail_window, fold_chunk;
+  int tail_chunks;  // hot-tail partials per sequence (ceil(tail_window / 64)); 0 without a tail
+  int tail_slot0;   // workspace slot of sequence 0's first hot-tail partial (after the split-K slots)
 };
+
+// Hot-tail partials per sequence of the delegated cache (64 tokens each).
+__host__ __device__ __forceinline__ int tail_chunk_count(int W) { return W > 0 ? (W + 63) / 64 : 0; }
+
+// Cold (int4) tokens of a delegated-cache sequence of len tokens (all of them without a tail).
+__host__ __device__ __forceinline__ int64_t cold_tokens(int64_t len, int W, int F) {
+  if (W <= 0) return len;
+  if (len <= W) return 0;
+  return (len - W + F - 1) / F * F;
+}
 
 cudaError_t launch_quantize(const QuantizeParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int head_dim, cudaStream_t s);

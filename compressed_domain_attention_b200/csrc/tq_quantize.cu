@@ -56,6 +56,28 @@ __device__ __forceinline__ void copy_k_f16(const QuantizeParams& p, int64_t kt) 
   for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
 }
 
+// Delegated cache: store the binary16 of the thread's 32 input V elements in the
+// hot tail at slot pos % W (non-finite results set the status, as for K).
+template <int D>
+__device__ __forceinline__ void write_tail_f16(const QuantizeParams& p, int64_t in_row, int b, int h, int part,
+                                               int64_t pos) {
+  float u[32];
+  load32(u, p.v, in_row * D + part * 32, p.in_dtype);
+  uint32_t w[16];
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const __half2 hv = __floats2half2_rn(u[2 * i], u[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    finite = finite && ((w[i] & 0x7C00u) != 0x7C00u) && ((w[i] & 0x7C000000u) != 0x7C000000u);
+  }
+  if (!finite) status_or(p.status, TQ_STATUS_NONFINITE);
+  const int64_t slot = ((int64_t)b * p.tail_window + pos % p.tail_window) * p.n_kv + h;
+  uint4* dst = reinterpret_cast<uint4*>(p.v_tail + slot * D + part * 32);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantizeParams p) {
   // Launched as a programmatic dependent of the previous kernel on the stream:
@@ -65,42 +87,109 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int NG = D / 32;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t vecs_per_tensor = (int64_t)p.batch * p.n_new * p.n_kv;
-  const int64_t thr_per_tensor = vecs_per_tensor * NG;
+  const int W = p.tail_window;  // > 0 only for the delegated cache
+  const int64_t vecs_k = (int64_t)p.batch * p.n_new * p.n_kv;
+  // V work items per (sequence, head): the new tokens, then (delegated) W fold candidates
+  const int v_rows = p.n_new + W;
   int64_t vec = gt / NG;
   const int part = (int)(gt % NG);
+  int which;
+  int64_t r;
+  bool in_range;
   if (p.k_f16) {
     // V threads first, then the K copies from the next warp boundary on, so that a
     // warp is all V (its lanes exchange butterflies) or all K.
-    const int64_t kbase = (thr_per_tensor + 31) / 32 * 32;
+    const int64_t thr_v = (int64_t)p.batch * v_rows * p.n_kv * NG;
+    const int64_t kbase = (thr_v + 31) / 32 * 32;
     if (gt >= kbase) {
-      if (gt - kbase < thr_per_tensor) copy_k_f16<D>(p, gt - kbase);
+      if (gt - kbase < vecs_k * NG) copy_k_f16<D>(p, gt - kbase);
       return;
     }
-    vec = gt < thr_per_tensor ? vecs_per_tensor + vec : 2 * vecs_per_tensor;  // V; the rest pads the warp
+    in_range = gt < thr_v;  // the rest pads the warp
+    which = 1;
+    r = in_range ? vec : 0;
+  } else {
+    in_range = vec < 2 * vecs_k;
+    which = in_range ? (int)(vec / vecs_k) : 0;  // 0 = K, 1 = V
+    r = in_range ? vec % vecs_k : 0;
   }
-  const bool in_range = vec < 2 * vecs_per_tensor;
-  const int which = in_range ? (int)(vec / vecs_per_tensor) : 0;  // 0 = K, 1 = V
-  const int64_t r = in_range ? vec % vecs_per_tensor : 0;
+  const int rows = which ? v_rows : p.n_new;
   const int h = (int)(r % p.n_kv);
   const int64_t bt = r / p.n_kv;
-  const int t = (int)(bt % p.n_new);
-  const int b = (int)(bt / p.n_new);
+  const int t = (int)(bt % rows);
+  const int b = (int)(bt / rows);
+  const int64_t in_row = ((int64_t)b * p.n_new + t) * p.n_kv + h;  // input vector of a new token
 
-  // the input rows and the start position are independent loads: issue both first
   float u[32];
   int64_t pos = 0;
-  if (in_range) {
-    load32(u, which ? p.v : p.k, r * D + part * 32, p.in_dtype);
-    pos = p.start_pos[b];
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = 0.f;
-  }
+  if (in_range) pos = p.start_pos[b];
   bool valid = in_range;
   if (in_range && (pos < 0 || pos + p.n_new > p.max_seq)) {
     valid = false;
     if (which == 0 && t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
+  }
+  int64_t dst = pos + t;     // position whose codes this item writes
+  int64_t tail_pos = -1;     // delegated: new token written to the hot tail after the encode
+  if (W == 0) {
+    if (in_range) {
+      load32(u, which ? p.v : p.k, in_row * D + part * 32, p.in_dtype);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = 0.f;
+    }
+  } else {
+    // Delegated cache (mlxcel guide, delegated cache variant): V grows from len0 to
+    // len1 tokens; positions below cold_tokens(len1) hold int4 codes, the rest the
+    // binary16 tail at slot pos % W. Each item encodes at most one vector, from the
+    // input (a new token that is cold at once) or from the tail (an old hot token
+    // that folds), and a new hot token then takes its slot. An old token whose slot a
+    // new hot token takes is folded by that token's item, before the overwrite.
+    const int64_t len0 = pos, len1 = pos + p.n_new;
+    const int64_t nc0 = cold_tokens(len0, W, p.fold_chunk), nc1 = cold_tokens(len1, W, p.fold_chunk);
+    int src = 0;  // 0 none, 1 input, 2 tail slot of dst
+    if (t < p.n_new) {
+      if (dst < nc1) {
+        src = 1;
+      } else {
+        tail_pos = dst;
+        const int64_t old = len0 - W + (dst - len0) % W;  // the old token in the same slot, if any
+        if (old >= nc0 && old >= 0) {
+          src = 2;
+          dst = old;
+        }
+      }
+    } else {
+      dst = nc0 + (t - p.n_new);
+      if (dst < min(nc1, len0)) {
+        const int64_t lo = max(len0, nc1);
+        const int64_t taker = lo + (((dst - lo) % W) + W) % W;  // first new hot token in this slot
+        if (taker >= len1) src = 2;
+      }
+    }
+    if (src == 0 || !valid) {
+      valid = false;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = 0.f;
+    } else if (src == 1) {
+      load32(u, p.v, in_row * D + part * 32, p.in_dtype);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = __half2float(__float2half_rn(u[i]));  // the tail's binary16 value
+    } else {
+      const uint4* hp = reinterpret_cast<const uint4*>(
+          p.v_tail + (((int64_t)b * W + dst % W) * p.n_kv + h) * D + part * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w4 = hp[j];
+        const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[k]));
+          u[8 * j + 2 * k] = f.x;
+          u[8 * j + 2 * k + 1] = f.y;
+        }
+      }
+    }
+    if (!(in_range && pos >= 0 && pos + p.n_new <= p.max_seq)) tail_pos = -1;
   }
   // sign diagonal, then the Walsh-Hadamard butterflies (strides 1, 2, ..., D/2 in
   // that order, packed pair operations that round each lane once as the scalar steps)
@@ -117,7 +206,10 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
     u[i + 1] = y.y;
     a = fmax_nan(a, fmax_nan(fabsf(y.x), fabsf(y.y)));
   }
-  if (!valid) return;
+  if (!valid) {
+    if (tail_pos >= 0) write_tail_f16<D>(p, in_row, b, h, part, tail_pos);
+    return;
+  }
 
   const float sigma32 = __fdiv_rn(a, 7.0f);
   const __half sig16 = __float2half_rn(sigma32);
@@ -163,11 +255,12 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
       }
     }
   }
-  const int64_t row = ((int64_t)b * p.max_seq + pos + t) * p.n_kv + h;
+  const int64_t row = ((int64_t)b * p.max_seq + dst) * p.n_kv + h;
   uint8_t* codes = which ? p.v_codes : p.k_codes;
   uint16_t* scales = which ? p.v_scales : p.k_scales;
   *reinterpret_cast<uint4*>(codes + row * (D / 2) + part * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   scales[row * NG + part] = sbits;
+  if (tail_pos >= 0) write_tail_f16<D>(p, in_row, b, h, part, tail_pos);
 }
 
 // Dequantise one group per thread: yhat = code * scale (exact in binary32);
@@ -222,7 +315,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const __grid_constant__
 template <int D>
 static cudaError_t launch_quantize_d(const QuantizeParams& p, cudaStream_t s) {
   const int64_t per_tensor = (int64_t)p.batch * p.n_new * p.n_kv * (D / 32);
-  const int64_t threads = p.k_f16 ? (per_tensor + 31) / 32 * 32 + per_tensor : 2 * per_tensor;
+  const int64_t per_v = (int64_t)p.batch * (p.n_new + p.tail_window) * p.n_kv * (D / 32);
+  const int64_t threads = p.k_f16 ? (per_v + 31) / 32 * 32 + per_tensor : 2 * per_tensor;
   const int64_t blocks = (threads + 255) / 256;
   // programmatic dependent launch: set-up overlaps the previous kernel's tail,
   // griddepcontrol.wait in the kernel orders the reads

@@ -98,6 +98,11 @@ def ragged_serving() -> Workload:
 
 GEMMA_SWEEP = (256, 512, 1024, 2048, 4096)
 
+# Hot-tail sizes for the delegated cache (the pages name the mode but give no
+# window): the most recent 256 V tokens stay binary16, folded 64 at a time.
+DELEGATED_WINDOW = 256
+DELEGATED_FOLD = 64
+
 
 def all_workloads() -> List[Workload]:
     return [tiny_single_head(), llama3_8b_layer(), *[gemma3_1b_sweep(t) for t in GEMMA_SWEEP],

@@ -24,11 +24,14 @@ TQ_STATUS_TIMEOUT = 4
 
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
-TQ_K_INT4, TQ_K_FP16 = 0, 1  # K storage format (V is always int4 codes + binary16 scales)
+# cache formats: int4 K + V; binary16 K + int4 V; binary16 K + V hot tail folded into int4
+TQ_K_INT4, TQ_K_FP16, TQ_KV_DELEGATED = 0, 1, 2
 
 # C symbols declared in include/tq.h
-EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_quantize_append", "tq_decode_attention", "tq_decode_attention_ex",
-           "tq_decode_attention_noalloc", "tq_dequantize_debug", "tq_status_string", "tq_last_cuda_error")
+EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_cache_layout_delegated", "tq_cold_length",
+           "tq_quantize_append", "tq_append_delegated", "tq_decode_attention", "tq_decode_attention_ex",
+           "tq_decode_attention_delegated", "tq_decode_attention_noalloc", "tq_dequantize_debug",
+           "tq_status_string", "tq_last_cuda_error")
 
 TQ_NOALLOC_WORKSPACE_BYTES = 8 << 20
 
@@ -45,6 +48,8 @@ class TqLayout(ctypes.Structure):
         ("decode_workspace_bytes", ctypes.c_uint64),
         ("max_ctas", ctypes.c_int32), ("k_format", ctypes.c_int32),
         ("k_bytes", ctypes.c_uint64), ("k_stride_tok", ctypes.c_int64), ("k_stride_seq", ctypes.c_int64),
+        ("tail_window", ctypes.c_int32), ("fold_chunk", ctypes.c_int32), ("tail_bytes", ctypes.c_uint64),
+        ("tail_stride_tok", ctypes.c_int64), ("tail_stride_seq", ctypes.c_int64),
     ]
 
 
@@ -77,8 +82,18 @@ def _lib():
         lib.tq_cache_layout.restype = I
         lib.tq_cache_layout_kv.argtypes = [I, I, I, I, I, I, U64, I, ctypes.POINTER(TqLayout)]
         lib.tq_cache_layout_kv.restype = I
+        lib.tq_cache_layout_delegated.argtypes = [I, I, I, I, I, I, U64, I, I, ctypes.POINTER(TqLayout)]
+        lib.tq_cache_layout_delegated.restype = I
+        lib.tq_cold_length.argtypes = [ctypes.POINTER(TqLayout), ctypes.c_int64]
+        lib.tq_cold_length.restype = ctypes.c_int64
         lib.tq_quantize_append.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
         lib.tq_quantize_append.restype = I
+        lib.tq_append_delegated.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
+        lib.tq_append_delegated.restype = I
+        lib.tq_decode_attention_delegated.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P,
+                                                      ctypes.c_float, P, P, ctypes.c_size_t, P,
+                                                      ctypes.POINTER(TqDecodeOpts), P]
+        lib.tq_decode_attention_delegated.restype = I
         lib.tq_decode_attention.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, ctypes.c_float, P, P,
                                             ctypes.c_size_t, P, P]
         lib.tq_decode_attention.restype = I
@@ -138,6 +153,22 @@ def tq_cache_layout_kv(batch, max_seq, n_kv_heads, n_q_heads, head_dim, k_format
     return out
 
 
+def tq_cache_layout_delegated(batch, max_seq, n_kv_heads, n_q_heads, head_dim, tail_window, fold_chunk,
+                              group_size=32, sign_seed=0) -> TqLayout:
+    """Delegated hot/cold cache: binary16 K; V in a binary16 tail of tail_window tokens, folded into int4
+    fold_chunk tokens at a time."""
+    out = TqLayout()
+    _check("tq_cache_layout_delegated", _lib().tq_cache_layout_delegated(
+        batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, ctypes.c_uint64(sign_seed), int(tail_window),
+        int(fold_chunk), ctypes.byref(out)))
+    return out
+
+
+def tq_cold_length(layout, length) -> int:
+    """Tokens of a sequence of `length` tokens held as int4 codes (all of them outside the delegated cache)."""
+    return int(_lib().tq_cold_length(ctypes.byref(layout), int(length)))
+
+
 def tq_cache_layout_status(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size=32, sign_seed=0):
     """Raw status code variant (for callers that test rejection paths)."""
     out = TqLayout()
@@ -155,6 +186,34 @@ def tq_quantize_append(layout, k, v, n_new, start_pos, k_codes, k_scales, v_code
                                      _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
                                      _ptr(v_scales), _ptr(status), _stream(stream))
     _check("tq_quantize_append", code)
+
+
+def tq_append_delegated(layout, k, v, n_new, start_pos, k_f16, v_codes, v_scales, v_tail, status=None,
+                        stream=None):
+    """Delegated-cache append. start_pos[b] must be sequence b's current length."""
+    for t in (k, v, start_pos, k_f16, v_codes, v_scales, v_tail):
+        assert t is None or t.is_contiguous()
+    code = _lib().tq_append_delegated(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
+                                      _ptr(start_pos), _ptr(k_f16), _ptr(v_codes), _ptr(v_scales), _ptr(v_tail),
+                                      _ptr(status), _stream(stream))
+    _check("tq_append_delegated", code)
+
+
+def tq_decode_attention_delegated(layout, q, seq_lens, k_f16, v_codes, v_scales, v_tail, sm_scale, out, workspace,
+                                  status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None):
+    """Decode over a delegated cache: the cold tokens through the split-K kernel, the hot tail in the merge."""
+    for t in (q, seq_lens, k_f16, v_codes, v_scales, v_tail, out, workspace):
+        assert t is None or t.is_contiguous()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    opts = None
+    if min_split_tokens or max_ctas or after_split_event is not None:
+        opts = TqDecodeOpts(int(min_split_tokens), int(max_ctas),
+                            ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None)
+    code = _lib().tq_decode_attention_delegated(
+        ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens), _ptr(k_f16), _ptr(v_codes), _ptr(v_scales),
+        _ptr(v_tail), ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes, _ptr(status),
+        ctypes.byref(opts) if opts is not None else None, _stream(stream))
+    _check("tq_decode_attention_delegated", code)
 
 
 def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out, workspace,
@@ -211,20 +270,26 @@ def sign_vector(layout):
 def alloc_cache(layout, device="cuda"):
     """Allocate (k_codes, k_scales, v_codes, v_scales) with the layout's sizes (zero-filled).
 
-    With layout.k_format == TQ_K_FP16, k_codes is the binary16 K buffer (k_bytes) and
-    k_scales is None.
+    With layout.k_format == TQ_K_FP16 or TQ_KV_DELEGATED, k_codes is the binary16 K buffer
+    (k_bytes) and k_scales is None; the delegated cache's V tail comes from alloc_tail.
     """
     import torch
     cb = int(layout.codes_bytes)
     sb = int(layout.scales_bytes)
     k_codes = torch.zeros(int(layout.k_bytes), dtype=torch.uint8, device=device)
     v_codes = torch.zeros(cb, dtype=torch.uint8, device=device)
-    if layout.k_format == TQ_K_FP16:
+    if layout.k_format != TQ_K_INT4:
         k_scales = None
     else:
         k_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
     v_scales = torch.zeros((sb + 1) // 2, dtype=torch.int16, device=device)
     return k_codes, k_scales, v_codes, v_scales
+
+
+def alloc_tail(layout, device="cuda"):
+    """The delegated cache's binary16 V tail [batch][tail_window][Hkv][D] as int16 bits (zero-filled)."""
+    import torch
+    return torch.zeros(int(layout.tail_bytes) // 2, dtype=torch.int16, device=device)
 
 
 def alloc_workspace(layout, device="cuda"):

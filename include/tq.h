@@ -20,6 +20,9 @@
  *  - the mlxcel guide, §"Cache modes": the recommended default mode keeps K in
  *    FP16 and compresses only V (K decides where attention looks, V is mixed
  *    after); that asymmetric cache is TQ_K_FP16 below.
+ *  - the mlxcel guide, §"Cache modes" (turbo4-delegated row) and §"Delegated
+ *    cache variant": K in FP16, the most recent V tokens kept in FP16 and older
+ *    ones stored in the 4-bit form; that cache is TQ_KV_DELEGATED below.
  *
  * Conventions fixed by this library where the pages are silent:
  *  - rotation: y = c_D * H * (s o x), H the Sylvester Hadamard matrix applied
@@ -37,6 +40,12 @@
  *  - with k_format TQ_K_FP16, K is instead one binary16 buffer
  *    [batch][max_seq][n_kv_heads][head_dim] (k_bytes) in the original domain and
  *    has no scales; V keeps its codes and scales.
+ *  - with k_format TQ_KV_DELEGATED, K is the binary16 buffer as above and V
+ *    has, besides its codes and scales, a binary16 hot tail
+ *    [batch][tail_window][n_kv_heads][head_dim] (tail_bytes): token t of a
+ *    sequence of len tokens is "cold" (int4 codes at position t) when
+ *    t < tq_cold_length(layout, len), else "hot" (binary16 in tail slot
+ *    t % tail_window).
  *    Allocate `scales_bytes` (slightly more than the array): decode reads
  *    scale rows in tile-sized blocks that may run past the last valid token.
  *  - every device buffer must be 16-byte aligned (cudaMalloc gives 256).
@@ -75,8 +84,9 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 
 /* How K is stored (V is always rotated int4 codes + binary16 group scales). */
 typedef enum {
-  TQ_K_INT4 = 0, /* K encoded like V (the symmetric cache) */
-  TQ_K_FP16 = 1  /* K as binary16 (round to nearest even) of the input, original domain */
+  TQ_K_INT4 = 0,      /* K encoded like V (the symmetric cache) */
+  TQ_K_FP16 = 1,      /* K as binary16 (round to nearest even) of the input, original domain */
+  TQ_KV_DELEGATED = 2 /* K as TQ_K_FP16; V as a binary16 hot tail folded into int4 codes (tq_cache_layout_delegated) */
 } tq_k_format;
 
 /* Filled by tq_cache_layout; plain data, caller-owned, never modified by the library. */
@@ -98,6 +108,11 @@ typedef struct {
   uint64_t k_bytes;            /* allocation size of the K buffer (codes_bytes for TQ_K_INT4) */
   int64_t k_stride_tok;        /* bytes between tokens of one sequence in the K buffer */
   int64_t k_stride_seq;        /* bytes between sequences in the K buffer */
+  int32_t tail_window;         /* TQ_KV_DELEGATED: hot V tokens kept in binary16 (W); 0 otherwise */
+  int32_t fold_chunk;          /* TQ_KV_DELEGATED: tokens folded into the int4 body at a time (F); 0 otherwise */
+  uint64_t tail_bytes;         /* allocation size of the hot tail (0 unless TQ_KV_DELEGATED) */
+  int64_t tail_stride_tok;     /* bytes between tail slots of one sequence = n_kv * D * 2 */
+  int64_t tail_stride_seq;     /* bytes between sequences in the tail     = W * n_kv * D * 2 */
 } tq_layout_t;
 
 /* Optional knobs for tq_decode_attention_ex (NULL = defaults). */
@@ -128,6 +143,24 @@ int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, in
                        int group_size, uint64_t sign_seed, int k_format, tq_layout_t* out);
 
 /*
+ * Delegated hot/cold cache (mlxcel guide, §"Cache modes", turbo4-delegated row,
+ * and §"Delegated cache variant"; the pages give no window sizes, so both are
+ * the caller's). K is stored as in TQ_K_FP16. V keeps the most recent tokens in
+ * binary16 in a ring of tail_window (W) slots per (sequence, kv head) and folds
+ * the oldest, fold_chunk (F) at a time, into the int4 body: a sequence of len
+ * tokens has tq_cold_length(len) = 0 for len <= W, else
+ * F * ceil((len - W) / F) cold tokens, so between W - F + 1 and W stay hot.
+ * 1 <= F <= W <= 1024; other arguments as tq_cache_layout_kv. Host only.
+ */
+int tq_cache_layout_delegated(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim,
+                              int group_size, uint64_t sign_seed, int tail_window, int fold_chunk,
+                              tq_layout_t* out);
+
+/* Cold (int4) tokens of a delegated-cache sequence of len tokens; len for other
+ * formats; -1 for a NULL layout or len < 0. Host only. */
+int64_t tq_cold_length(const tq_layout_t* layout, int64_t len);
+
+/*
  * Quantise and append n_new tokens to every sequence (Open-TQ-Metal abstract:
  * the fused sign-randomised transform + per-group abs-max + int4 nibble pack,
  * run when the cache is appended to).
@@ -141,6 +174,7 @@ int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, in
  *                and k_scales is not used (may be NULL).
  * n_new == 0 is a no-op. Codes and scales are bit-exact with the reference
  * definition (IEEE binary32 steps, no contraction, round-half-even).
+ * A TQ_KV_DELEGATED layout returns TQ_ERR_INVALID_ARG (use tq_append_delegated).
  */
 int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype,
                        int n_new, const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales,
@@ -173,7 +207,40 @@ int tq_decode_attention(const tq_layout_t* layout, const void* q, int q_dtype,
                         const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
                         void* workspace, size_t ws_bytes, int32_t* d_status, void* stream);
 
-/* tq_decode_attention with explicit options (opts may be NULL). */
+/*
+ * Append to a delegated cache (layout from tq_cache_layout_delegated). Every
+ * new K vector is stored as binary16. Each sequence's V grows from
+ * len0 = d_start_pos[b] to len1 = len0 + n_new tokens: tokens that end up
+ * hot are written to the tail as binary16; tokens below tq_cold_length(len1)
+ * are encoded (SRHT, per-group abs-max, int4) from their binary16 value -
+ * taken from the tail if they were hot before, from the input otherwise - so
+ * the cache does not depend on how the tokens were split into calls.
+ *   v_tail   device binary16 [batch][W][n_kv_heads][head_dim] (layout->tail_bytes)
+ * d_start_pos[b] must be the sequence's current length: the tail holds the
+ * tokens [tq_cold_length(len0), len0) only. Slots of folded tokens keep stale
+ * values. Other arguments, limits and status bits as tq_quantize_append.
+ */
+int tq_append_delegated(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                        const int32_t* d_start_pos, uint16_t* k_f16, uint8_t* v_codes, uint16_t* v_scales,
+                        uint16_t* v_tail, int32_t* d_status, void* stream);
+
+/*
+ * Decode over a delegated cache: the split-K kernel runs on the cold tokens
+ * [0, tq_cold_length(len_b)) exactly as for TQ_K_FP16; the merge kernel also
+ * attends to the hot tokens (binary16 K and V, fp32 arithmetic) and combines
+ * the two segments by their running max and sum before writing the output.
+ * Arguments as tq_decode_attention_ex, plus v_tail; the workspace is
+ * layout->decode_workspace_bytes as usual. head_dim <= 128.
+ */
+int tq_decode_attention_delegated(const tq_layout_t* layout, const void* q, int q_dtype,
+                                  const int32_t* d_seq_lens, const uint16_t* k_f16, const uint8_t* v_codes,
+                                  const uint16_t* v_scales, const uint16_t* v_tail, float sm_scale, float* out,
+                                  void* workspace, size_t ws_bytes, int32_t* d_status,
+                                  const tq_decode_opts_t* opts, void* stream);
+
+/* tq_decode_attention with explicit options (opts may be NULL). A
+ * TQ_KV_DELEGATED layout returns TQ_ERR_INVALID_ARG here and in
+ * tq_decode_attention / tq_decode_attention_noalloc. */
 int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype,
                            const int32_t* d_seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
                            const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,

@@ -98,6 +98,91 @@ class OracleCache:
         return out, st
 
 
+class DelegatedGpuCache:
+    """A delegated hot/cold cache in device memory (binary16 K, binary16 V tail + int4 V body)."""
+
+    def __init__(self, batch, max_seq, n_kv, n_q, D, window, fold, sign_seed=0, device="cuda"):
+        self.layout = tq.tq_cache_layout_delegated(batch, max_seq, n_kv, n_q, D, window, fold, 32, sign_seed)
+        self.k16, _, self.v_codes, self.v_scales = tq.alloc_cache(self.layout, device)
+        self.tail = tq.alloc_tail(self.layout, device)
+        self.device = device
+        self.window, self.fold = window, fold
+
+    def seq_view(self, b):
+        L = self.layout
+        l1 = tq.tq_cache_layout_delegated(1, L.max_seq, L.n_kv_heads, L.n_q_heads, L.head_dim, self.window,
+                                          self.fold, 32, L.sign_seed)
+        cs, ss, ks_ = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
+        ts = int(L.tail_stride_seq) // 2
+        return (l1, self.k16[b * ks_:(b + 1) * ks_], self.v_codes[b * cs:(b + 1) * cs], self.v_scales[b * ss:],
+                self.tail[b * ts:(b + 1) * ts])
+
+    def append_seq(self, b, k, v, start, status=None):
+        l1, kc, vc, vs, tl = self.seq_view(b)
+        sp = torch.tensor([start], dtype=torch.int32, device=self.device)
+        tq.tq_append_delegated(l1, k[None].contiguous(), v[None].contiguous(), k.shape[0], sp, kc, vc, vs, tl, status)
+
+    def append_all(self, k, v, start_pos, status=None):
+        sp = torch.tensor(start_pos, dtype=torch.int32, device=self.device)
+        tq.tq_append_delegated(self.layout, k.contiguous(), v.contiguous(), k.shape[1], sp, self.k16, self.v_codes,
+                               self.v_scales, self.tail, status)
+
+    def host_arrays(self):
+        """(k16 bits [B][S][H][D], v_codes, v_scales bits, tail bits [B][W][H][D]) as numpy."""
+        L = self.layout
+        B, S, H, D = L.batch, L.max_seq, L.n_kv_heads, L.head_dim
+        n_s = B * S * H * (D // 32)
+        k16 = self.k16.cpu().numpy().view(np.uint16).reshape(B, S, H, D)
+        vc = self.v_codes.cpu().numpy().reshape(B, S, H, D // 2)
+        vs = self.v_scales[:n_s].cpu().numpy().view(np.uint16).reshape(B, S, H, D // 32)
+        tail = self.tail.cpu().numpy().view(np.uint16).reshape(B, self.window, H, D)
+        return k16, vc, vs, tail
+
+    def decode(self, q, seq_lens, sm_scale, status=None, **opts):
+        L = self.layout
+        out = torch.full((L.batch, L.n_q_heads, L.head_dim), float("nan"), dtype=torch.float32, device=self.device)
+        ws = tq.alloc_workspace(L, self.device)
+        lens = torch.tensor(seq_lens, dtype=torch.int32, device=self.device)
+        tq.tq_decode_attention_delegated(L, q.contiguous(), lens, self.k16, self.v_codes, self.v_scales, self.tail,
+                                         sm_scale, out, ws, status, **opts)
+        return out
+
+
+class DelegatedOracleCache:
+    def __init__(self, batch, max_seq, n_kv, D, window, fold, sign_seed=0):
+        self.signs = oracle.sign_vector(sign_seed, D)
+        self.window, self.fold = window, fold
+        self.k16 = oracle.new_k16_cache(batch, max_seq, n_kv, D)
+        self.vc, self.vs = oracle.new_cache(batch, max_seq, n_kv, D)
+        self.tail = oracle.new_tail(batch, window, n_kv, D)
+
+    def append_seq(self, b, k, v, start):
+        st = oracle.append_delegated(self.signs, np_f32(k)[None], np_f32(v)[None], np.array([start], np.int32),
+                                     self.window, self.fold, self.k16[b:b + 1], self.vc[b:b + 1],
+                                     self.vs[b:b + 1], self.tail[b:b + 1])
+        assert st == 0
+
+    def decode(self, q, seq_lens, sm_scale, which=None):
+        return oracle.decode_attention_delegated(self.signs, np_f32(q), np.asarray(seq_lens, np.int32), self.k16,
+                                                 self.vc, self.vs, self.tail, self.window, self.fold, sm_scale,
+                                                 which)
+
+
+def assert_delegated_caches_equal(gpu, orc, seqs, lens):
+    """Bit-exact where the cache is defined: every K row, the int4 body below the cold length,
+    and the tail slots of the hot tokens (slots of folded tokens are unspecified)."""
+    k16, vc, vs, tail = gpu.host_arrays()
+    W, F = gpu.window, gpu.fold
+    for b in seqs:
+        n = lens[b]
+        nc = oracle.cold_length(n, W, F)
+        assert np.array_equal(k16[b, :n], orc.k16[b, :n]), f"binary16 K differs in sequence {b}"
+        assert np.array_equal(vc[b, :nc], orc.vc[b, :nc]), f"V codes differ in sequence {b}"
+        assert np.array_equal(vs[b, :nc], orc.vs[b, :nc]), f"V scales differ in sequence {b}"
+        live = [t % W for t in range(nc, n)]
+        assert np.array_equal(tail[b, live], orc.tail[b, live]), f"V tail differs in sequence {b}"
+
+
 def assert_close(got, ref, atol=ATOL, rtol_l2=RTOL_L2, what=""):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)

@@ -27,7 +27,7 @@ def lib():
 
 def header_functions():
     text = open(os.path.join(ROOT, "include", "tq.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(tq_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|const char\*)\s+(tq_\w+)\s*\(", text, re.M)))
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -176,3 +176,43 @@ def test_layout_kv_formats():
     with pytest.raises(tq.TqError) as exc:
         tq.tq_cache_layout_kv(3, 100, 8, 32, 128, 7)
     assert exc.value.code == tq.TQ_ERR_INVALID_ARG
+
+
+def test_layout_delegated_and_cold_length():
+    L = tq.tq_cache_layout_delegated(3, 100, 8, 32, 128, 16, 4)
+    assert L.k_format == tq.TQ_KV_DELEGATED and (L.tail_window, L.fold_chunk) == (16, 4)
+    assert L.k_bytes == 3 * 100 * 8 * 128 * 2
+    assert L.tail_stride_tok == 8 * 128 * 2 and L.tail_stride_seq == 16 * 8 * 128 * 2
+    assert L.tail_bytes == 3 * 16 * 8 * 128 * 2
+    L4 = tq.tq_cache_layout(3, 100, 8, 32, 128)
+    assert (L.codes_bytes, L.scales_bytes) == (L4.codes_bytes, L4.scales_bytes)
+    # the worked rule: 0 up to W, then F * ceil((len - W) / F)
+    assert [tq.tq_cold_length(L, n) for n in (0, 1, 16, 17, 20, 21, 24, 25, 100)] == [0, 0, 0, 4, 4, 8, 8, 12, 84]
+    assert tq.tq_cold_length(L4, 77) == 77
+    for bad in ((0, 1), (16, 0), (16, 17), (1025, 1), (-1, 1)):
+        with pytest.raises(tq.TqError) as exc:
+            tq.tq_cache_layout_delegated(3, 100, 8, 32, 128, *bad)
+        assert exc.value.code == tq.TQ_ERR_INVALID_ARG
+    with pytest.raises(tq.TqError) as exc:  # the window sizes come only through the delegated constructor
+        tq.tq_cache_layout_kv(3, 100, 8, 32, 128, tq.TQ_KV_DELEGATED)
+    assert exc.value.code == tq.TQ_ERR_INVALID_ARG
+
+
+def test_delegated_layout_rejected_by_the_other_entry_points():
+    # argument checks run before any device work, so these need no GPU
+    import ctypes
+    L = tq.tq_cache_layout_delegated(1, 64, 1, 4, 64, 8, 4)
+    lib = tq._lib()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the layout check fails first
+    assert lib.tq_quantize_append(ctypes.byref(L), fake, fake, 0, 1, fake, fake, None, fake, fake, None,
+                                  None) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_decode_attention(ctypes.byref(L), fake, 0, fake, fake, None, fake, fake, ctypes.c_float(0.1),
+                                   fake, fake, 1 << 30, None, None) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_decode_attention_noalloc(ctypes.byref(L), fake, 0, fake, fake, None, fake, fake,
+                                           ctypes.c_float(0.1), fake, None, None) == tq.TQ_ERR_INVALID_ARG
+    L16 = tq.tq_cache_layout_kv(1, 64, 1, 4, 64, tq.TQ_K_FP16)
+    assert lib.tq_append_delegated(ctypes.byref(L16), fake, fake, 0, 1, fake, fake, fake, fake, fake, None,
+                                   None) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_decode_attention_delegated(ctypes.byref(L16), fake, 0, fake, fake, fake, fake, fake,
+                                             ctypes.c_float(0.1), fake, fake, 1 << 30, None, None,
+                                             None) == tq.TQ_ERR_INVALID_ARG
