@@ -1099,18 +1099,28 @@ __global__ void __launch_bounds__(kTailThreads) decode_tail_kernel(const __grid_
     const int64_t rstride = (int64_t)p.n_kv * D;  // binary16 elements between tokens (K) or slots (V)
     const uint16_t* kg = p.k16 + (((int64_t)b * p.max_seq + t_lo) * p.n_kv + kvh) * D;
     const uint16_t* vg = p.v_tail + ((int64_t)b * W * p.n_kv + kvh) * D;
+    // a thread copies piece c of rows j0, j0 + RSTEP, ...; RSTEP is a multiple of 8
+    // (of 32 at D = 32), so the swizzled piece is the same in every row it copies
     const int c = tid % CPR;
     constexpr int RSTEP = kTailThreads / CPR;
-    int j = tid / CPR;
-    int slot_v = (t_lo + j) % W;
-    for (; j < kTailTokens; j += RSTEP) {
-      const int pc = tile_piece<D>(j, c);
+    static_assert(RSTEP % 8 == 0, "one swizzle phase per thread");
+    const int j0 = tid / CPR;
+    const int pc = tile_piece<D>(j0, c);
+    uint32_t ks_dst = smem_u32(&ks[j0 * D + pc * 8]);
+    uint32_t vs_dst = smem_u32(&vsm[j0 * D + pc * 8]);
+    const uint16_t* ksrc = kg + (int64_t)j0 * rstride + c * 8;
+    const uint16_t* vcol = vg + c * 8;
+    int slot_v = (t_lo + j0) % W;
+    for (int j = j0; j < kTailTokens; j += RSTEP) {
       if (j < n) {
-        cp_async16(smem_u32(&ks[j * D + pc * 8]), kg + (int64_t)j * rstride + c * 8);
-        cp_async16(smem_u32(&vsm[j * D + pc * 8]), vg + (int64_t)slot_v * rstride + c * 8);
+        cp_async16(ks_dst, ksrc);
+        cp_async16(vs_dst, vcol + (int64_t)slot_v * rstride);
       } else {
-        *reinterpret_cast<uint4*>(&vsm[j * D + pc * 8]) = make_uint4(0u, 0u, 0u, 0u);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs_dst), "r"(0u) : "memory");
       }
+      ks_dst += RSTEP * D * 2;
+      vs_dst += RSTEP * D * 2;
+      ksrc += RSTEP * rstride;
       slot_v += RSTEP;
       while (slot_v >= W) slot_v -= W;
     }
@@ -1122,18 +1132,45 @@ __global__ void __launch_bounds__(kTailThreads) decode_tail_kernel(const __grid_
   float f_h = 1.f;
   {
     float x[KS][4];
-    float mx = 0.f;
-    const bool has = gid < G;
-    const int64_t qoff = ((int64_t)b * p.n_q + (int64_t)kvh * G + gid) * D;
+    const int64_t qoff = ((int64_t)b * p.n_q + (int64_t)kvh * G + (gid < G ? gid : 0)) * D + 2 * tig;
+    // pairs (d, d + 1), d = 16 kk + 2 tig (+ 8): one 8- or 4-byte load each
+    if (p.q_dtype == TQ_F32) {
+      const float* qp = reinterpret_cast<const float*>(p.q) + qoff;
 #pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
+      for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 v = *reinterpret_cast<const float2*>(qp + 16 * kk + 8 * h);
+          x[kk][2 * h] = v.x;
+          x[kk][2 * h + 1] = v.y;
+        }
+    } else {
+      const uint16_t* qp = reinterpret_cast<const uint16_t*>(p.q) + qoff;
+      const bool bf = p.q_dtype == TQ_BF16;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(qp + 16 * kk + 8 * h);
+          if (bf) {
+            x[kk][2 * h] = __uint_as_float(w << 16);
+            x[kk][2 * h + 1] = __uint_as_float(w & 0xffff0000u);
+          } else {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+            x[kk][2 * h] = f.x;
+            x[kk][2 * h + 1] = f.y;
+          }
+        }
+    }
+    float mx = 0.f;
+    const float qsc = gid < G ? p.sm_scale_log2 : 0.f;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int d = 16 * kk + 8 * (e >> 1) + 2 * tig + (e & 1);
-        x[kk][e] = has ? load_scalar(p.q, qoff + d, p.q_dtype) * p.sm_scale_log2 : 0.f;
+        x[kk][e] *= qsc;
         mx = fmaxf(mx, fabsf(x[kk][e]));
       }
-    }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     int ex = 0;
