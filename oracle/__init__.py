@@ -48,6 +48,9 @@ def _signatures():
         "oracle_quantize_append_kf16": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P, P, P], i32),
         "oracle_decode_attention_kf16": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, f32, P, P], i32),
         "oracle_cold_length": ([i64, ctypes.c_int, ctypes.c_int], i64),
+        "oracle_encode_lambda": ([P, P, P, ctypes.c_int, i64, P, P], i32),
+        "oracle_quantize_append_lambda": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P, P, P, P, P, P], i32),
+        "oracle_decode_attention_ext": ([ctypes.c_int] * 5 + [P] * 10 + [f32, ctypes.c_double, P, P, P], i32),
         "oracle_append_delegated": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
                                                           P, P, P, P], i32),
         "oracle_decode_attention_delegated": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
@@ -248,6 +251,57 @@ def decode_attention_kf16(signs, q, seq_lens, k_f16, v_codes, v_scales, sm_scale
         _p(_c(v_codes, np.uint8)), _p(_c(v_scales, np.uint16)), ctypes.c_float(sm_scale),
         None if w is None else _p(w), _p(out))
     return out, int(st)
+
+
+def _opt(a, dtype):
+    return None if a is None else _c(a, dtype)
+
+
+def encode_lambda(x, signs, lam):
+    """SRHT, per-channel lambda (None = identity), quantise, pack -> (packed, scale bits, status)."""
+    x = _c(x, np.float32)
+    D = x.shape[-1]
+    lam = _opt(lam, np.float32)
+    packed = np.empty(x.shape[:-1] + (D // 2,), np.uint8)
+    scales = np.empty(x.shape[:-1] + (D // 32,), np.uint16)
+    st = _load().oracle_encode_lambda(_p(x), _p(_c(signs, np.float32)), None if lam is None else _p(lam), D,
+                                      x.size // D, _p(packed), _p(scales))
+    return packed, scales, int(st)
+
+
+def quantize_append_lambda(signs, k, v, start_pos, lambda_k, lambda_v, k_codes, k_scales, v_codes, v_scales) -> int:
+    """quantize_append with per-channel lambda vectors (None = identity). In place."""
+    k = _c(k, np.float32)
+    v = _c(v, np.float32)
+    B, n_new, n_kv, D = k.shape
+    max_seq = k_codes.shape[1]
+    lk, lv = _opt(lambda_k, np.float32), _opt(lambda_v, np.float32)
+    return int(_load().oracle_quantize_append_lambda(
+        B, max_seq, n_kv, D, _p(_c(signs, np.float32)), _p(k), _p(v), n_new, _p(_c(start_pos, np.int32)),
+        None if lk is None else _p(lk), None if lv is None else _p(lv), _p(k_codes), _p(k_scales), _p(v_codes),
+        _p(v_scales)))
+
+
+def decode_attention_ext(signs, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, lambda_k=None,
+                         lambda_v=None, tau=0.0, which=None, k_f16=None):
+    """Decode with lambda and the sparse-V threshold -> (out, bound, status); bound as in the C comments."""
+    q = _c(q, np.float32)
+    B, n_q, D = q.shape
+    max_seq, n_kv = v_codes.shape[1], v_codes.shape[2]
+    out = np.zeros((B, n_q, D), np.float32)
+    bound = np.zeros((B, n_q, D), np.float32)
+    w = None if which is None else _c(which, np.uint8)
+    lk, lv = _opt(lambda_k, np.float32), _opt(lambda_v, np.float32)
+    kc = None if k_codes is None else _c(k_codes, np.uint8)
+    ks = None if k_scales is None else _c(k_scales, np.uint16)
+    kf = None if k_f16 is None else _c(k_f16, np.uint16)
+    st = _load().oracle_decode_attention_ext(
+        B, max_seq, n_kv, n_q, D, _p(_c(signs, np.float32)), _p(q), _p(_c(seq_lens, np.int32)),
+        None if kc is None else _p(kc), None if ks is None else _p(ks), None if kf is None else _p(kf),
+        _p(_c(v_codes, np.uint8)), _p(_c(v_scales, np.uint16)), None if lk is None else _p(lk),
+        None if lv is None else _p(lv), ctypes.c_float(sm_scale), ctypes.c_double(tau),
+        None if w is None else _p(w), _p(out), _p(bound))
+    return out, bound, int(st)
 
 
 def cold_length(length: int, window: int, fold: int) -> int:

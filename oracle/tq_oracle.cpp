@@ -29,6 +29,11 @@
 //          V as an FP16 hot tail plus a Turbo4 cold body) and §"Delegated cache
 //          variant" (recent tokens stay FP16, older V tokens are stored in the
 //          4-bit form; the FP16 sidecars are folded into it).
+//  [OTQ-lam] the Open-TQ-Metal abstract's list of the fused kernel's steps:
+//          sign-randomised transform, per-channel lambda, per-group abs-max,
+//          int4 pack (lambda sits between the transform and the abs-max).
+//  [MLX-sparse] the mlxcel guide, §"Sparse-V dequant threshold": V dequant may
+//          be skipped where the attention weight is below a threshold (1e-6).
 //  [AMD]   "TurboQuant on AMD GPUs" (oracore.dev), §4: Walsh-Hadamard spreads
 //          energy evenly and suits kernels better than a dense random rotation.
 //
@@ -242,15 +247,25 @@ int64_t cold_length(int64_t len, int W, int F) {
 // nullptr: every V token is int4; otherwise tokens t >= cold_length(len_b)
 // take their binary16 tail value, mapped to the rotated domain by the forward
 // SRHT so that the weighted sum stays in one domain (the transform is linear).
+// Optional [OTQ-lam] lambda_k / lambda_v (nullptr = identity): the stored codes
+// encode lambda o y, so the rotated-domain value is (code * sigma) / lambda,
+// taken in binary64 here. Optional [MLX-sparse] threshold tau > 0: the V term
+// of token t is dropped when exp(z_t - max z) < tau (its weight relative to
+// the largest score); the softmax sum keeps every token. `bound` (nullable)
+// receives, per output element, sum over dropped t of w_t |V_t,i| in the
+// original domain (w_t the exact normalised weight), which bounds the change
+// any rule that drops a subset of those tokens can make.
 int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const float* s, const float* q,
                     const int32_t* seq_lens, const uint8_t* k_codes, const uint16_t* k_scales,
                     const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales,
-                    const uint16_t* v_tail, int W, int F, float sm_scale, const uint8_t* which, float* out) {
+                    const uint16_t* v_tail, int W, int F, float sm_scale, const uint8_t* which, float* out,
+                    const float* lambda_k = nullptr, const float* lambda_v = nullptr, double tau = 0.0,
+                    float* bound = nullptr) {
   int32_t st = 0;
   const int G = n_q / n_kv;
   const int64_t cb = D / 2, sb = D / 32;
-  std::vector<float> qr(D), yk(D), yv(D), xv(D), o32(D);
-  std::vector<double> z, acc(D);
+  std::vector<float> qr(D), yk(D), yv(D), xv(D), o32(D), xb(D);
+  std::vector<double> z, acc(D), bnd(D);
   for (int b = 0; b < batch; ++b) {
     const int len = seq_lens[b];
     const int64_t n_cold = v_tail ? cold_length(len, W, F) : len;
@@ -260,6 +275,8 @@ int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const floa
       if (len <= 0 || len > max_seq) {
         if (len > max_seq) st |= ORC_STATUS_CAPACITY;
         for (int i = 0; i < D; ++i) o[i] = 0.0f;
+        if (bound)
+          for (int i = 0; i < D; ++i) bound[((int64_t)b * n_q + hq) * D + i] = 0.0f;
         continue;
       }
       const int kv = hq / G;
@@ -278,7 +295,11 @@ int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const floa
           dequantize_rotated(k_codes + row * cb, k_scales + row * sb, D, yk.data());
         }
         double dot = 0.0;
-        for (int i = 0; i < D; ++i) dot += (double)qr[i] * (double)yk[i];
+        if (lambda_k && !k_f16) {
+          for (int i = 0; i < D; ++i) dot += (double)qr[i] * ((double)yk[i] / (double)lambda_k[i]);
+        } else {
+          for (int i = 0; i < D; ++i) dot += (double)qr[i] * (double)yk[i];
+        }
         z[t] = (double)sm_scale * dot;
       }
       double m = z[0];
@@ -290,8 +311,21 @@ int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const floa
         l += z[t];
       }
       for (int i = 0; i < D; ++i) acc[i] = 0.0;
+      for (int i = 0; i < D; ++i) bnd[i] = 0.0;
       for (int t = 0; t < len; ++t) {
         const int64_t row = ((int64_t)b * max_seq + t) * n_kv + kv;
+        // z[t] holds exp(z_t - max z) here: the weight relative to the largest score
+        const bool dropped = tau > 0.0 && t < n_cold && z[t] < tau;
+        if (dropped) {
+          if (bound) {  // the dropped token's V in the original domain
+            dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, xb.data());
+            if (lambda_v)
+              for (int i = 0; i < D; ++i) xb[i] = (float)((double)xb[i] / (double)lambda_v[i]);
+            srht_inverse_vec(xb.data(), s, D, xv.data());
+            for (int i = 0; i < D; ++i) bnd[i] += z[t] / l * std::fabs((double)xv[i]);
+          }
+          continue;
+        }
         if (t < n_cold) {
           dequantize_rotated(v_codes + row * cb, v_scales + row * sb, D, yv.data());
         } else {
@@ -300,10 +334,16 @@ int32_t decode_body(int batch, int max_seq, int n_kv, int n_q, int D, const floa
           srht_forward_vec(xv.data(), s, D, yv.data());
         }
         const double w = z[t] / l;
-        for (int i = 0; i < D; ++i) acc[i] += w * (double)yv[i];
+        if (lambda_v && t < n_cold) {
+          for (int i = 0; i < D; ++i) acc[i] += w * ((double)yv[i] / (double)lambda_v[i]);
+        } else {
+          for (int i = 0; i < D; ++i) acc[i] += w * (double)yv[i];
+        }
       }
       for (int i = 0; i < D; ++i) o32[i] = (float)acc[i];
       srht_inverse_vec(o32.data(), s, D, o);
+      if (bound)
+        for (int i = 0; i < D; ++i) bound[((int64_t)b * n_q + hq) * D + i] = (float)bnd[i];
     }
   }
   return st;
@@ -475,6 +515,62 @@ int32_t oracle_decode_attention_kf16(int batch, int max_seq, int n_kv, int n_q, 
                                      const uint8_t* which, float* out) {
   return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, nullptr, nullptr, k_f16, v_codes, v_scales,
                      nullptr, 0, 0, sm_scale, which, out);
+}
+
+// [OTQ-lam] encoding with a per-channel lambda: y = SRHT(x), then
+// y_i <- fl(y_i * lambda_i) (one binary32 multiply), then quantise and pack.
+// lambda == nullptr is the identity (oracle_encode).
+int32_t oracle_encode_lambda(const float* x, const float* s, const float* lambda, int D, int64_t n_vec,
+                             uint8_t* bytes, uint16_t* scales) {
+  std::vector<float> y(D);
+  std::vector<int8_t> codes(D);
+  int32_t st = 0;
+  for (int64_t v = 0; v < n_vec; ++v) {
+    srht_forward_vec(x + v * D, s, D, y.data());
+    if (lambda)
+      for (int i = 0; i < D; ++i) y[i] = y[i] * lambda[i];
+    st |= quantize_rotated(y.data(), D, codes.data(), scales + v * (D / 32));
+    pack_codes(codes.data(), D, bytes + v * (D / 2));
+  }
+  return st;
+}
+
+// oracle_quantize_append with per-channel lambda vectors for K and V (nullable).
+int32_t oracle_quantize_append_lambda(int batch, int max_seq, int n_kv, int D, const float* s, const float* k,
+                                      const float* v, int n_new, const int32_t* start_pos, const float* lambda_k,
+                                      const float* lambda_v, uint8_t* k_codes, uint16_t* k_scales,
+                                      uint8_t* v_codes, uint16_t* v_scales) {
+  int32_t st = 0;
+  const int64_t cb = D / 2, sb = D / 32;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t p0 = start_pos[b];
+    if (p0 < 0 || p0 + n_new > max_seq) {
+      st |= ORC_STATUS_CAPACITY;
+      continue;
+    }
+    for (int t = 0; t < n_new; ++t) {
+      for (int h = 0; h < n_kv; ++h) {
+        const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
+        const int64_t row = ((int64_t)b * max_seq + p0 + t) * n_kv + h;
+        st |= oracle_encode_lambda(k + src, s, lambda_k, D, 1, k_codes + row * cb, k_scales + row * sb);
+        st |= oracle_encode_lambda(v + src, s, lambda_v, D, 1, v_codes + row * cb, v_scales + row * sb);
+      }
+    }
+  }
+  return st;
+}
+
+// Decode with the optional extensions: lambda_k (int4 K only) and lambda_v
+// [OTQ-lam], the sparse-V threshold tau [MLX-sparse] and its error bound (see
+// decode_body). k_f16 != nullptr selects the asymmetric cache (k_codes and
+// k_scales unused).
+int32_t oracle_decode_attention_ext(int batch, int max_seq, int n_kv, int n_q, int D, const float* s,
+                                    const float* q, const int32_t* seq_lens, const uint8_t* k_codes,
+                                    const uint16_t* k_scales, const uint16_t* k_f16, const uint8_t* v_codes,
+                                    const uint16_t* v_scales, const float* lambda_k, const float* lambda_v,
+                                    float sm_scale, double tau, const uint8_t* which, float* out, float* bound) {
+  return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, k_codes, k_scales, k_f16, v_codes, v_scales,
+                     nullptr, 0, 0, sm_scale, which, out, lambda_k, lambda_v, tau, bound);
 }
 
 // Delegated hot/cold cache [MLX-deleg]: K as binary16 for every token (as in

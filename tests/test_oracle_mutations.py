@@ -182,3 +182,53 @@ def test_planted_delegated_mistake_is_caught(name, tmp_path, monkeypatch):
     lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
     monkeypatch.setattr(oracle, "_lib", lib)
     assert failing_delegated_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"
+
+
+EXT_MUTATIONS = {
+    "lambda_divides_instead": ("      for (int i = 0; i < D; ++i) y[i] = y[i] * lambda[i];",
+                               "      for (int i = 0; i < D; ++i) y[i] = y[i] / lambda[i];"),
+    "lambda_before_transform": ("    srht_forward_vec(x + v * D, s, D, y.data());\n    if (lambda)\n      for (int i = 0; i < D; ++i) y[i] = y[i] * lambda[i];",
+                                "    std::vector<float> xl(x + v * D, x + v * D + D);\n    if (lambda)\n      for (int i = 0; i < D; ++i) xl[i] = xl[i] * lambda[i];\n    srht_forward_vec(xl.data(), s, D, y.data());"),
+    "lambda_k_not_undone": ("dot += (double)qr[i] * ((double)yk[i] / (double)lambda_k[i]);",
+                            "dot += (double)qr[i] * (double)yk[i];"),
+    "lambda_v_not_undone": ("acc[i] += w * ((double)yv[i] / (double)lambda_v[i]);", "acc[i] += w * (double)yv[i];"),
+    "sparse_normalised_weight": ("const bool dropped = tau > 0.0 && t < n_cold && z[t] < tau;",
+                                 "const bool dropped = tau > 0.0 && t < n_cold && z[t] / l < tau;"),
+    "sparse_drops_the_sum_too": ("        z[t] = std::exp(z[t] - m);\n        l += z[t];",
+                                 "        z[t] = std::exp(z[t] - m);\n        l += (tau > 0.0 && z[t] < tau) ? 0.0 : z[t];"),
+}
+
+
+def ext_pins(orc):
+    yield lambda: pins.test_lambda_sits_between_the_transform_and_the_abs_max(orc)
+    yield lambda: pins.test_lambda_powers_of_two_per_group_keep_codes_and_shift_scales(orc)
+    yield lambda: pins.test_lambda_attention_equals_fp64(orc, 128, 8, 2, 40)
+    yield lambda: pins.test_sparse_v_zero_threshold_is_exact_and_the_drop_rule(orc)
+
+
+def failing_ext_pins(orc):
+    failed = 0
+    for check in ext_pins(orc):
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_ext_pins_pass_on_committed_oracle(orc):
+    assert failing_ext_pins(orc) == 0
+
+
+@pytest.mark.parametrize("name", sorted(EXT_MUTATIONS))
+def test_planted_lambda_or_sparse_mistake_is_caught(name, tmp_path, monkeypatch):
+    before, after = EXT_MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "tq_oracle_mut.cpp"
+    mutated.write_text(src.replace(before, after))
+    lib_path = tmp_path / f"libtq_oracle_{name}.so"
+    subprocess.run(["g++", *CXXFLAGS, "-o", str(lib_path), str(mutated)], check=True)
+    lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert failing_ext_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"

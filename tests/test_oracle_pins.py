@@ -701,3 +701,127 @@ def test_delegated_special_cases(orc):
     assert st & orc.STATUS_CAPACITY and np.all(out == 0)
     st = orc.append_delegated(s, k[:, :1], v[:, :1], np.array([6], np.int32), W, F, k16, vc, vs, tail)
     assert st & orc.STATUS_CAPACITY
+
+
+# ---------------------------------------------------------------- per-channel lambda and sparse-V
+# Open-TQ-Metal abstract (the fused kernel's step list: transform, per-channel
+# lambda, per-group abs-max, int4 pack); mlxcel guide §"Sparse-V dequant
+# threshold" (skip V dequant where the attention weight is below 1e-6).
+
+def test_lambda_sits_between_the_transform_and_the_abs_max(orc):
+    rng = np.random.default_rng(17)
+    D = 128
+    s = orc.sign_vector(0, D)
+    x = heavy_tailed(rng, 9, D)
+    lam = np.exp(rng.uniform(-1, 1, D)).astype(np.float32)
+    got_p, got_s, st = orc.encode_lambda(x, s, lam)
+    assert st == 0
+    # the definition restated: the pinned transform, one binary32 multiply per channel
+    # (numpy's IEEE float32 product), then the pinned quantiser and packing
+    y = orc.srht_forward(x, s) * lam
+    codes, scales, _ = orc.quantize_rotated(y)
+    assert np.array_equal(got_p, orc.pack(codes)) and np.array_equal(got_s, scales)
+    # lambda = None and lambda = 1 are the plain encoder
+    p0, s0, _ = orc.encode(x, s)
+    p1, s1, _ = orc.encode_lambda(x, s, None)
+    p2, s2, _ = orc.encode_lambda(x, s, np.ones(D, np.float32))
+    assert np.array_equal(p0, p1) and np.array_equal(p0, p2) and np.array_equal(s0, s1) and np.array_equal(s0, s2)
+
+
+def test_lambda_powers_of_two_per_group_keep_codes_and_shift_scales(orc):
+    rng = np.random.default_rng(18)
+    D = 128
+    s = orc.sign_vector(0, D)
+    x = rng.standard_normal((7, D)).astype(np.float32)
+    e = np.array([-3, 0, 2, 5])  # one exponent per group of 32
+    lam = np.repeat(np.exp2(e), 32).astype(np.float32)
+    p_l, s_l, _ = orc.encode_lambda(x, s, lam)
+    p_0, s_0, _ = orc.encode(x, s)
+    assert np.array_equal(p_l, p_0)  # y * 2^e and sigma * 2^e: the same quotients
+    want = (s_0.view(np.float16).astype(np.float64) * np.exp2(e)).astype(np.float16).view(np.uint16)
+    assert np.array_equal(s_l, want)
+
+
+def np_dequant_original_lambda(packed, scale_bits, signs, lam):
+    D = signs.shape[0]
+    y = np_dequant_rotated(packed, scale_bits, D)
+    if lam is not None:
+        y = y / lam.astype(np.float64)
+    return (y @ hadamard(D).T) / np.sqrt(D) * signs.astype(np.float64)
+
+
+def make_cache_lambda(orc, rng, B, T, Hkv, D, s, lk, lv):
+    k = np.stack([heavy_tailed(rng, T * Hkv, D).reshape(T, Hkv, D) for _ in range(B)])
+    v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    kc, ks = orc.new_cache(B, T, Hkv, D)
+    vc, vs = orc.new_cache(B, T, Hkv, D)
+    st = orc.quantize_append_lambda(s, k, v, np.zeros(B, np.int32), lk, lv, kc, ks, vc, vs)
+    assert st == 0
+    return kc, ks, vc, vs
+
+
+def brute_force_ext(q, lens, kc, ks, vc, vs, s, scale, lk=None, lv=None, tau=0.0):
+    """fp64 attention over the dequantised cache (lambda undone), dropping the V term of tokens
+    with exp(z - max z) < tau; also the bound sum_dropped w |V|."""
+    B, Hq, D = q.shape
+    Hkv = vc.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    bound = np.zeros((B, Hq, D))
+    for b in range(B):
+        L = lens[b]
+        if L == 0:
+            continue
+        for hq in range(Hq):
+            kv = hq // G
+            K = np_dequant_original_lambda(kc[b, :L, kv], ks[b, :L, kv], s, lk)
+            V = np_dequant_original_lambda(vc[b, :L, kv], vs[b, :L, kv], s, lv)
+            z = K @ q[b, hq].astype(np.float64) * scale
+            r = np.exp(z - z.max())
+            w = r / r.sum()
+            keep = ~(r < tau) if tau > 0 else np.ones(L, bool)
+            out[b, hq] = w[keep] @ V[keep]
+            bound[b, hq] = w[~keep] @ np.abs(V[~keep]) if (~keep).any() else 0.0
+    return out, bound
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,T", [(128, 8, 2, 40), (64, 4, 1, 33), (32, 2, 2, 17)])
+def test_lambda_attention_equals_fp64(orc, D, Hq, Hkv, T):
+    rng = np.random.default_rng(D + Hq + T)
+    s = orc.sign_vector(3, D)
+    lk = np.exp(rng.uniform(-1, 1, D)).astype(np.float32)
+    lv = np.exp(rng.uniform(-1, 1, D)).astype(np.float32)
+    kc, ks, vc, vs = make_cache_lambda(orc, rng, 2, T, Hkv, D, s, lk, lv)
+    q = rng.standard_normal((2, Hq, D)).astype(np.float32)
+    lens = np.array([T, T // 2], np.int32)
+    got, bound, st = orc.decode_attention_ext(s, q, lens, kc, ks, vc, vs, 0.2, lk, lv)
+    assert st == 0 and np.all(bound == 0)
+    ref, _ = brute_force_ext(q, lens, kc, ks, vc, vs, s, 0.2, lk, lv)
+    assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_sparse_v_zero_threshold_is_exact_and_the_drop_rule(orc):
+    rng = np.random.default_rng(21)
+    D, Hq, Hkv, T, B = 128, 8, 2, 300, 2
+    s = orc.sign_vector(0, D)
+    kc, ks, vc, vs = make_cache_lambda(orc, rng, B, T, Hkv, D, s, None, None)
+    q = (4.0 * rng.standard_normal((B, Hq, D))).astype(np.float32)  # peaked weights
+    lens = np.array([T, 200], np.int32)
+    exact, _ = orc.decode_attention(s, q, lens, kc, ks, vc, vs, 0.3)
+    got0, b0, _ = orc.decode_attention_ext(s, q, lens, kc, ks, vc, vs, 0.3, tau=0.0)
+    assert np.array_equal(got0, exact) and np.all(b0 == 0)
+    for tau in (1e-6, 1e-3, 0.5):
+        got, bound, st = orc.decode_attention_ext(s, q, lens, kc, ks, vc, vs, 0.3, tau=tau)
+        ref, rb = brute_force_ext(q, lens, kc, ks, vc, vs, s, 0.3, tau=tau)
+        assert st == 0
+        assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+        assert np.max(np.abs(bound - rb)) < 2e-5 * max(1.0, rb.max())  # binary32 inverse transform per token
+        # the bound covers the change from exact attention
+        assert np.all(np.abs(got.astype(np.float64) - exact) <= bound + 1e-5)
+    assert rb.max() > 0  # tau = 0.5 drops tokens here
+    # near-uniform weights: each normalised weight is about 1/T, each relative weight about 1,
+    # so a threshold between the two separates "relative to the largest score" from "normalised"
+    qd = (0.05 * rng.standard_normal((B, Hq, D))).astype(np.float32)
+    got, bound, _ = orc.decode_attention_ext(s, qd, lens, kc, ks, vc, vs, 0.3, tau=0.01)
+    ref, rb = brute_force_ext(qd, lens, kc, ks, vc, vs, s, 0.3, tau=0.01)
+    assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
