@@ -50,6 +50,10 @@ def parse_args(argv=None):
                     help="cache format: int4 K and V (symmetric cache); binary16 K in the original domain with "
                          "int4 V (the asymmetric cache of the mlxcel guide's recommended mode); or 'delegated', "
                          "binary16 K with a binary16 V hot tail folded into int4 V (the guide's delegated mode)")
+    ap.add_argument("--lambda", dest="lam", action="store_true",
+                    help="write and read the cache with seeded per-channel lambda vectors (K with int4 K, and V)")
+    ap.add_argument("--sparse-v", type=float, default=0.0, metavar="TAU",
+                    help="sparse-V threshold of the decode (0 = exact attention; the mlxcel guide's default is 1e-6)")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report instead of the step benchmark: decode and prefill-quantise "
                          "times (median, p10, p90; cold L2, and warm L2 where the cache fits) for every workload "
@@ -71,6 +75,15 @@ FORMATS = ("int4", "fp16", "delegated")
 def delegated_window():
     from compressed_domain_attention_b200 import synthetic as syn
     return syn.DELEGATED_WINDOW, syn.DELEGATED_FOLD
+
+
+def bench_lambdas(D, fmt, device):
+    """Seeded per-channel lambda vectors exp(U(-1, 1)) for K (int4 K only) and V."""
+    import torch
+    g = torch.Generator("cpu").manual_seed(1234)
+    lk = torch.exp(torch.rand(D, generator=g) * 2 - 1).float()
+    lv = torch.exp(torch.rand(D, generator=g) * 2 - 1).float()
+    return (lk.to(device) if fmt == "int4" else None), lv.to(device)
 
 
 def cold_count(n, fmt):
@@ -278,13 +291,18 @@ class OracleStep:
     re-appends the new token at position len_b and decodes over len_b + 1.
     """
 
-    def __init__(self, w, tensors, seqs, fmt="int4"):
+    def __init__(self, w, tensors, seqs, fmt="int4", lam=False, tau=0.0):
         import numpy as np
         import oracle
         from compressed_domain_attention_b200 import synthetic as syn
         self.oracle, self.np = oracle, np
         D, H = w.head_dim, w.n_kv_heads
-        self.w, self.seqs, self.fmt = w, seqs, fmt
+        self.w, self.seqs, self.fmt, self.tau = w, seqs, fmt, tau
+        self.lk = self.lv = None
+        if lam:
+            lk, lv = bench_lambdas(D, fmt, "cpu")
+            self.lk = None if lk is None else lk.numpy()
+            self.lv = lv.numpy()
         self.s = oracle.sign_vector(0, D)
         n = len(seqs)
         cap = max(w.seq_lens[b] for b in seqs) + 1
@@ -313,7 +331,20 @@ class OracleStep:
             self.oracle.append_delegated(self.s, k, v, start, self.W, self.F, self.kc[sl], self.vc[sl], self.vs[sl],
                                          self.tail[sl])
         elif self.fmt == "fp16":
-            self.oracle.quantize_append_kf16(self.s, k, v, start, self.kc[sl], self.vc[sl], self.vs[sl])
+            if self.lv is not None:  # binary16 K as numpy rounds it, V through the lambda encoder
+                np_ = self.np
+                n = k.shape[1]
+                for j, b in enumerate(range(i0, i1)):
+                    p0 = int(start[j])
+                    self.kc[b, p0:p0 + n] = k[j].astype(np_.float16).view(np_.uint16)
+                kd, ksd = self.oracle.new_cache(i1 - i0, self.vc.shape[1], self.vc.shape[2], self.w.head_dim)
+                self.oracle.quantize_append_lambda(self.s, k, v, start, None, self.lv, kd, ksd, self.vc[sl],
+                                                   self.vs[sl])
+            else:
+                self.oracle.quantize_append_kf16(self.s, k, v, start, self.kc[sl], self.vc[sl], self.vs[sl])
+        elif self.lk is not None or self.lv is not None:
+            self.oracle.quantize_append_lambda(self.s, k, v, start, self.lk, self.lv, self.kc[sl], self.ks[sl],
+                                               self.vc[sl], self.vs[sl])
         else:
             self.oracle.quantize_append(self.s, k, v, start, self.kc[sl], self.ks[sl], self.vc[sl], self.vs[sl])
 
@@ -322,6 +353,11 @@ class OracleStep:
         if self.fmt == "delegated":
             self.oracle.decode_attention_delegated(self.s, q, lens, self.kc[sl], self.vc[sl], self.vs[sl],
                                                    self.tail[sl], self.W, self.F, self.w.scale)
+        elif self.lk is not None or self.lv is not None or self.tau > 0:
+            kf = self.fmt == "fp16"
+            self.oracle.decode_attention_ext(self.s, q, lens, None if kf else self.kc[sl],
+                                             None if kf else self.ks[sl], self.vc[sl], self.vs[sl], self.w.scale,
+                                             self.lk, self.lv, self.tau, k_f16=self.kc[sl] if kf else None)
         elif self.fmt == "fp16":
             self.oracle.decode_attention_kf16(self.s, q, lens, self.kc[sl], self.vc[sl], self.vs[sl], self.w.scale)
         else:
@@ -362,9 +398,9 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, tensors, target_tokens, fmt="int4"):
+def cpu_baseline(w, tensors, target_tokens, fmt="int4", lam=False, tau=0.0):
     seqs = oracle_sample(w, target_tokens)
-    o = OracleStep(w, tensors, seqs, fmt)
+    o = OracleStep(w, tensors, seqs, fmt, lam, tau)
     dt = o.run()
     line = {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
@@ -491,9 +527,10 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, fmt="
 class DeviceCache:
     """One cache format in device memory, driven through the library's C ABI (tq.py)."""
 
-    def __init__(self, w, cap, fmt, dev):
+    def __init__(self, w, cap, fmt, dev, lam=False, tau=0.0):
         from compressed_domain_attention_b200 import tq
-        self.tq, self.fmt = tq, fmt
+        self.tq, self.fmt, self.tau = tq, fmt, tau
+        self.lk, self.lv = bench_lambdas(w.head_dim, fmt, dev) if lam else (None, None)
         shape = (cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
         if fmt == "delegated":
             W, F = delegated_window()
@@ -522,21 +559,24 @@ class DeviceCache:
                                    stream)
         else:
             tq.tq_quantize_append(self.l1, k, v, n, zero, kc, None if self.ks is None else self.ks[b * ss:], vc, vs,
-                                  status, stream)
+                                  status, stream, lambda_k=self.lk, lambda_v=self.lv)
 
     def append(self, k, v, n, start, status, stream):
         if self.fmt == "delegated":
             self.tq.tq_append_delegated(self.L, k, v, n, start, self.kc, self.vc, self.vs, self.tail, status, stream)
         else:
-            self.tq.tq_quantize_append(self.L, k, v, n, start, self.kc, self.ks, self.vc, self.vs, status, stream)
+            self.tq.tq_quantize_append(self.L, k, v, n, start, self.kc, self.ks, self.vc, self.vs, status, stream,
+                                       lambda_k=self.lk, lambda_v=self.lv)
 
     def decode(self, q, lens, scale, out, status, stream, after_split_event=None):
         if self.fmt == "delegated":
             self.tq.tq_decode_attention_delegated(self.L, q, lens, self.kc, self.vc, self.vs, self.tail, scale, out,
-                                                  self.wsp, status, stream, after_split_event=after_split_event)
+                                                  self.wsp, status, stream, after_split_event=after_split_event,
+                                                  sparse_v_threshold=self.tau)
         else:
             self.tq.tq_decode_attention(self.L, q, lens, self.kc, self.ks, self.vc, self.vs, scale, out, self.wsp,
-                                        status, stream, after_split_event=after_split_event)
+                                        status, stream, after_split_event=after_split_event, lambda_k=self.lk,
+                                        lambda_v=self.lv, sparse_v_threshold=self.tau)
 
 
 # ----------------------------------------------------------------------------- per-configuration sweep
@@ -672,7 +712,8 @@ def run_reference(args):
         w.n_append = 1
     seqs = oracle_sample(w, 8192)
     t = syn.generate(w, device="cpu", seq_subset=seqs)
-    o = OracleStep(w, t, seqs, getattr(args, "k_format", "int4"))
+    o = OracleStep(w, t, seqs, getattr(args, "k_format", "int4"), getattr(args, "lam", False),
+                   getattr(args, "sparse_v", 0.0))
     for _ in range(args.warmup):
         o.run()
     tot_t = sum(o.run() for _ in range(args.steps))
@@ -683,7 +724,9 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode / f64 attention",
             "data": "synthetic (seeded)", "config": {"workload": w.name, "global_batch": w.batch,
-                                                     "k_format": getattr(args, "k_format", "int4")},
+                                                     "k_format": getattr(args, "k_format", "int4"),
+                                                     "lambda": bool(getattr(args, "lam", False)),
+                                                     "sparse_v_threshold": getattr(args, "sparse_v", 0.0)},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -706,7 +749,9 @@ def run_tq(args):
     cap = max(w.seq_lens) + w.n_append
     t = syn.generate(w, device="cuda")
     fmt = args.k_format
-    cache = DeviceCache(w, cap, fmt, dev)
+    if args.lam and fmt == "delegated":
+        raise SystemExit("--lambda applies to the int4 and fp16 formats (the delegated tail is binary16)")
+    cache = DeviceCache(w, cap, fmt, dev, args.lam, args.sparse_v)
     L = cache.L
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
@@ -900,13 +945,13 @@ def run_tq(args):
     cfg = {"workload": w.name, "global_batch": w.batch * ws, "kv_tokens_per_seq_step": lens_step if w.batch <= 4
            else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-           "k_format": args.k_format,
+           "k_format": args.k_format, "lambda": bool(args.lam), "sparse_v_threshold": args.sparse_v,
            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
            "l2": f"inputs larger than L2 (cache {cache_bytes / 1e9:.2f} GB per replica > 126 MB), no flush",
            "algorithmic_bytes_per_step": bytes_step}
     total_bytes = sum_over_ranks(bytes_step * args.steps, dev)  # every rank takes part
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        extra["cpu_baseline"] = cpu_baseline(w, t, 300000, fmt)
+        extra["cpu_baseline"] = cpu_baseline(w, t, 300000, fmt, args.lam, args.sparse_v)
     if rank == 0:
         line = assemble_line(n_gpus=ws, steps=args.steps, warmup=args.warmup, total_bytes_all_ranks=total_bytes,
                              max_time_s=max_t, workload=cfg, extra=extra)

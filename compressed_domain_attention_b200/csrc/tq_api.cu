@@ -249,7 +249,14 @@ namespace {
 
 int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
                 const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
-                uint16_t* v_scales, uint16_t* v_tail, int32_t* d_status, void* stream) {
+                uint16_t* v_scales, uint16_t* v_tail, const tq_append_opts_t* opts, int32_t* d_status,
+                void* stream) {
+  const float* lam_k = opts ? opts->lambda_k : nullptr;
+  const float* lam_v = opts ? opts->lambda_v : nullptr;
+  // lambda scales quantised vectors: not binary16 K, not the delegated cache's tail
+  if (lam_k && layout->k_format != TQ_K_INT4) return TQ_ERR_INVALID_ARG;
+  if ((lam_k || lam_v) && layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  if ((lam_k && !aligned16(lam_k)) || (lam_v && !aligned16(lam_v))) return TQ_ERR_INVALID_ARG;
   if (n_new < 0) return TQ_ERR_INVALID_ARG;
   if (n_new > layout->max_seq) return TQ_ERR_CAPACITY;
   if (in_dtype != TQ_F32 && in_dtype != TQ_BF16 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
@@ -283,6 +290,8 @@ int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_
   p.v_tail = v_tail;
   p.tail_window = layout->tail_window;
   p.fold_chunk = layout->fold_chunk;
+  p.lambda_k = lam_k;
+  p.lambda_v = lam_v;
   cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
@@ -296,7 +305,17 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
   if (r != TQ_OK) return r;
   if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
   return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
-                     d_status, stream);
+                     nullptr, d_status, stream);
+}
+
+int tq_quantize_append_ex(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                          const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
+                          uint16_t* v_scales, const tq_append_opts_t* opts, int32_t* d_status, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
+                     opts, d_status, stream);
 }
 
 int tq_append_delegated(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
@@ -306,7 +325,7 @@ int tq_append_delegated(const tq_layout_t* layout, const void* k, const void* v,
   if (r != TQ_OK) return r;
   if (layout->k_format != TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
   return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, reinterpret_cast<uint8_t*>(k_f16), nullptr,
-                     v_codes, v_scales, v_tail, d_status, stream);
+                     v_codes, v_scales, v_tail, nullptr, d_status, stream);
 }
 
 namespace {
@@ -338,13 +357,25 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
   int grid = sms;
   int min_split = 128;
   cudaEvent_t ev = nullptr;
+  const float* lam_k = nullptr;
+  const float* lam_v = nullptr;
+  float sparse_lt = -INFINITY;
   if (opts != nullptr) {
     if (opts->max_ctas < 0 || opts->max_ctas > layout->max_ctas || opts->min_split_tokens < 0)
       return TQ_ERR_INVALID_ARG;
     if (opts->max_ctas > 0) grid = opts->max_ctas;
     if (opts->min_split_tokens > 0) min_split = opts->min_split_tokens;
     ev = reinterpret_cast<cudaEvent_t>(opts->after_split_event);
+    lam_k = opts->lambda_k;
+    lam_v = opts->lambda_v;
+    if (lam_k && kf16) return TQ_ERR_INVALID_ARG;             // binary16 K carries no lambda
+    if ((lam_k || lam_v) && deleg) return TQ_ERR_INVALID_ARG;  // nor does the binary16 tail
+    if ((lam_k && !aligned16(lam_k)) || (lam_v && !aligned16(lam_v))) return TQ_ERR_INVALID_ARG;
+    const float tau = opts->sparse_v_threshold;
+    if (!(tau >= 0.f) || !std::isfinite(tau)) return TQ_ERR_INVALID_ARG;
+    if (tau > 0.f) sparse_lt = std::log2(tau);
   }
+  if (sparse_lt > -INFINITY && D != 64 && D != 128) return TQ_ERR_UNSUPPORTED;  // sparse-V kernels: D 64, 128
   if (grid > layout->max_ctas) grid = layout->max_ctas;
   const int W = deleg ? layout->tail_window : 0;
   if (ws_bytes < workspace_bytes(layout->batch, Hq, D, grid, W)) return TQ_ERR_INVALID_ARG;
@@ -387,6 +418,9 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
   p.fold_chunk = layout->fold_chunk;
   p.tail_chunks = tqk::tail_chunk_count(W);
   p.tail_slot0 = grid + layout->batch;
+  p.lambda_k = lam_k;
+  p.lambda_v = lam_v;
+  p.sparse_lt = sparse_lt;
   cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }

@@ -216,7 +216,7 @@ struct TileWalker {
 // the query's binary16 hi/lo pieces of 4 heads in the 8 N columns, which halves
 // their count; otherwise the 8 heads' hi (rows 0-7) and lo (rows 8-15) pieces
 // are the M rows and the tokens the N columns.
-template <int D, int HKV, bool TOK_M, bool KF16>
+template <int D, int HKV, bool TOK_M, bool KF16, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap) {
@@ -452,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool dead = false;
   int tile_i = 0;
 
+  constexpr bool sparse = SPARSE;  // sparse-V threshold set (a separate instantiation)
   while (!walk.done()) {
     const int b = walk.b;
     const int seg_hi = walk.seg_hi;
@@ -476,6 +477,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) u[i] = flip_sign(u[i], sw, i);
           fwht_group_x2<NG>(u, part);
+          if (p.lambda_k != nullptr) {  // the cache holds lambda o y: q pairs with y / lambda
+            const float4* l4 = reinterpret_cast<const float4*>(p.lambda_k + part * 32);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 lv = __ldg(l4 + i / 4);
+              u[i] = __fdividef(u[i], lv.x);  // a few ulp: far inside the decode tolerance
+              u[i + 1] = __fdividef(u[i + 1], lv.y);
+              u[i + 2] = __fdividef(u[i + 2], lv.z);
+              u[i + 3] = __fdividef(u[i + 3], lv.w);
+            }
+          }
         }
         float mx = 0.f;
 #pragma unroll
@@ -627,6 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // P^T fragments for P.V, per 16-token k-step: tokens (2 tig, 2 tig + 1) and
           // (2 tig + 8, 2 tig + 9) of head gid
           float2 pb[KSP][2];
+          bool pv_live = true;  // cleared by the sparse-V rule when no weight of the unit is kept
+          (void)pv_live;
           if constexpr (TOK_M) {
             // --- scores S[token 16 mt + gid + 8 e][head tig], per group g. A = K codes (rows:
             //     tokens gid, gid + 8 of the m-tile), B = q pieces (columns 2j, 2j + 1: hi, lo
@@ -739,8 +753,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
               const float2 z = __ffma2_rn(s2[mt], make_float2(f_h, f_h), make_float2(-mb, -mb));
-              const float2 pp = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+              float2 pp = make_float2(ex2_approx(z.x), ex2_approx(z.y));
               lsum = __fadd2_rn(lsum, pp);
+              if constexpr (sparse) {  // the V term only: the sum above keeps the token
+                if (z.x < p.sparse_lt) pp.x = 0.f;
+                if (z.y < p.sparse_lt) pp.y = 0.f;
+              }
               const float x0 = __shfl_sync(0xffffffffu, pp.x, src0 & 31);
               const float x1 = __shfl_sync(0xffffffffu, pp.x, src1 & 31);
               const float y0 = __shfl_sync(0xffffffffu, pp.y, src0 & 31);
@@ -749,6 +767,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               pb[mt][1] = head_ok ? make_float2(y0, y1) : make_float2(0.f, 0.f);
             }
             l_run += lsum.x + lsum.y;
+            if constexpr (sparse) {
+              bool nz = false;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt)
+                nz = nz || pb[mt][0].x != 0.f || pb[mt][0].y != 0.f || pb[mt][1].x != 0.f || pb[mt][1].y != 0.f;
+              pv_live = __any_sync(0xffffffffu, nz);
+            }
           } else {
             // --- scores S[head gid][token nt*8 + 2*tig + e], per group g
             float2 s2[NT], s2b[NT];  // even and odd groups: two independent chains
@@ -864,8 +889,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 z = __ffma2_rn(s2[nt], make_float2(f_h, f_h), make_float2(-mb, -mb));
               p2[nt] = make_float2(ex2_approx(z.x), ex2_approx(z.y));
               lsum = __fadd2_rn(lsum, p2[nt]);
+              if constexpr (sparse) {  // the V term only: the sum above keeps the token
+                if (z.x < p.sparse_lt) p2[nt].x = 0.f;
+                if (z.y < p.sparse_lt) p2[nt].y = 0.f;
+              }
             }
             l_run += lsum.x + lsum.y;
+            if constexpr (sparse) {
+              bool nz = false;
+  #pragma unroll
+              for (int nt = 0; nt < NT; ++nt) nz = nz || p2[nt].x != 0.f || p2[nt].y != 0.f;
+              pv_live = __any_sync(0xffffffffu, nz);
+            }
   #pragma unroll
             for (int ks = 0; ks < KSP; ++ks) {
               pb[ks][0] = p2[2 * ks];
@@ -884,6 +919,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const __half2 k128 = __ushort_as_half2_pair(0x0080u);
 #pragma unroll
           for (int g4 = 0; g4 < NG * NT; g4 += 4) {
+            if constexpr (sparse) {
+              if (!pv_live) break;  // sparse-V: every weight of this unit fell below the threshold
+            }
             uint32_t vw[4];
             ldmatrix_x4_trans(vw, vc + r0 * RB + v_off[g4 / 4]);
 #pragma unroll
@@ -1479,7 +1517,9 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
     float sum = 0.f;
 #pragma unroll
     for (int q = 0; q < PH; ++q) sum += accs[q][d];
-    lsv[d] = sum * inv_l;  // lsv[] is free again: reused for the normalised vector
+    float o = sum * inv_l;
+    if (p.lambda_v != nullptr) o = __fdividef(o, __ldg(p.lambda_v + d));  // the V codes hold lambda o y
+    lsv[d] = o;  // lsv[] is free again: reused for the normalised vector
   }
   __syncthreads();
   if (tid < 32) {
@@ -1495,15 +1535,15 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   }
 }
 
-template <int D, int HKV, bool TOK_M, bool KF16>
+template <int D, int HKV, bool TOK_M, bool KF16, bool SPARSE>
 static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
                                     cudaStream_t s, cudaEvent_t ev) {
   using C = DecodeCfg<D, HKV, KF16>;
   const int smem = C::OFF_PREFIX + 8 * (p.batch + 1) + 8 * 16;
   static bool attr_set = false;  // per instantiation; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV, TOK_M, KF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_MAX);
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, HKV, TOK_M, KF16, SPARSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_MAX);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -1519,7 +1559,7 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   kattr[0].val.programmaticStreamSerializationAllowed = 1;
   kcfg.attrs = kattr;
   kcfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M, KF16>, p, kmap, vmap);
+  cudaError_t e = cudaLaunchKernelEx(&kcfg, decode_split_kernel<D, HKV, TOK_M, KF16, SPARSE>, p, kmap, vmap);
   if (e != cudaSuccess) return e;
   const bool few = (int64_t)p.batch * p.n_q < 2 * (int64_t)p.grid;  // merge blocks vs SMs
   if (ev != nullptr) {  // timing split: plain stream order between the kernels
@@ -1561,19 +1601,31 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, kMergeThreads>, p);
 }
 
-template <int D, int HKV>
-static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
-                                    cudaStream_t s, cudaEvent_t ev) {
+template <int D, int HKV, bool SPARSE>
+static cudaError_t launch_decode_dhs(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
+                                     cudaStream_t s, cudaEvent_t ev) {
   if constexpr (D <= 128) {
     if (p.k_f16) {
-      if (p.group <= 4) return launch_decode_dht<D, HKV, true, true>(p, km, vm, s, ev);
-      return launch_decode_dht<D, HKV, false, true>(p, km, vm, s, ev);
+      if (p.group <= 4) return launch_decode_dht<D, HKV, true, true, SPARSE>(p, km, vm, s, ev);
+      return launch_decode_dht<D, HKV, false, true, SPARSE>(p, km, vm, s, ev);
     }
   } else {
     if (p.k_f16) return cudaErrorInvalidValue;  // binary16 K tiles: head_dim <= 128
   }
-  if (p.group <= 4) return launch_decode_dht<D, HKV, true, false>(p, km, vm, s, ev);
-  return launch_decode_dht<D, HKV, false, false>(p, km, vm, s, ev);
+  if (p.group <= 4) return launch_decode_dht<D, HKV, true, false, SPARSE>(p, km, vm, s, ev);
+  return launch_decode_dht<D, HKV, false, false, SPARSE>(p, km, vm, s, ev);
+}
+
+// The sparse-V rule is a separate instantiation of the split-K kernel (head dims
+// 64 and 128), so that the exact kernel carries none of its instructions.
+template <int D, int HKV>
+static cudaError_t launch_decode_dh(const DecodeParams& p, const TensorMap128& km, const TensorMap128& vm,
+                                    cudaStream_t s, cudaEvent_t ev) {
+  if (p.sparse_lt > -INFINITY) {
+    if constexpr (D == 64 || D == 128) return launch_decode_dhs<D, HKV, true>(p, km, vm, s, ev);
+    return cudaErrorNotSupported;
+  }
+  return launch_decode_dhs<D, HKV, false>(p, km, vm, s, ev);
 }
 
 template <int D>

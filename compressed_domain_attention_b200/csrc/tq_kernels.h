@@ -23,6 +23,8 @@ struct QuantizeParams {
   // delegated cache (tail_window > 0, with k_f16): binary16 V hot tail [batch][W][n_kv][D]
   uint16_t* v_tail;
   int tail_window, fold_chunk;
+  const float* lambda_k;  // per-channel lambda in the rotated domain (nullable)
+  const float* lambda_v;
 };
 
 struct DequantParams {
@@ -65,6 +67,9 @@ struct DecodeParams {
   int tail_window, fold_chunk;
   int tail_chunks;  // hot-tail partials per sequence (ceil(tail_window / 64)); 0 without a tail
   int tail_slot0;   // workspace slot of sequence 0's first hot-tail partial (after the split-K slots)
+  const float* lambda_k;  // per-channel lambda of the cache (nullable): q is divided by lambda_k,
+  const float* lambda_v;  // the merged V sum by lambda_v, both in the rotated domain
+  float sparse_lt;        // log2 of the sparse-V threshold; -inf = off
 };
 
 // Hot-tail partials per sequence of the delegated cache (64 tokens each).

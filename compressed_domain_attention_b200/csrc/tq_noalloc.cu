@@ -94,7 +94,7 @@ extern "C" int tq_decode_attention_noalloc(const tq_layout_t* layout, const void
   int err = 0;
   void* ws = ws_address_for_current_device(&err);
   if (ws == nullptr) return TQ_ERR_CUDA;
-  tq_decode_opts_t opts;
+  tq_decode_opts_t opts = {};
   opts.min_split_tokens = 0;
   opts.max_ctas = sms;
   opts.after_split_event = nullptr;

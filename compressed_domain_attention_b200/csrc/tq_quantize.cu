@@ -199,12 +199,31 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
   fwht_group_x2<NG>(u, part);
 
   float a = 0.f;
+  // per-channel lambda (Open-TQ-Metal abstract: between the transform and the
+  // abs-max): one more binary32 multiply per element
+  const float* lam = which ? p.lambda_v : p.lambda_k;
+  if (lam != nullptr) {
+    const float4* l4 = reinterpret_cast<const float4*>(lam + part * 32);
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float2 y = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(p.c_d));
-    u[i] = y.x;
-    u[i + 1] = y.y;
-    a = fmax_nan(a, fmax_nan(fabsf(y.x), fabsf(y.y)));
+    for (int i = 0; i < 32; i += 4) {
+      const float4 lv = __ldg(l4 + i / 4);
+      const float2 y0 = __fmul2_rn(__fmul2_rn(make_float2(u[i], u[i + 1]), f2(p.c_d)), make_float2(lv.x, lv.y));
+      const float2 y1 =
+          __fmul2_rn(__fmul2_rn(make_float2(u[i + 2], u[i + 3]), f2(p.c_d)), make_float2(lv.z, lv.w));
+      u[i] = y0.x;
+      u[i + 1] = y0.y;
+      u[i + 2] = y1.x;
+      u[i + 3] = y1.y;
+      a = fmax_nan(a, fmax_nan(fmax_nan(fabsf(y0.x), fabsf(y0.y)), fmax_nan(fabsf(y1.x), fabsf(y1.y))));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 y = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(p.c_d));
+      u[i] = y.x;
+      u[i + 1] = y.y;
+      a = fmax_nan(a, fmax_nan(fabsf(y.x), fabsf(y.y)));
+    }
   }
   if (!valid) {
     if (tail_pos >= 0) write_tail_f16<D>(p, in_row, b, h, part, tail_pos);

@@ -29,7 +29,7 @@ TQ_K_INT4, TQ_K_FP16, TQ_KV_DELEGATED = 0, 1, 2
 
 # C symbols declared in include/tq.h
 EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_cache_layout_delegated", "tq_cold_length",
-           "tq_quantize_append", "tq_append_delegated", "tq_decode_attention", "tq_decode_attention_ex",
+           "tq_quantize_append", "tq_quantize_append_ex", "tq_append_delegated", "tq_decode_attention", "tq_decode_attention_ex",
            "tq_decode_attention_delegated", "tq_decode_attention_noalloc", "tq_dequantize_debug",
            "tq_status_string", "tq_last_cuda_error")
 
@@ -55,7 +55,12 @@ class TqLayout(ctypes.Structure):
 
 class TqDecodeOpts(ctypes.Structure):
     _fields_ = [("min_split_tokens", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("after_split_event", ctypes.c_void_p)]
+                ("after_split_event", ctypes.c_void_p), ("lambda_k", ctypes.c_void_p),
+                ("lambda_v", ctypes.c_void_p), ("sparse_v_threshold", ctypes.c_float)]
+
+
+class TqAppendOpts(ctypes.Structure):
+    _fields_ = [("lambda_k", ctypes.c_void_p), ("lambda_v", ctypes.c_void_p)]
 
 
 class TqError(RuntimeError):
@@ -88,6 +93,9 @@ def _lib():
         lib.tq_cold_length.restype = ctypes.c_int64
         lib.tq_quantize_append.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
         lib.tq_quantize_append.restype = I
+        lib.tq_quantize_append_ex.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P,
+                                              ctypes.POINTER(TqAppendOpts), P, P]
+        lib.tq_quantize_append_ex.restype = I
         lib.tq_append_delegated.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
         lib.tq_append_delegated.restype = I
         lib.tq_decode_attention_delegated.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P,
@@ -178,14 +186,24 @@ def tq_cache_layout_status(batch, max_seq, n_kv_heads, n_q_heads, head_dim, grou
 
 
 def tq_quantize_append(layout, k, v, n_new, start_pos, k_codes, k_scales, v_codes, v_scales, status=None,
-                       stream=None):
-    """k, v: [batch][n_new][Hkv][D] (f32/bf16/f16, CUDA, contiguous); start_pos: int32 [batch] on the device."""
-    for t in (k, v, start_pos, k_codes, k_scales, v_codes, v_scales):
+                       stream=None, lambda_k=None, lambda_v=None):
+    """k, v: [batch][n_new][Hkv][D] (f32/bf16/f16, CUDA, contiguous); start_pos: int32 [batch] on the device.
+
+    lambda_k / lambda_v: optional float32 [D] device vectors (per-channel lambda, tq_quantize_append_ex).
+    """
+    for t in (k, v, start_pos, k_codes, k_scales, v_codes, v_scales, lambda_k, lambda_v):
         assert t is None or t.is_contiguous()
-    code = _lib().tq_quantize_append(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
-                                     _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
-                                     _ptr(v_scales), _ptr(status), _stream(stream))
-    _check("tq_quantize_append", code)
+    if lambda_k is None and lambda_v is None:
+        code = _lib().tq_quantize_append(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
+                                         _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                         _ptr(v_scales), _ptr(status), _stream(stream))
+        _check("tq_quantize_append", code)
+        return
+    opts = TqAppendOpts(_ptr(lambda_k), _ptr(lambda_v))
+    code = _lib().tq_quantize_append_ex(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
+                                        _ptr(start_pos), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                        _ptr(v_scales), ctypes.byref(opts), _ptr(status), _stream(stream))
+    _check("tq_quantize_append_ex", code)
 
 
 def tq_append_delegated(layout, k, v, n_new, start_pos, k_f16, v_codes, v_scales, v_tail, status=None,
@@ -199,16 +217,27 @@ def tq_append_delegated(layout, k, v, n_new, start_pos, k_f16, v_codes, v_scales
     _check("tq_append_delegated", code)
 
 
+def _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k=None, lambda_v=None,
+                 sparse_v_threshold=0.0):
+    """TqDecodeOpts for the given knobs, or None when all are at their defaults."""
+    if not (min_split_tokens or max_ctas or after_split_event is not None or lambda_k is not None
+            or lambda_v is not None or sparse_v_threshold):
+        return None
+    for t in (lambda_k, lambda_v):
+        assert t is None or t.is_contiguous()
+    ev = ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None
+    return TqDecodeOpts(int(min_split_tokens), int(max_ctas), ev, _ptr(lambda_k), _ptr(lambda_v),
+                        float(sparse_v_threshold))
+
+
 def tq_decode_attention_delegated(layout, q, seq_lens, k_f16, v_codes, v_scales, v_tail, sm_scale, out, workspace,
-                                  status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None):
+                                  status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None,
+                                  sparse_v_threshold=0.0):
     """Decode over a delegated cache: the cold tokens through the split-K kernel, the hot tail in the merge."""
     for t in (q, seq_lens, k_f16, v_codes, v_scales, v_tail, out, workspace):
         assert t is None or t.is_contiguous()
     ws_bytes = workspace.numel() * workspace.element_size()
-    opts = None
-    if min_split_tokens or max_ctas or after_split_event is not None:
-        opts = TqDecodeOpts(int(min_split_tokens), int(max_ctas),
-                            ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None)
+    opts = _decode_opts(min_split_tokens, max_ctas, after_split_event, sparse_v_threshold=sparse_v_threshold)
     code = _lib().tq_decode_attention_delegated(
         ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens), _ptr(k_f16), _ptr(v_codes), _ptr(v_scales),
         _ptr(v_tail), ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes, _ptr(status),
@@ -217,15 +246,19 @@ def tq_decode_attention_delegated(layout, q, seq_lens, k_f16, v_codes, v_scales,
 
 
 def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out, workspace,
-                        status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None):
-    """q: [batch][Hq][D]; out: float32 [batch][Hq][D]; workspace: >= layout.decode_workspace_bytes bytes."""
+                        status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None,
+                        lambda_k=None, lambda_v=None, sparse_v_threshold=0.0):
+    """q: [batch][Hq][D]; out: float32 [batch][Hq][D]; workspace: >= layout.decode_workspace_bytes bytes.
+
+    lambda_k / lambda_v: the per-channel lambda the cache was written with; sparse_v_threshold: the
+    sparse-V rule's threshold (0 = exact). Any of these selects tq_decode_attention_ex.
+    """
     for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out, workspace):
         assert t is None or t.is_contiguous()
     ws_bytes = workspace.numel() * workspace.element_size()
     lib = _lib()
-    if min_split_tokens or max_ctas or after_split_event is not None:
-        opts = TqDecodeOpts(int(min_split_tokens), int(max_ctas),
-                            ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None)
+    opts = _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k, lambda_v, sparse_v_threshold)
+    if opts is not None:
         code = lib.tq_decode_attention_ex(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
                                           _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
                                           ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace), ws_bytes,

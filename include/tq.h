@@ -115,12 +115,38 @@ typedef struct {
   int64_t tail_stride_seq;     /* bytes between sequences in the tail     = W * n_kv * D * 2 */
 } tq_layout_t;
 
-/* Optional knobs for tq_decode_attention_ex (NULL = defaults). */
+/* Optional knobs for tq_decode_attention_ex / _delegated (NULL = defaults; zero-fill unused fields). */
 typedef struct {
   int32_t min_split_tokens; /* 0 = default; otherwise the smallest token range one CTA takes */
   int32_t max_ctas;         /* 0 = default (one per SM); otherwise the split-K grid, <= layout.max_ctas */
   void* after_split_event;  /* a cudaEvent_t recorded on `stream` between the split-K and merge kernels, or NULL */
+  /* Per-channel lambda the cache was written with (tq_append_opts_t), device
+   * float32 [head_dim], 16-byte aligned, positive and finite; NULL = identity.
+   * lambda_k only with int4 K; neither with the delegated cache. */
+  const float* lambda_k;
+  const float* lambda_v;
+  /* Sparse-V threshold (mlxcel guide, §"Sparse-V dequant threshold"; the guide's
+   * default is 1e-6): 0 = off (exact attention). Otherwise the V term of an int4
+   * V token is dropped when its softmax weight relative to the running maximum
+   * of its split range is below the threshold; the softmax sum keeps every
+   * token. A dropped token's normalised weight is then below the threshold too,
+   * so the output moves by at most sum over dropped t of w_t |V_t|. A unit of
+   * 16-32 tokens whose weights all fall below skips its V decode and MMAs.
+   * Head dims 64 and 128 (otherwise TQ_ERR_UNSUPPORTED). */
+  float sparse_v_threshold;
 } tq_decode_opts_t;
+
+/* Optional knobs for tq_quantize_append_ex (NULL = defaults). */
+typedef struct {
+  /* Per-channel lambda (Open-TQ-Metal abstract: the fused quantiser's steps are
+   * the transform, a per-channel lambda, the per-group abs-max and the pack):
+   * the rotated vector y is multiplied by lambda (one binary32 multiply per
+   * element) before the abs-max. Device float32 [head_dim], 16-byte aligned,
+   * positive and finite (not checked on the device); NULL = identity. lambda_k
+   * only with int4 K. The decode must be given the same vectors. */
+  const float* lambda_k;
+  const float* lambda_v;
+} tq_append_opts_t;
 
 /*
  * Validate a cache shape and fill *out. Host only: no device work, no CUDA
@@ -179,6 +205,11 @@ int64_t tq_cold_length(const tq_layout_t* layout, int64_t len);
 int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, int in_dtype,
                        int n_new, const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales,
                        uint8_t* v_codes, uint16_t* v_scales, int32_t* d_status, void* stream);
+
+/* tq_quantize_append with options (opts may be NULL). */
+int tq_quantize_append_ex(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                          const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
+                          uint16_t* v_scales, const tq_append_opts_t* opts, int32_t* d_status, void* stream);
 
 /*
  * One decode query per sequence over its packed cache (Open-TQ-Metal arXiv
