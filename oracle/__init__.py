@@ -49,6 +49,10 @@ def _signatures():
         "oracle_decode_attention_kf16": ([ctypes.c_int] * 5 + [P, P, P, P, P, P, f32, P, P], i32),
         "oracle_cold_length": ([i64, ctypes.c_int, ctypes.c_int], i64),
         "oracle_encode_lambda": ([P, P, P, ctypes.c_int, i64, P, P], i32),
+        "oracle_quantize_append_paged": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P] + [ctypes.c_int] * 3
+                                         + [P] * 5, i32),
+        "oracle_decode_attention_paged": ([ctypes.c_int] * 5 + [P, P, P, P] + [ctypes.c_int] * 3 + [P] * 5
+                                          + [f32, P, P], i32),
         "oracle_quantize_append_lambda": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, P, P, P, P, P, P], i32),
         "oracle_decode_attention_ext": ([ctypes.c_int] * 5 + [P] * 10 + [f32, ctypes.c_double, P, P, P], i32),
         "oracle_append_delegated": ([ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int,
@@ -302,6 +306,50 @@ def decode_attention_ext(signs, q, seq_lens, k_codes, k_scales, v_codes, v_scale
         None if lv is None else _p(lv), ctypes.c_float(sm_scale), ctypes.c_double(tau),
         None if w is None else _p(w), _p(out), _p(bound))
     return out, bound, int(st)
+
+
+def new_pool(n_pages, P, n_kv, D, k_f16=False):
+    """Zeroed paged pools: (K codes or binary16 K, K scales or None, V codes, V scales), rows n_pages * P."""
+    rows = n_pages * P
+    if k_f16:
+        kc, ks = np.zeros((rows, n_kv, D), np.uint16), None
+    else:
+        kc, ks = np.zeros((rows, n_kv, D // 2), np.uint8), np.zeros((rows, n_kv, D // 32), np.uint16)
+    return kc, ks, np.zeros((rows, n_kv, D // 2), np.uint8), np.zeros((rows, n_kv, D // 32), np.uint16)
+
+
+def quantize_append_paged(signs, k, v, start_pos, table, P, max_seq, pools) -> int:
+    """Append k, v [B][n_new][Hkv][D] through the block table table [B][max_pages] into pools (in place)."""
+    k = _c(k, np.float32)
+    v = _c(v, np.float32)
+    B, n_new, n_kv, D = k.shape
+    kc, ks, vc, vs = pools
+    kf16 = kc.dtype == np.uint16
+    n_pages = vc.shape[0] // P
+    table = _c(table, np.int32)
+    return int(_load().oracle_quantize_append_paged(
+        B, max_seq, n_kv, D, _p(_c(signs, np.float32)), _p(k), _p(v), n_new, _p(_c(start_pos, np.int32)),
+        _p(table), P, table.shape[1], n_pages, None if kf16 else _p(kc), None if kf16 else _p(ks),
+        _p(kc) if kf16 else None, _p(vc), _p(vs)))
+
+
+def decode_attention_paged(signs, q, seq_lens, table, P, max_seq, pools, sm_scale, which=None):
+    """Decode over paged pools -> (out [B][Hq][D] float32, status)."""
+    q = _c(q, np.float32)
+    B, n_q, D = q.shape
+    kc, ks, vc, vs = pools
+    kf16 = kc.dtype == np.uint16
+    n_kv = vc.shape[1]
+    n_pages = vc.shape[0] // P
+    table = _c(table, np.int32)
+    out = np.zeros((B, n_q, D), np.float32)
+    w = None if which is None else _c(which, np.uint8)
+    st = _load().oracle_decode_attention_paged(
+        B, max_seq, n_kv, n_q, D, _p(_c(signs, np.float32)), _p(q), _p(_c(seq_lens, np.int32)), _p(table), P,
+        table.shape[1], n_pages, None if kf16 else _p(_c(kc, np.uint8)), None if kf16 else _p(_c(ks, np.uint16)),
+        _p(_c(kc, np.uint16)) if kf16 else None, _p(_c(vc, np.uint8)), _p(_c(vs, np.uint16)),
+        ctypes.c_float(sm_scale), None if w is None else _p(w), _p(out))
+    return out, int(st)
 
 
 def cold_length(length: int, window: int, fold: int) -> int:

@@ -34,6 +34,8 @@
 //          int4 pack (lambda sits between the transform and the abs-max).
 //  [MLX-sparse] the mlxcel guide, §"Sparse-V dequant threshold": V dequant may
 //          be skipped where the attention weight is below a threshold (1e-6).
+//  [MLX-paged] the same guide, §"Known limitations / paged KV scheduler": a
+//          paged decode storage backend (it cites PagedAttention).
 //  [AMD]   "TurboQuant on AMD GPUs" (oracore.dev), §4: Walsh-Hadamard spreads
 //          energy evenly and suits kernels better than a dense random rotation.
 //
@@ -571,6 +573,91 @@ int32_t oracle_decode_attention_ext(int batch, int max_seq, int n_kv, int n_q, i
                                     float sm_scale, double tau, const uint8_t* which, float* out, float* bound) {
   return decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, k_codes, k_scales, k_f16, v_codes, v_scales,
                      nullptr, 0, 0, sm_scale, which, out, lambda_k, lambda_v, tau, bound);
+}
+
+// ---- paged storage [MLX-paged] ----
+// Reading taken: a paged cache holds the same rows as the contiguous one, placed
+// in a pool of n_pages pages of P tokens; token t of sequence b sits at pool row
+// table[b * max_pages + t / P] * P + t % P. Rows are [n_kv][...] as before. An
+// entry outside [0, n_pages) is an unmapped page: appends to it are skipped and
+// raise ORC_STATUS_CAPACITY. k_f16 != nullptr selects binary16 K (k_codes and
+// k_scales unused), as in the asymmetric cache.
+int32_t oracle_quantize_append_paged(int batch, int max_seq, int n_kv, int D, const float* s, const float* k,
+                                     const float* v, int n_new, const int32_t* start_pos, const int32_t* table,
+                                     int P, int max_pages, int n_pages, uint8_t* k_codes, uint16_t* k_scales,
+                                     uint16_t* k_f16, uint8_t* v_codes, uint16_t* v_scales) {
+  int32_t st = 0;
+  const int64_t cb = D / 2, sb = D / 32;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t p0 = start_pos[b];
+    if (p0 < 0 || p0 + n_new > max_seq) {
+      st |= ORC_STATUS_CAPACITY;
+      continue;
+    }
+    for (int t = 0; t < n_new; ++t) {
+      const int64_t pos = p0 + t;
+      const int pg = table[(int64_t)b * max_pages + pos / P];
+      if (pg < 0 || pg >= n_pages) {
+        st |= ORC_STATUS_CAPACITY;
+        continue;
+      }
+      const int64_t prow = (int64_t)pg * P + pos % P;
+      for (int h = 0; h < n_kv; ++h) {
+        const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
+        const int64_t row = prow * n_kv + h;
+        if (k_f16) {
+          for (int i = 0; i < D; ++i) {
+            const uint16_t hbits = f32_to_f16_rne(k[src + i]);
+            if ((hbits & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
+            k_f16[row * D + i] = hbits;
+          }
+        } else {
+          st |= oracle_encode(k + src, s, D, 1, k_codes + row * cb, k_scales + row * sb);
+        }
+        st |= oracle_encode(v + src, s, D, 1, v_codes + row * cb, v_scales + row * sb);
+      }
+    }
+  }
+  return st;
+}
+
+// Decode over a paged cache: each sequence's rows are gathered through the
+// table into the contiguous layout, then the contiguous decode runs unchanged.
+int32_t oracle_decode_attention_paged(int batch, int max_seq, int n_kv, int n_q, int D, const float* s,
+                                      const float* q, const int32_t* seq_lens, const int32_t* table, int P,
+                                      int max_pages, int n_pages, const uint8_t* k_codes, const uint16_t* k_scales,
+                                      const uint16_t* k_f16, const uint8_t* v_codes, const uint16_t* v_scales,
+                                      float sm_scale, const uint8_t* which, float* out) {
+  const int64_t cb = D / 2, sb = D / 32, rows = (int64_t)batch * max_seq * n_kv;
+  std::vector<uint8_t> kc(k_f16 ? 0 : rows * cb), vc(rows * cb);
+  std::vector<uint16_t> ks(k_f16 ? 0 : rows * sb), kf(k_f16 ? rows * D : 0), vs(rows * sb);
+  int32_t st = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int len = seq_lens[b];
+    for (int64_t t = 0; t < len && t < max_seq; ++t) {
+      const int pg = table[(int64_t)b * max_pages + t / P];
+      if (pg < 0 || pg >= n_pages) {
+        st |= ORC_STATUS_CAPACITY;
+        continue;  // its rows stay zero
+      }
+      for (int h = 0; h < n_kv; ++h) {
+        const int64_t src = ((int64_t)pg * P + t % P) * n_kv + h;
+        const int64_t dst = ((int64_t)b * max_seq + t) * n_kv + h;
+        std::memcpy(&vc[dst * cb], v_codes + src * cb, cb);
+        std::memcpy(&vs[dst * sb], v_scales + src * sb, sb * 2);
+        if (k_f16) {
+          std::memcpy(&kf[dst * D], k_f16 + src * D, D * 2);
+        } else {
+          std::memcpy(&kc[dst * cb], k_codes + src * cb, cb);
+          std::memcpy(&ks[dst * sb], k_scales + src * sb, sb * 2);
+        }
+      }
+    }
+  }
+  st |= decode_body(batch, max_seq, n_kv, n_q, D, s, q, seq_lens, k_f16 ? nullptr : kc.data(),
+                    k_f16 ? nullptr : ks.data(), k_f16 ? kf.data() : nullptr, vc.data(), vs.data(), nullptr, 0, 0,
+                    sm_scale, which, out);
+  return st;
 }
 
 // Delegated hot/cold cache [MLX-deleg]: K as binary16 for every token (as in

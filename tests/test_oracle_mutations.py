@@ -232,3 +232,43 @@ def test_planted_lambda_or_sparse_mistake_is_caught(name, tmp_path, monkeypatch)
     lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
     monkeypatch.setattr(oracle, "_lib", lib)
     assert failing_ext_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"
+
+
+PAGED_MUTATIONS = {
+    "paged_append_row_shifted": ("const int64_t prow = (int64_t)pg * P + pos % P;",
+                                 "const int64_t prow = (int64_t)pg * P + (pos + 1) % P;"),
+    "paged_gather_row_shifted": ("const int64_t src = ((int64_t)pg * P + t % P) * n_kv + h;",
+                                 "const int64_t src = ((int64_t)pg * P + (t + 1) % P) * n_kv + h;"),
+    "paged_page_index_off_by_one": ("const int pg = table[(int64_t)b * max_pages + pos / P];",
+                                    "const int pg = table[(int64_t)b * max_pages + (pos + 1) / P];"),
+}
+
+
+def failing_paged_pins(orc):
+    failed = 0
+    for check in (lambda: pins.test_paged_cache_is_the_contiguous_cache_with_rows_moved(orc, False),
+                  lambda: pins.test_paged_cache_is_the_contiguous_cache_with_rows_moved(orc, True),
+                  lambda: pins.test_paged_unmapped_page_is_skipped_with_status(orc)):
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_paged_pins_pass_on_committed_oracle(orc):
+    assert failing_paged_pins(orc) == 0
+
+
+@pytest.mark.parametrize("name", sorted(PAGED_MUTATIONS))
+def test_planted_paged_mistake_is_caught(name, tmp_path, monkeypatch):
+    before, after = PAGED_MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not unique"
+    mutated = tmp_path / "tq_oracle_mut.cpp"
+    mutated.write_text(src.replace(before, after))
+    lib_path = tmp_path / f"libtq_oracle_{name}.so"
+    subprocess.run(["g++", *CXXFLAGS, "-o", str(lib_path), str(mutated)], check=True)
+    lib = oracle.bind(ctypes.CDLL(os.fspath(lib_path)))
+    monkeypatch.setattr(oracle, "_lib", lib)
+    assert failing_paged_pins(oracle) >= 1, f"no pin caught the planted mistake {name}"

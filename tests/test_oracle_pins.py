@@ -825,3 +825,69 @@ def test_sparse_v_zero_threshold_is_exact_and_the_drop_rule(orc):
     got, bound, _ = orc.decode_attention_ext(s, qd, lens, kc, ks, vc, vs, 0.3, tau=0.01)
     ref, rb = brute_force_ext(qd, lens, kc, ks, vc, vs, s, 0.3, tau=0.01)
     assert np.max(np.abs(got - ref)) < 2e-6 * max(1.0, np.abs(ref).max())
+
+
+# ---------------------------------------------------------------- paged storage
+# mlxcel guide, §"Known limitations / paged KV scheduler": a paged decode storage
+# backend. A paged cache is the contiguous cache with its rows moved to pool pages.
+
+def paged_table(rng, B, max_seq, P, n_pages):
+    max_pages = -(-max_seq // P)
+    perm = rng.permutation(n_pages)[: B * max_pages]
+    return perm.reshape(B, max_pages).astype(np.int32)
+
+
+@pytest.mark.parametrize("kf16", [False, True])
+def test_paged_cache_is_the_contiguous_cache_with_rows_moved(orc, kf16):
+    rng = np.random.default_rng(61 + kf16)
+    B, T, Hkv, D, P = 3, 45, 2, 64, 16
+    n_pages = B * (-(-T // P)) + 5
+    s = orc.sign_vector(0, D)
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    table = paged_table(rng, B, T, P, n_pages)
+    pools = orc.new_pool(n_pages, P, Hkv, D, kf16)
+    # in chunks that cross page boundaries
+    pos = 0
+    for c in (7, 16, 1, 21):
+        st = orc.quantize_append_paged(s, k[:, pos:pos + c], v[:, pos:pos + c], np.full(B, pos, np.int32), table,
+                                       P, T, pools)
+        assert st == 0
+        pos += c
+    # the pinned contiguous append of the same tokens
+    vc, vs = orc.new_cache(B, T, Hkv, D)
+    if kf16:
+        kc = orc.new_k16_cache(B, T, Hkv, D)
+        orc.quantize_append_kf16(s, k, v, np.zeros(B, np.int32), kc, vc, vs)
+    else:
+        kc, ks = orc.new_cache(B, T, Hkv, D)
+        orc.quantize_append(s, k, v, np.zeros(B, np.int32), kc, ks, vc, vs)
+    pk, pks, pv, pvs = pools
+    for b in range(B):
+        for t in range(T):
+            r = table[b, t // P] * P + t % P
+            assert np.array_equal(pk[r], kc[b, t]) and np.array_equal(pv[r], vc[b, t]) and np.array_equal(pvs[r], vs[b, t])
+            if not kf16:
+                assert np.array_equal(pks[r], ks[b, t])
+    # decode: the same values as the contiguous decode
+    q = rng.standard_normal((B, 4, D)).astype(np.float32)
+    lens = np.array([T, 17, 0], np.int32)
+    got, st = orc.decode_attention_paged(s, q, lens, table, P, T, pools, 0.15)
+    if kf16:
+        ref, _ = orc.decode_attention_kf16(s, q, lens, kc, vc, vs, 0.15)
+    else:
+        ref, _ = orc.decode_attention(s, q, lens, kc, ks, vc, vs, 0.15)
+    assert st == 0 and np.array_equal(got, ref)
+
+
+def test_paged_unmapped_page_is_skipped_with_status(orc):
+    rng = np.random.default_rng(63)
+    B, T, Hkv, D, P = 1, 40, 1, 32, 16
+    s = orc.sign_vector(0, D)
+    table = np.array([[2, -1, 0]], np.int32)
+    pools = orc.new_pool(3, P, Hkv, D)
+    k = rng.standard_normal((B, T, Hkv, D)).astype(np.float32)
+    st = orc.quantize_append_paged(s, k, k, np.zeros(B, np.int32), table, P, T, pools)
+    assert st & orc.STATUS_CAPACITY
+    assert np.all(pools[2][1 * P:2 * P] == 0)  # page 1 was never mapped, so never written
+    assert np.any(pools[2][2 * P:3 * P] != 0) and np.any(pools[2][0:P] != 0)
