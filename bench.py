@@ -54,6 +54,9 @@ def parse_args(argv=None):
                     help="write and read the cache with seeded per-channel lambda vectors (K with int4 K, and V)")
     ap.add_argument("--sparse-v", type=float, default=0.0, metavar="TAU",
                     help="sparse-V threshold of the decode (0 = exact attention; the mlxcel guide's default is 1e-6)")
+    ap.add_argument("--paged", type=int, default=0, metavar="P",
+                    help="paged storage with P-token pages (a seeded random permutation of the pool's pages); "
+                         "int4 and fp16 formats")
     ap.add_argument("--sweep", action="store_true",
                     help="per-configuration report instead of the step benchmark: decode and prefill-quantise "
                          "times (median, p10, p90; cold L2, and warm L2 where the cache fits) for every workload "
@@ -527,12 +530,21 @@ def reference_points(w, t, L, kc, ks, vc, vs, lens1, q, dev, stream, args, fmt="
 class DeviceCache:
     """One cache format in device memory, driven through the library's C ABI (tq.py)."""
 
-    def __init__(self, w, cap, fmt, dev, lam=False, tau=0.0):
+    def __init__(self, w, cap, fmt, dev, lam=False, tau=0.0, page=0):
+        import torch
         from compressed_domain_attention_b200 import tq
-        self.tq, self.fmt, self.tau = tq, fmt, tau
+        self.tq, self.fmt, self.tau, self.page = tq, fmt, tau, page
         self.lk, self.lv = bench_lambdas(w.head_dim, fmt, dev) if lam else (None, None)
         shape = (cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
-        if fmt == "delegated":
+        if page:
+            kfmt = tq.TQ_K_INT4 if fmt == "int4" else tq.TQ_K_FP16
+            max_pages = -(-cap // page)
+            n_pages = w.batch * max_pages
+            self.L = tq.tq_cache_layout_paged(w.batch, *shape, kfmt, page, n_pages)
+            self.l1 = tq.tq_cache_layout_paged(1, *shape, kfmt, page, n_pages)
+            g = torch.Generator("cpu").manual_seed(77)  # pages scattered over the pool
+            self.table = torch.randperm(n_pages, generator=g).view(w.batch, max_pages).to(torch.int32).to(dev)
+        elif fmt == "delegated":
             W, F = delegated_window()
             self.L = tq.tq_cache_layout_delegated(w.batch, *shape, W, F)
             self.l1 = tq.tq_cache_layout_delegated(1, *shape, W, F)
@@ -551,6 +563,10 @@ class DeviceCache:
     def append_seq(self, b, k, v, n, zero, status, stream):
         """Prefill of sequence b alone (n tokens at position 0) through a batch-1 view."""
         L, tq = self.L, self.tq
+        if self.page:
+            tq.tq_quantize_append_paged(self.l1, k, v, n, zero, self.table[b:b + 1], self.kc, self.ks, self.vc,
+                                        self.vs, status, stream, lambda_k=self.lk, lambda_v=self.lv)
+            return
         cs, ss, kst = int(L.code_stride_seq), int(L.scale_stride_seq), int(L.k_stride_seq)
         kc, vc, vs = self.kc[b * kst:(b + 1) * kst], self.vc[b * cs:(b + 1) * cs], self.vs[b * ss:]
         if self.fmt == "delegated":
@@ -562,14 +578,21 @@ class DeviceCache:
                                   status, stream, lambda_k=self.lk, lambda_v=self.lv)
 
     def append(self, k, v, n, start, status, stream):
-        if self.fmt == "delegated":
+        if self.page:
+            self.tq.tq_quantize_append_paged(self.L, k, v, n, start, self.table, self.kc, self.ks, self.vc, self.vs,
+                                             status, stream, lambda_k=self.lk, lambda_v=self.lv)
+        elif self.fmt == "delegated":
             self.tq.tq_append_delegated(self.L, k, v, n, start, self.kc, self.vc, self.vs, self.tail, status, stream)
         else:
             self.tq.tq_quantize_append(self.L, k, v, n, start, self.kc, self.ks, self.vc, self.vs, status, stream,
                                        lambda_k=self.lk, lambda_v=self.lv)
 
     def decode(self, q, lens, scale, out, status, stream, after_split_event=None):
-        if self.fmt == "delegated":
+        if self.page:
+            self.tq.tq_decode_attention_paged(self.L, q, lens, self.table, self.kc, self.ks, self.vc, self.vs, scale,
+                                              out, self.wsp, status, stream, after_split_event=after_split_event,
+                                              lambda_k=self.lk, lambda_v=self.lv, sparse_v_threshold=self.tau)
+        elif self.fmt == "delegated":
             self.tq.tq_decode_attention_delegated(self.L, q, lens, self.kc, self.vc, self.vs, self.tail, scale, out,
                                                   self.wsp, status, stream, after_split_event=after_split_event,
                                                   sparse_v_threshold=self.tau)
@@ -751,7 +774,9 @@ def run_tq(args):
     fmt = args.k_format
     if args.lam and fmt == "delegated":
         raise SystemExit("--lambda applies to the int4 and fp16 formats (the delegated tail is binary16)")
-    cache = DeviceCache(w, cap, fmt, dev, args.lam, args.sparse_v)
+    if args.paged and fmt == "delegated":
+        raise SystemExit("--paged applies to the int4 and fp16 formats")
+    cache = DeviceCache(w, cap, fmt, dev, args.lam, args.sparse_v, args.paged)
     L = cache.L
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
@@ -916,7 +941,8 @@ def run_tq(args):
     peak, peak_kind = load_peaks()
     achieved = bytes_split / (split_avg / 1e3) / 1e9
     traffic = load_traffic(f"decode_split_kernel/{w.name}" + {"int4": "", "fp16": "/k_fp16",
-                                                                "delegated": "/delegated"}[fmt])
+                                                                "delegated": "/delegated"}[fmt]
+                           + (f"/paged{args.paged}" if args.paged else ""))
     cache_bytes = cache.nbytes()
     extra = {
         "tokens_per_s": round(ws * w.batch * w.n_append * args.steps / max_t, 1),
@@ -946,6 +972,7 @@ def run_tq(args):
            else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
            "k_format": args.k_format, "lambda": bool(args.lam), "sparse_v_threshold": args.sparse_v,
+           "page_tokens": args.paged,
            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
            "l2": f"inputs larger than L2 (cache {cache_bytes / 1e9:.2f} GB per replica > 126 MB), no flush",
            "algorithmic_bytes_per_step": bytes_step}

@@ -71,14 +71,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 3-D view of a codes buffer: (D/2 bytes, batch*max_seq tokens, n_kv heads),
+// Token rows of a cache buffer: batch * max_seq, or n_pages * page_tokens when paged.
+uint64_t pool_rows(const tq_layout_t* L) {
+  return L->page_tokens > 0 ? (uint64_t)L->n_pages * (uint64_t)L->page_tokens
+                            : (uint64_t)L->batch * (uint64_t)L->max_seq;
+}
+
+// 3-D view of a codes buffer: (D/2 bytes, token rows, n_kv heads),
 // box (D/2, tile, n_kv); the shared-memory image is [head][tile][D/2] with the
 // swizzle matching the row pitch.
 int encode_codes_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::TensorMap128* out) {
   auto enc = get_encode_fn();
   if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
   const int rb = L->head_dim / 2;
-  cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq, (cuuint64_t)L->n_kv_heads};
+  cuuint64_t dims[3] = {(cuuint64_t)rb, (cuuint64_t)pool_rows(L), (cuuint64_t)L->n_kv_heads};
   cuuint64_t strides[2] = {(cuuint64_t)L->code_stride_tok, (cuuint64_t)rb};
   cuuint32_t box[3] = {(cuuint32_t)rb, (cuuint32_t)tile, (cuuint32_t)L->n_kv_heads};
   cuuint32_t estr[3] = {1, 1, 1};
@@ -110,8 +116,7 @@ int encode_k16_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::Ten
   const int D = L->head_dim;
   const int inner = D < 64 ? D : 64;
   const int lines = D / inner;
-  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)L->batch * (cuuint64_t)L->max_seq, (cuuint64_t)lines,
-                        (cuuint64_t)L->n_kv_heads};
+  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)pool_rows(L), (cuuint64_t)lines, (cuuint64_t)L->n_kv_heads};
   cuuint64_t strides[3] = {(cuuint64_t)L->k_stride_tok, (cuuint64_t)inner * 2, (cuuint64_t)D * 2};
   cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)tile, (cuuint32_t)lines, (cuuint32_t)L->n_kv_heads};
   cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -129,13 +134,15 @@ int encode_k16_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::Ten
 }
 
 int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
-                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, tq_layout_t* out);
+                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, int page_tokens, int n_pages,
+                 tq_layout_t* out);
 
 int check_layout(const tq_layout_t* L) {
   if (L == nullptr) return TQ_ERR_INVALID_ARG;
   tq_layout_t chk;
   const int r = build_layout(L->batch, L->max_seq, L->n_kv_heads, L->n_q_heads, L->head_dim, L->group_size,
-                             L->sign_seed, L->k_format, L->tail_window, L->fold_chunk, &chk);
+                             L->sign_seed, L->k_format, L->tail_window, L->fold_chunk, L->page_tokens, L->n_pages,
+                             &chk);
   if (r != TQ_OK) return r;
   if (std::memcmp(&chk, L, sizeof(chk)) != 0) return TQ_ERR_INVALID_ARG;  // edited or stale layout
   return TQ_OK;
@@ -159,8 +166,14 @@ uint64_t workspace_bytes(int batch, int n_q, int D, int max_ctas, int tail_windo
 constexpr int kMaxTailWindow = 1024;  // the merge kernel keeps one score per hot token in shared memory
 
 int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
-                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, tq_layout_t* out) {
+                 uint64_t sign_seed, int k_format, int tail_window, int fold_chunk, int page_tokens, int n_pages,
+                 tq_layout_t* out) {
   if (out == nullptr) return TQ_ERR_INVALID_ARG;
+  if (page_tokens != 0 || n_pages != 0) {
+    if (k_format != TQ_K_INT4 && k_format != TQ_K_FP16) return TQ_ERR_INVALID_ARG;
+    if (!is_pow2(page_tokens) || page_tokens > 4096 || n_pages <= 0) return TQ_ERR_INVALID_ARG;
+    if ((int64_t)n_pages * page_tokens > (int64_t)INT32_MAX) return TQ_ERR_UNSUPPORTED;
+  }
   if (k_format != TQ_K_INT4 && k_format != TQ_K_FP16 && k_format != TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
   if (k_format == TQ_KV_DELEGATED) {
     if (tail_window < 1 || tail_window > kMaxTailWindow || fold_chunk < 1 || fold_chunk > tail_window)
@@ -174,6 +187,11 @@ int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head
   if (!is_pow2(head_dim) || head_dim < 32 || head_dim > 256) return TQ_ERR_UNSUPPORTED;
   if (group_size != 32) return TQ_ERR_UNSUPPORTED;
   if ((int64_t)batch * (int64_t)max_seq > (int64_t)INT32_MAX) return TQ_ERR_UNSUPPORTED;  // tensor-copy coordinates
+  if (page_tokens > 0) {  // no decode tile may cross a page
+    const int tile = tqk::decode_tile_tokens(head_dim, n_kv_heads, k_format == TQ_K_FP16 ? 1 : 0);
+    if (tile <= 0 || page_tokens % tile != 0) return TQ_ERR_UNSUPPORTED;
+  }
+  const int64_t rows = page_tokens > 0 ? (int64_t)n_pages * page_tokens : (int64_t)batch * max_seq;
   tq_layout_t L;
   std::memset(&L, 0, sizeof(L));
   L.batch = batch;
@@ -192,9 +210,9 @@ int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head
   L.code_stride_seq = (int64_t)max_seq * L.code_stride_tok;
   L.scale_stride_tok = (int64_t)n_kv_heads * L.n_groups;
   L.scale_stride_seq = (int64_t)max_seq * L.scale_stride_tok;
-  L.codes_bytes = (uint64_t)batch * (uint64_t)L.code_stride_seq;
+  L.codes_bytes = (uint64_t)rows * (uint64_t)L.code_stride_tok;
   const uint64_t srow = (uint64_t)L.scale_stride_tok * 2ull;
-  L.scales_bytes = (uint64_t)batch * (uint64_t)L.scale_stride_seq * 2ull + kMaxTileTokens * srow + 32ull;
+  L.scales_bytes = (uint64_t)rows * srow + kMaxTileTokens * srow + 32ull;
   L.max_ctas = kMaxCtas;
   L.decode_workspace_bytes =
       workspace_bytes(batch, n_q_heads, head_dim, kMaxCtas, k_format == TQ_KV_DELEGATED ? tail_window : 0);
@@ -202,11 +220,19 @@ int build_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head
   if (k_format != TQ_K_INT4) {
     L.k_stride_tok = (int64_t)n_kv_heads * head_dim * 2;
     L.k_stride_seq = (int64_t)max_seq * L.k_stride_tok;
-    L.k_bytes = (uint64_t)batch * (uint64_t)L.k_stride_seq;
+    L.k_bytes = (uint64_t)rows * (uint64_t)L.k_stride_tok;
   } else {
     L.k_stride_tok = L.code_stride_tok;
     L.k_stride_seq = L.code_stride_seq;
     L.k_bytes = L.codes_bytes;
+  }
+  if (page_tokens > 0) {
+    L.page_tokens = page_tokens;
+    L.n_pages = n_pages;
+    L.max_pages = (max_seq + page_tokens - 1) / page_tokens;
+    L.code_stride_seq = 0;  // no per-sequence slabs
+    L.scale_stride_seq = 0;
+    L.k_stride_seq = 0;
   }
   if (k_format == TQ_KV_DELEGATED) {
     L.tail_window = tail_window;
@@ -225,19 +251,28 @@ extern "C" {
 
 int tq_cache_layout(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
                     uint64_t sign_seed, tq_layout_t* out) {
-  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_K_INT4, 0, 0, out);
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_K_INT4, 0, 0, 0, 0,
+                      out);
 }
 
 int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
                        uint64_t sign_seed, int k_format, tq_layout_t* out) {
   if (k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;  // needs the window sizes
-  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, k_format, 0, 0, out);
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, k_format, 0, 0, 0, 0,
+                      out);
 }
 
 int tq_cache_layout_delegated(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
                               uint64_t sign_seed, int tail_window, int fold_chunk, tq_layout_t* out) {
   return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, TQ_KV_DELEGATED,
-                      tail_window, fold_chunk, out);
+                      tail_window, fold_chunk, 0, 0, out);
+}
+
+int tq_cache_layout_paged(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                          uint64_t sign_seed, int k_format, int page_tokens, int n_pages, tq_layout_t* out) {
+  if (page_tokens <= 0 || n_pages <= 0) return TQ_ERR_INVALID_ARG;
+  return build_layout(batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, sign_seed, k_format, 0, 0,
+                      page_tokens, n_pages, out);
 }
 
 int64_t tq_cold_length(const tq_layout_t* layout, int64_t len) {
@@ -250,7 +285,8 @@ namespace {
 int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
                 const int32_t* d_start_pos, uint8_t* k_codes, uint16_t* k_scales, uint8_t* v_codes,
                 uint16_t* v_scales, uint16_t* v_tail, const tq_append_opts_t* opts, int32_t* d_status,
-                void* stream) {
+                void* stream, const int32_t* d_block_table = nullptr) {
+  if ((layout->page_tokens > 0) != (d_block_table != nullptr)) return TQ_ERR_INVALID_ARG;
   const float* lam_k = opts ? opts->lambda_k : nullptr;
   const float* lam_v = opts ? opts->lambda_v : nullptr;
   // lambda scales quantised vectors: not binary16 K, not the delegated cache's tail
@@ -292,6 +328,10 @@ int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_
   p.fold_chunk = layout->fold_chunk;
   p.lambda_k = lam_k;
   p.lambda_v = lam_v;
+  p.block_table = d_block_table;
+  p.page_tokens = layout->page_tokens;
+  p.max_pages = layout->max_pages;
+  p.n_pages = layout->n_pages;
   cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
@@ -303,7 +343,7 @@ int tq_quantize_append(const tq_layout_t* layout, const void* k, const void* v, 
                        uint16_t* v_scales, int32_t* d_status, void* stream) {
   int r = check_layout(layout);
   if (r != TQ_OK) return r;
-  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  if (layout->k_format == TQ_KV_DELEGATED || layout->page_tokens > 0) return TQ_ERR_INVALID_ARG;
   return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
                      nullptr, d_status, stream);
 }
@@ -313,9 +353,20 @@ int tq_quantize_append_ex(const tq_layout_t* layout, const void* k, const void* 
                           uint16_t* v_scales, const tq_append_opts_t* opts, int32_t* d_status, void* stream) {
   int r = check_layout(layout);
   if (r != TQ_OK) return r;
-  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  if (layout->k_format == TQ_KV_DELEGATED || layout->page_tokens > 0) return TQ_ERR_INVALID_ARG;
   return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
                      opts, d_status, stream);
+}
+
+int tq_quantize_append_paged(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                             const int32_t* d_start_pos, const int32_t* d_block_table, uint8_t* k_codes,
+                             uint16_t* k_scales, uint8_t* v_codes, uint16_t* v_scales, const tq_append_opts_t* opts,
+                             int32_t* d_status, void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->page_tokens <= 0 || d_block_table == nullptr) return TQ_ERR_INVALID_ARG;
+  return append_impl(layout, k, v, in_dtype, n_new, d_start_pos, k_codes, k_scales, v_codes, v_scales, nullptr,
+                     opts, d_status, stream, d_block_table);
 }
 
 int tq_append_delegated(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
@@ -333,8 +384,10 @@ namespace {
 int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
                 const uint8_t* k_codes, const uint16_t* k_scales, const uint8_t* v_codes, const uint16_t* v_scales,
                 const uint16_t* v_tail, float sm_scale, float* out, void* workspace, size_t ws_bytes,
-                int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
+                int32_t* d_status, const tq_decode_opts_t* opts, void* stream,
+                const int32_t* d_block_table = nullptr) {
   int r = TQ_OK;
+  if ((layout->page_tokens > 0) != (d_block_table != nullptr)) return TQ_ERR_INVALID_ARG;
   const int D = layout->head_dim, Hkv = layout->n_kv_heads, Hq = layout->n_q_heads;
   const int G = Hq / Hkv;
   if (layout->batch > kMaxBatchDecode) return TQ_ERR_UNSUPPORTED;
@@ -421,6 +474,11 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
   p.lambda_k = lam_k;
   p.lambda_v = lam_v;
   p.sparse_lt = sparse_lt;
+  p.block_table = d_block_table;
+  p.page_tokens = layout->page_tokens;
+  p.max_pages = layout->max_pages;
+  p.n_pages = layout->n_pages;
+  p.len_align = layout->page_tokens > 0 ? tile : 1;
   cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
@@ -433,9 +491,21 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
                            int32_t* d_status, const tq_decode_opts_t* opts, void* stream) {
   int r = check_layout(layout);
   if (r != TQ_OK) return r;
-  if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;
+  if (layout->k_format == TQ_KV_DELEGATED || layout->page_tokens > 0) return TQ_ERR_INVALID_ARG;
   return decode_impl(layout, q, q_dtype, d_seq_lens, k_codes, k_scales, v_codes, v_scales, nullptr, sm_scale, out,
                      workspace, ws_bytes, d_status, opts, stream);
+}
+
+int tq_decode_attention_paged(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                              const int32_t* d_block_table, const uint8_t* k_codes, const uint16_t* k_scales,
+                              const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
+                              void* workspace, size_t ws_bytes, int32_t* d_status, const tq_decode_opts_t* opts,
+                              void* stream) {
+  int r = check_layout(layout);
+  if (r != TQ_OK) return r;
+  if (layout->page_tokens <= 0 || d_block_table == nullptr) return TQ_ERR_INVALID_ARG;
+  return decode_impl(layout, q, q_dtype, d_seq_lens, k_codes, k_scales, v_codes, v_scales, nullptr, sm_scale, out,
+                     workspace, ws_bytes, d_status, opts, stream, d_block_table);
 }
 
 int tq_decode_attention_delegated(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,

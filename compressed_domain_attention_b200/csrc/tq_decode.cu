@@ -129,7 +129,12 @@ __device__ void block_prefix_lengths(const DecodeParams& p, int64_t* prefix, int
     int64_t L = 0;
     if (b < p.batch) {
       const int x = p.seq_lens[b];
-      if (x < 0 || x > p.max_seq) bad = true; else L = cold_tokens(x, p.tail_window, p.fold_chunk);
+      if (x < 0 || x > p.max_seq) {
+        bad = true;
+      } else {  // padded to whole tiles with paged storage (len_align 1 otherwise)
+        L = cold_tokens(x, p.tail_window, p.fold_chunk);
+        L = (L + p.len_align - 1) / p.len_align * p.len_align;
+      }
     }
     v[i] = L;
     local += L;
@@ -163,6 +168,19 @@ __device__ void block_prefix_lengths(const DecodeParams& p, int64_t* prefix, int
   __syncthreads();
 }
 
+// First cache row of the tile of sequence b starting at token t0: b * max_seq + t0,
+// or through the block table with paged storage (the tile lies in one page). An
+// unmapped page gives ok = false and row 0 (the producer then points its tensor
+// copies past the pool, where they read zeros, and copies its scales from row 0;
+// the converters must locate the scales at the same row).
+__device__ __forceinline__ int64_t tile_first_row(const DecodeParams& p, int b, int t0, bool& ok) {
+  ok = true;
+  if (p.page_tokens <= 0) return (int64_t)b * p.max_seq + t0;
+  const int pg = p.block_table[(int64_t)b * p.max_pages + t0 / p.page_tokens];
+  ok = pg >= 0 && pg < p.n_pages;
+  return ok ? (int64_t)pg * p.page_tokens + t0 % p.page_tokens : 0;
+}
+
 // Tile walk shared by the producer and the consumers: visits every
 // (sequence b, token offset t0, tokens valid in the tile) of this CTA's range.
 struct TileWalker {
@@ -171,12 +189,17 @@ struct TileWalker {
   int64_t lo, hi;
   int b;
   int seg_lo, seg_hi, t0;  // token offsets within sequence b (< max_seq)
+  const int32_t* lens;     // paged storage: true lengths (the prefix holds padded ones); else nullptr
+  int max_seq;
 
-  __device__ void start(const int64_t* pf, int nb, int64_t l, int64_t h) {
+  __device__ void start(const int64_t* pf, int nb, int64_t l, int64_t h, const int32_t* true_lens = nullptr,
+                        int ms = 0) {
     prefix = pf;
     batch = nb;
     lo = l;
     hi = h;
+    lens = true_lens;
+    max_seq = ms;
     // first sequence whose token range ends after lo
     int a = 0, z = nb - 1;
     while (a < z) {
@@ -191,7 +214,11 @@ struct TileWalker {
   __device__ void next_segment_from(int bb) {
     for (b = bb; b < batch && prefix[b] < hi; ++b) {
       const int64_t s0 = max(lo, prefix[b]) - prefix[b];
-      const int64_t s1 = min(hi, prefix[b + 1]) - prefix[b];
+      int64_t s1 = min(hi, prefix[b + 1]) - prefix[b];
+      if (lens != nullptr) {  // the padding past the true length is never read
+        const int x = lens[b];
+        s1 = min(s1, (int64_t)((x < 0 || x > max_seq) ? 0 : x));
+      }
       if (s0 < s1) {
         seg_lo = (int)s0;
         seg_hi = (int)s1;
@@ -252,7 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t T_sum = prefix[p.batch];
   int64_t R = (T_sum + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
-  R = ((R + 15) / 16) * 16;
+  const int64_t r_align = p.len_align > 16 ? p.len_align : 16;  // whole tiles with paged storage
+  R = ((R + r_align - 1) / r_align) * r_align;
   if (blockIdx.x == 0) {  // header for the merge kernel
     int64_t* hdr = ws_header(p.ws_ml);
     for (int i = tid; i <= p.batch; i += kThreads) hdr[i] = prefix[i];
@@ -270,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   TileWalker walk;
-  walk.start(prefix, p.batch, lo, hi);
+  walk.start(prefix, p.batch, lo, hi, p.page_tokens > 0 ? p.seq_lens : nullptr, p.max_seq);
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -290,13 +318,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*reinterpret_cast<volatile int*>(&misc[0]) != 0) break;
       uint8_t* sb = smem + stage * C::STAGE_BYTES;
       mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
-      const int row = (int)((int64_t)walk.b * p.max_seq + walk.t0);
+      // paged storage: the tile lies in one page (tiles start at multiples of the tile
+      // size, pages hold whole tiles)
+      bool mapped;
+      const int srow = (int)tile_first_row(p, walk.b, walk.t0, mapped);  // first scale row of the tile
+      if (!mapped) status_or(p.status, TQ_STATUS_CAPACITY);
+      const int row = mapped ? srow : p.n_pages * p.page_tokens;  // past the pool: zero-filled copies
       if constexpr (KF16)
         tma_load_4d(sb, &kmap, &full[stage], 0, row, 0, 0, pol);
       else
         tma_load_3d(sb, &kmap, &full[stage], 0, row, 0, pol);
       tma_load_3d(sb + C::OFF_VCODE, &vmap, &full[stage], 0, row, 0, pol);
-      const int64_t soff = (int64_t)row * C::SROW;  // byte offset of the tile's first scale row
+      const int64_t soff = (int64_t)srow * C::SROW;  // byte offset of the tile's first scale row
       const int64_t salign = soff & ~(int64_t)15;
       if constexpr (!KF16) bulk_load(sb + C::OFF_RAW, ks_base + salign, C::SCALE_SLAB, &full[stage], pol);
       bulk_load(sb + C::OFF_RAWV, vs_base + salign, C::SCALE_SLAB, &full[stage], pol);
@@ -352,7 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!dead) {
         uint8_t* sb = smem + stage * C::STAGE_BYTES;
-        const int64_t row0 = (int64_t)walk.b * p.max_seq + walk.t0;
+        bool mapped;
+        const int64_t row0 = tile_first_row(p, walk.b, walk.t0, mapped);  // the producer's scale row
         const int soff = (int)((row0 * C::SROW) & 15);
         const int nv = min(T_TILE, walk.seg_hi - walk.t0);
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
@@ -1400,7 +1434,8 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   for (int i = tid; i < p.batch; i += NTH) {
     int x = p.seq_lens[i];
     if (x < 0 || x > p.max_seq) x = 0;
-    const long long c = cold_tokens(x, p.tail_window, p.fold_chunk);
+    long long c = cold_tokens(x, p.tail_window, p.fold_chunk);
+    c = (c + p.len_align - 1) / p.len_align * p.len_align;  // the split-K kernel's padded lengths
     total += c;
     if (i < b) before += c;
   }
@@ -1426,7 +1461,9 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   const int64_t len_b = cold_tokens(len_all, p.tail_window, p.fold_chunk);
   int64_t R = (total + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
-  R = ((R + 15) / 16) * 16;
+  const int64_t r_align = p.len_align > 16 ? p.len_align : 16;
+  R = ((R + r_align - 1) / r_align) * r_align;
+  // the last partial is that of the CTA holding the last TRUE token (padding is never read)
   const int64_t P0 = before, P1 = before + len_b;
   // Delegated cache: the hot tail's partials (one per chunk of hot tokens, in the
   // rotated domain like the rest) follow in slots tail_slot0 + b * tail_chunks + k.

@@ -25,6 +25,10 @@ struct QuantizeParams {
   int tail_window, fold_chunk;
   const float* lambda_k;  // per-channel lambda in the rotated domain (nullable)
   const float* lambda_v;
+  // paged storage (page_tokens > 0): pool row of token t of sequence b =
+  // block_table[b * max_pages + t / page_tokens] * page_tokens + t % page_tokens
+  const int32_t* block_table;
+  int page_tokens, max_pages, n_pages;
 };
 
 struct DequantParams {
@@ -70,6 +74,12 @@ struct DecodeParams {
   const float* lambda_k;  // per-channel lambda of the cache (nullable): q is divided by lambda_k,
   const float* lambda_v;  // the merged V sum by lambda_v, both in the rotated domain
   float sparse_lt;        // log2 of the sparse-V threshold; -inf = off
+  // paged storage (page_tokens > 0): as in QuantizeParams. len_align: each
+  // sequence's length is padded to a multiple of it in the split-K token space
+  // (the kernel's tile, so that no tile crosses a page), 1 without paging.
+  const int32_t* block_table;
+  int page_tokens, max_pages, n_pages;
+  int len_align;
 };
 
 // Hot-tail partials per sequence of the delegated cache (64 tokens each).

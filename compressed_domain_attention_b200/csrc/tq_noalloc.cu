@@ -81,6 +81,7 @@ extern "C" int tq_decode_attention_noalloc(const tq_layout_t* layout, const void
                                            int32_t* d_status, void* stream) {
   if (layout == nullptr) return TQ_ERR_INVALID_ARG;
   if (layout->k_format == TQ_KV_DELEGATED) return TQ_ERR_INVALID_ARG;  // no hot-tail argument here
+  if (layout->page_tokens > 0) return TQ_ERR_INVALID_ARG;              // no block-table argument here
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return TQ_ERR_CUDA;

@@ -23,6 +23,16 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
+// Cache row of token t of sequence b: b * max_seq + t, or through the block table
+// with paged storage (ok = false for an entry outside [0, n_pages)).
+__device__ __forceinline__ int64_t token_row(const QuantizeParams& p, int b, int64_t t, bool& ok) {
+  ok = true;
+  if (p.page_tokens <= 0) return (int64_t)b * p.max_seq + t;
+  const int pg = p.block_table[(int64_t)b * p.max_pages + t / p.page_tokens];
+  ok = pg >= 0 && pg < p.n_pages;
+  return (int64_t)(ok ? pg : 0) * p.page_tokens + t % p.page_tokens;
+}
+
 // Asymmetric cache (mlxcel guide, cache modes: K kept in FP16): thread kt stores
 // the binary16 (round to nearest even) of 32 consecutive K elements.
 template <int D>
@@ -50,7 +60,12 @@ __device__ __forceinline__ void copy_k_f16(const QuantizeParams& p, int64_t kt) 
     finite = finite && ((w[i] & 0x7C00u) != 0x7C00u) && ((w[i] & 0x7C000000u) != 0x7C000000u);
   }
   if (!finite) status_or(p.status, TQ_STATUS_NONFINITE);
-  const int64_t row = ((int64_t)b * p.max_seq + pos + t) * p.n_kv + h;
+  bool ok;
+  const int64_t row = token_row(p, b, pos + t, ok) * p.n_kv + h;
+  if (!ok) {
+    if (part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
+    return;
+  }
   uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.k_codes) + row * D + part * 32);
 #pragma unroll
   for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
@@ -274,7 +289,12 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
       }
     }
   }
-  const int64_t row = ((int64_t)b * p.max_seq + dst) * p.n_kv + h;
+  bool row_ok;
+  const int64_t row = token_row(p, b, dst, row_ok) * p.n_kv + h;
+  if (!row_ok) {  // an unmapped page: nothing is written
+    if (part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
+    return;
+  }
   uint8_t* codes = which ? p.v_codes : p.k_codes;
   uint16_t* scales = which ? p.v_scales : p.k_scales;
   *reinterpret_cast<uint4*>(codes + row * (D / 2) + part * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);

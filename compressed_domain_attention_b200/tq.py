@@ -28,10 +28,11 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 TQ_K_INT4, TQ_K_FP16, TQ_KV_DELEGATED = 0, 1, 2
 
 # C symbols declared in include/tq.h
-EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_cache_layout_delegated", "tq_cold_length",
-           "tq_quantize_append", "tq_quantize_append_ex", "tq_append_delegated", "tq_decode_attention", "tq_decode_attention_ex",
-           "tq_decode_attention_delegated", "tq_decode_attention_noalloc", "tq_dequantize_debug",
-           "tq_status_string", "tq_last_cuda_error")
+EXPORTS = ("tq_cache_layout", "tq_cache_layout_kv", "tq_cache_layout_delegated", "tq_cache_layout_paged",
+           "tq_cold_length", "tq_quantize_append", "tq_quantize_append_ex", "tq_quantize_append_paged",
+           "tq_append_delegated", "tq_decode_attention", "tq_decode_attention_ex", "tq_decode_attention_delegated",
+           "tq_decode_attention_paged", "tq_decode_attention_noalloc", "tq_dequantize_debug", "tq_status_string",
+           "tq_last_cuda_error")
 
 TQ_NOALLOC_WORKSPACE_BYTES = 8 << 20
 
@@ -50,6 +51,8 @@ class TqLayout(ctypes.Structure):
         ("k_bytes", ctypes.c_uint64), ("k_stride_tok", ctypes.c_int64), ("k_stride_seq", ctypes.c_int64),
         ("tail_window", ctypes.c_int32), ("fold_chunk", ctypes.c_int32), ("tail_bytes", ctypes.c_uint64),
         ("tail_stride_tok", ctypes.c_int64), ("tail_stride_seq", ctypes.c_int64),
+        ("page_tokens", ctypes.c_int32), ("n_pages", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+        ("reserved_paged", ctypes.c_int32),
     ]
 
 
@@ -96,6 +99,14 @@ def _lib():
         lib.tq_quantize_append_ex.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P,
                                               ctypes.POINTER(TqAppendOpts), P, P]
         lib.tq_quantize_append_ex.restype = I
+        lib.tq_cache_layout_paged.argtypes = [I, I, I, I, I, I, U64, I, I, I, ctypes.POINTER(TqLayout)]
+        lib.tq_cache_layout_paged.restype = I
+        lib.tq_quantize_append_paged.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P,
+                                                 ctypes.POINTER(TqAppendOpts), P, P]
+        lib.tq_quantize_append_paged.restype = I
+        lib.tq_decode_attention_paged.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P, P, ctypes.c_float,
+                                                  P, P, ctypes.c_size_t, P, ctypes.POINTER(TqDecodeOpts), P]
+        lib.tq_decode_attention_paged.restype = I
         lib.tq_append_delegated.argtypes = [ctypes.POINTER(TqLayout), P, P, I, I, P, P, P, P, P, P, P]
         lib.tq_append_delegated.restype = I
         lib.tq_decode_attention_delegated.argtypes = [ctypes.POINTER(TqLayout), P, I, P, P, P, P, P,
@@ -170,6 +181,45 @@ def tq_cache_layout_delegated(batch, max_seq, n_kv_heads, n_q_heads, head_dim, t
         batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, ctypes.c_uint64(sign_seed), int(tail_window),
         int(fold_chunk), ctypes.byref(out)))
     return out
+
+
+def tq_cache_layout_paged(batch, max_seq, n_kv_heads, n_q_heads, head_dim, k_format, page_tokens, n_pages,
+                          group_size=32, sign_seed=0) -> TqLayout:
+    """Paged storage: pools of n_pages pages of page_tokens tokens, addressed through a block table."""
+    out = TqLayout()
+    _check("tq_cache_layout_paged", _lib().tq_cache_layout_paged(
+        batch, max_seq, n_kv_heads, n_q_heads, head_dim, group_size, ctypes.c_uint64(sign_seed), int(k_format),
+        int(page_tokens), int(n_pages), ctypes.byref(out)))
+    return out
+
+
+def tq_quantize_append_paged(layout, k, v, n_new, start_pos, block_table, k_codes, k_scales, v_codes, v_scales,
+                             status=None, stream=None, lambda_k=None, lambda_v=None):
+    """Append through the block table (int32 [batch][max_pages] on the device)."""
+    for t in (k, v, start_pos, block_table, k_codes, k_scales, v_codes, v_scales, lambda_k, lambda_v):
+        assert t is None or t.is_contiguous()
+    opts = TqAppendOpts(_ptr(lambda_k), _ptr(lambda_v)) if (lambda_k is not None or lambda_v is not None) else None
+    code = _lib().tq_quantize_append_paged(ctypes.byref(layout), _ptr(k), _ptr(v), _dtype_code(k), int(n_new),
+                                           _ptr(start_pos), _ptr(block_table), _ptr(k_codes), _ptr(k_scales),
+                                           _ptr(v_codes), _ptr(v_scales),
+                                           ctypes.byref(opts) if opts is not None else None, _ptr(status),
+                                           _stream(stream))
+    _check("tq_quantize_append_paged", code)
+
+
+def tq_decode_attention_paged(layout, q, seq_lens, block_table, k_codes, k_scales, v_codes, v_scales, sm_scale, out,
+                              workspace, status=None, stream=None, min_split_tokens=0, max_ctas=0,
+                              after_split_event=None, lambda_k=None, lambda_v=None, sparse_v_threshold=0.0):
+    """Decode over a paged cache through the block table."""
+    for t in (q, seq_lens, block_table, k_codes, k_scales, v_codes, v_scales, out, workspace):
+        assert t is None or t.is_contiguous()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    opts = _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k, lambda_v, sparse_v_threshold)
+    code = _lib().tq_decode_attention_paged(
+        ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens), _ptr(block_table), _ptr(k_codes),
+        _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), ctypes.c_float(sm_scale), _ptr(out), _ptr(workspace),
+        ws_bytes, _ptr(status), ctypes.byref(opts) if opts is not None else None, _stream(stream))
+    _check("tq_decode_attention_paged", code)
 
 
 def tq_cold_length(layout, length) -> int:

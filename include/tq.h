@@ -113,6 +113,10 @@ typedef struct {
   uint64_t tail_bytes;         /* allocation size of the hot tail (0 unless TQ_KV_DELEGATED) */
   int64_t tail_stride_tok;     /* bytes between tail slots of one sequence = n_kv * D * 2 */
   int64_t tail_stride_seq;     /* bytes between sequences in the tail     = W * n_kv * D * 2 */
+  int32_t page_tokens;         /* paged storage: tokens per page (P); 0 = per-sequence slabs */
+  int32_t n_pages;             /* paged storage: pages in each pool */
+  int32_t max_pages;           /* paged storage: block-table entries per sequence = ceil(max_seq / P) */
+  int32_t reserved_paged;
 } tq_layout_t;
 
 /* Optional knobs for tq_decode_attention_ex / _delegated (NULL = defaults; zero-fill unused fields). */
@@ -181,6 +185,43 @@ int tq_cache_layout_kv(int batch, int max_seq, int n_kv_heads, int n_q_heads, in
 int tq_cache_layout_delegated(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim,
                               int group_size, uint64_t sign_seed, int tail_window, int fold_chunk,
                               tq_layout_t* out);
+
+/*
+ * Paged storage (mlxcel guide, §"Known limitations / paged KV scheduler": the
+ * paged decode storage backend; it cites PagedAttention). The caches become
+ * pools of n_pages pages of P = page_tokens tokens: codes
+ * [n_pages * P][n_kv_heads][head_dim/2], scales [n_pages * P][n_kv_heads][head_dim/32]
+ * (binary16 K [n_pages * P][n_kv_heads][head_dim] with TQ_K_FP16), i.e. the
+ * contiguous layout with batch * max_seq rows replaced by n_pages * P rows. A
+ * caller-owned device block table int32 [batch][max_pages] maps token t of
+ * sequence b to pool row table[b][t / P] * P + t % P. P is a power of two,
+ * at least the decode kernel's token tile for this shape (16 to 256; else
+ * TQ_ERR_UNSUPPORTED) and at most 4096. k_format TQ_K_INT4 or TQ_K_FP16.
+ */
+int tq_cache_layout_paged(int batch, int max_seq, int n_kv_heads, int n_q_heads, int head_dim, int group_size,
+                          uint64_t sign_seed, int k_format, int page_tokens, int n_pages, tq_layout_t* out);
+
+/*
+ * tq_quantize_append_ex on a paged layout. d_block_table: device int32
+ * [batch][max_pages]; every page a token lands in must be mapped (an entry
+ * outside [0, n_pages) skips that token's vectors and sets TQ_STATUS_CAPACITY).
+ */
+int tq_quantize_append_paged(const tq_layout_t* layout, const void* k, const void* v, int in_dtype, int n_new,
+                             const int32_t* d_start_pos, const int32_t* d_block_table, uint8_t* k_codes,
+                             uint16_t* k_scales, uint8_t* v_codes, uint16_t* v_scales, const tq_append_opts_t* opts,
+                             int32_t* d_status, void* stream);
+
+/*
+ * tq_decode_attention_ex on a paged layout: the split-K kernel's token tiles
+ * are read through the block table (each tile lies in one page). A table entry
+ * outside [0, n_pages) on a sequence's token range reads zeros for that tile
+ * and sets TQ_STATUS_CAPACITY. Workspace as layout->decode_workspace_bytes.
+ */
+int tq_decode_attention_paged(const tq_layout_t* layout, const void* q, int q_dtype, const int32_t* d_seq_lens,
+                              const int32_t* d_block_table, const uint8_t* k_codes, const uint16_t* k_scales,
+                              const uint8_t* v_codes, const uint16_t* v_scales, float sm_scale, float* out,
+                              void* workspace, size_t ws_bytes, int32_t* d_status, const tq_decode_opts_t* opts,
+                              void* stream);
 
 /* Cold (int4) tokens of a delegated-cache sequence of len tokens; len for other
  * formats; -1 for a NULL layout or len < 0. Host only. */

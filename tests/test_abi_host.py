@@ -216,3 +216,27 @@ def test_delegated_layout_rejected_by_the_other_entry_points():
     assert lib.tq_decode_attention_delegated(ctypes.byref(L16), fake, 0, fake, fake, fake, fake, fake,
                                              ctypes.c_float(0.1), fake, fake, 1 << 30, None, None,
                                              None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_layout_paged_sizes_and_checks():
+    L = tq.tq_cache_layout_paged(4, 1000, 8, 32, 128, tq.TQ_K_INT4, 64, 70)
+    assert (L.page_tokens, L.n_pages, L.max_pages) == (64, 70, 16)
+    assert L.codes_bytes == 70 * 64 * 8 * 64
+    assert L.code_stride_seq == 0 and L.code_stride_tok == 8 * 64
+    L16 = tq.tq_cache_layout_paged(4, 1000, 8, 32, 128, tq.TQ_K_FP16, 64, 70)
+    assert L16.k_bytes == 70 * 64 * 8 * 128 * 2
+    for args, code in (((4, 1000, 8, 32, 128, tq.TQ_K_INT4, 48, 70), tq.TQ_ERR_INVALID_ARG),   # not a power of two
+                       ((4, 1000, 8, 32, 128, tq.TQ_K_INT4, 64, 0), tq.TQ_ERR_INVALID_ARG),    # no pages
+                       ((4, 1000, 8, 32, 128, tq.TQ_KV_DELEGATED, 64, 70), tq.TQ_ERR_INVALID_ARG),
+                       ((4, 1000, 1, 4, 128, tq.TQ_K_INT4, 64, 70), tq.TQ_ERR_UNSUPPORTED)):   # tile of 256 tokens
+        with pytest.raises(tq.TqError) as exc:
+            tq.tq_cache_layout_paged(*args)
+        assert exc.value.code == code
+    # the slab entry points refuse a paged layout (no block table), before any device work
+    import ctypes
+    lib = tq._lib()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.tq_quantize_append(ctypes.byref(L), fake, fake, 0, 1, fake, fake, fake, fake, fake, None,
+                                  None) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_decode_attention(ctypes.byref(L), fake, 0, fake, fake, fake, fake, fake, ctypes.c_float(0.1),
+                                   fake, fake, 1 << 30, None, None) == tq.TQ_ERR_INVALID_ARG
