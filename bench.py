@@ -821,12 +821,39 @@ def run_tq(args):
         clocks.start()
         time.sleep(0.3)
     torch.cuda.synchronize()
-    # timed region: the production path (split-K and merge kernels back to back)
+    # The K steps captured once as a CUDA graph, so that the timed region measures the
+    # device (a ~50 us step is otherwise paced by the host's launch calls); eager
+    # launches if capture is refused.
+    step_mode = "cuda graph of the K steps"
+    sgraph = torch.cuda.CUDAGraph()
+    sstream = torch.cuda.Stream(device=dev)
+    try:
+        sstream.wait_stream(stream)
+        with torch.cuda.graph(sgraph, stream=sstream):
+            for _ in range(args.steps):
+                cache.append(k_new, v_new, w.n_append, lens, status, sstream)
+                cache.decode(q, lens1, w.scale, out, status, sstream)
+        with torch.cuda.stream(sstream):
+            sgraph.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # noqa: BLE001 - reported in the output line
+        sgraph = None
+        step_mode = f"eager launches (graph capture failed: {type(exc).__name__})"
+        torch.cuda.synchronize()
+    barrier(dev)
+    # timed region: the production path (append, split-K and merge kernels back to back)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    stop.record(stream)
+    if sgraph is not None:
+        sstream.wait_stream(stream)
+        with torch.cuda.stream(sstream):  # replay() launches on the current stream
+            start.record(sstream)
+            sgraph.replay()
+            stop.record(sstream)
+    else:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
     clk = clocks.stop() if clocks else None
@@ -960,7 +987,8 @@ def run_tq(args):
                 "d2h_bytes_per_step": int(out.numel() * out.element_size()),
                 "copies": "pinned host buffers; step i+1's inputs in and step i's output out on a copy "
                           "stream while step i computes (double-buffered, event-ordered)", "launch": e2e_mode},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (4 if fmt == "delegated" else 3) * args.steps,
+        "step_launch": step_mode,
         "kernel_timing": "split-K/merge durations from a second pass of the same K steps with an event "
                          "between the two kernels (the timed region itself launches the merge as a "
                          "programmatic dependent)",
