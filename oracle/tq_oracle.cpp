@@ -233,6 +233,18 @@ void dequantize_rotated(const uint8_t* bytes, const uint16_t* scales, int D, flo
   for (int i = 0; i < D; ++i) yhat[i] = (float)codes[i] * f16_to_f32(scales[i / 32]);
 }
 
+// [MLX-modes] binary16 (round to nearest even) of one K row; a non-finite
+// result raises ORC_STATUS_NONFINITE (its bits are stored as converted).
+int32_t store_k_f16(const float* x, int D, uint16_t* dst) {
+  int32_t st = 0;
+  for (int i = 0; i < D; ++i) {
+    const uint16_t hbits = f32_to_f16_rne(x[i]);
+    if ((hbits & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
+    dst[i] = hbits;
+  }
+  return st;
+}
+
 // ---- delegated hot/cold cache [MLX-deleg] ----
 // Reading taken (the guide names the parts, not the policy): the hot tail holds
 // the most recent tokens' V in binary16, at most W of them, in a ring of W slots
@@ -495,11 +507,7 @@ int32_t oracle_quantize_append_kf16(int batch, int max_seq, int n_kv, int D, con
       for (int h = 0; h < n_kv; ++h) {
         const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
         const int64_t row = ((int64_t)b * max_seq + p0 + t) * n_kv + h;
-        for (int i = 0; i < D; ++i) {
-          const uint16_t hbits = f32_to_f16_rne(k[src + i]);
-          if ((hbits & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
-          k_f16[row * D + i] = hbits;
-        }
+        st |= store_k_f16(k + src, D, k_f16 + row * D);
         st |= oracle_encode(v + src, s, D, 1, v_codes + row * cb, v_scales + row * sb);
       }
     }
@@ -606,11 +614,7 @@ int32_t oracle_quantize_append_paged(int batch, int max_seq, int n_kv, int D, co
         const int64_t src = (((int64_t)b * n_new + t) * n_kv + h) * D;
         const int64_t row = prow * n_kv + h;
         if (k_f16) {
-          for (int i = 0; i < D; ++i) {
-            const uint16_t hbits = f32_to_f16_rne(k[src + i]);
-            if ((hbits & 0x7C00u) == 0x7C00u) st |= ORC_STATUS_NONFINITE;
-            k_f16[row * D + i] = hbits;
-          }
+          st |= store_k_f16(k + src, D, k_f16 + row * D);
         } else {
           st |= oracle_encode(k + src, s, D, 1, k_codes + row * cb, k_scales + row * sb);
         }

@@ -92,7 +92,7 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
 
 # Planted mistakes in the asymmetric (binary16 K) path, checked by its own pins.
 KF16_MUTATIONS = {
-    "kf16_k_index_reversed": ("k_f16[row * D + i] = hbits;", "k_f16[row * D + (D - 1 - i)] = hbits;"),
+    "kf16_k_index_reversed": ("    dst[i] = hbits;", "    dst[D - 1 - i] = hbits;"),
     "kf16_q_rotated": ("std::memcpy(qr.data(), q + ((int64_t)b * n_q + hq) * D, sizeof(float) * D);",
                        "srht_forward_vec(q + ((int64_t)b * n_q + hq) * D, s, D, qr.data());"),
     "kf16_k_halved": ("for (int i = 0; i < D; ++i) yk[i] = f16_to_f32(k_f16[row * D + i]);",
