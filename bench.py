@@ -646,13 +646,17 @@ def run_sweep(args):
     for fmt in ("fp16", "delegated"):
         cfgs += [("c1", syn.llama3_8b_layer, fmt), ("c3", syn.llama31_70b_long, fmt),
                  ("c4", syn.ragged_serving, fmt)]
+    # paged storage (64-token pages) on the long-context and serving shapes
+    cfgs += [("c3", syn.llama31_70b_long, "int4/paged64"), ("c4", syn.ragged_serving, "int4/paged64")]
     for tag, make, fmt in cfgs:
         fmt = fmt or "int4"
+        page = int(fmt.split("/paged")[1]) if "/paged" in fmt else 0
+        fmt = fmt.split("/")[0]
         w = make()
         t = syn.generate(w, device="cuda")
         n_app = max(w.n_append, 1)
         cap = max(w.seq_lens) + n_app
-        cache = DeviceCache(w, cap, fmt, dev)
+        cache = DeviceCache(w, cap, fmt, dev, page=page)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
         zero = torch.zeros(1, dtype=torch.int32, device=dev)
         kb = [t.k[b][None].contiguous() for b in range(w.batch)]
@@ -704,7 +708,7 @@ def run_sweep(args):
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the sweep ({w.name})")
         ms = cold["median"]
-        line = {"sweep": tag, "workload": w.name, "k_format": fmt, "batch": w.batch,
+        line = {"sweep": tag, "workload": w.name, "k_format": fmt, "page_tokens": page, "batch": w.batch,
                 "tokens": sum(w.seq_lens), "cache_bytes_read": nbytes,
                 "decode_ms_cold_l2": cold, "decode_gbs": round(nbytes / ms / 1e6, 1),
                 "pct_of_8_tbs": round(nbytes / ms / 1e6 / 80.0, 2),

@@ -106,6 +106,7 @@ struct DecodeCfg {
   static constexpr int OFF_PREFIX = OFF_MISC + 64;
   static constexpr int SMEM_MAX = OFF_PREFIX + 8 * (kMaxBatch + 1) + 8 * 16;
   static_assert(T_TILE <= 256, "tensor-copy box limit");
+  static_assert((T_TILE & (T_TILE - 1)) == 0, "paged storage rounds lengths to tiles with a mask");
   static_assert(CODE_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "tiles must stay swizzle-aligned");
   static_assert((2 * NG * NT) % 4 == 0, "ldmatrix.x4 batches");
   static_assert(SMEM_MAX <= 232448, "shared memory per block");
@@ -133,7 +134,7 @@ __device__ void block_prefix_lengths(const DecodeParams& p, int64_t* prefix, int
         bad = true;
       } else {  // padded to whole tiles with paged storage (len_align 1 otherwise)
         L = cold_tokens(x, p.tail_window, p.fold_chunk);
-        L = (L + p.len_align - 1) / p.len_align * p.len_align;
+        L = (L + p.len_align - 1) & ~(int64_t)(p.len_align - 1);  // len_align is a power of two
       }
     }
     v[i] = L;
@@ -279,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t T_sum = prefix[p.batch];
   int64_t R = (T_sum + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
-  const int64_t r_align = p.len_align > 16 ? p.len_align : 16;  // whole tiles with paged storage
-  R = ((R + r_align - 1) / r_align) * r_align;
+  const int64_t r_align = p.len_align > 16 ? p.len_align : 16;  // whole tiles with paged storage (a power of two)
+  R = (R + r_align - 1) & ~(r_align - 1);
   if (blockIdx.x == 0) {  // header for the merge kernel
     int64_t* hdr = ws_header(p.ws_ml);
     for (int i = tid; i <= p.batch; i += kThreads) hdr[i] = prefix[i];
@@ -1435,7 +1436,7 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
     int x = p.seq_lens[i];
     if (x < 0 || x > p.max_seq) x = 0;
     long long c = cold_tokens(x, p.tail_window, p.fold_chunk);
-    c = (c + p.len_align - 1) / p.len_align * p.len_align;  // the split-K kernel's padded lengths
+    c = (c + p.len_align - 1) & ~(long long)(p.len_align - 1);  // the split-K kernel's padded lengths
     total += c;
     if (i < b) before += c;
   }
@@ -1462,7 +1463,7 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   int64_t R = (total + p.grid - 1) / p.grid;
   if (R < p.min_split) R = p.min_split;
   const int64_t r_align = p.len_align > 16 ? p.len_align : 16;
-  R = ((R + r_align - 1) / r_align) * r_align;
+  R = (R + r_align - 1) & ~(r_align - 1);
   // the last partial is that of the CTA holding the last TRUE token (padding is never read)
   const int64_t P0 = before, P1 = before + len_b;
   // Delegated cache: the hot tail's partials (one per chunk of hot tokens, in the
