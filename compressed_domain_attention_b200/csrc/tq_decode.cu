@@ -350,10 +350,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ converters
     // binary16 scale rows [token][head][group] -> fp32 [head][unit][group][tig][n-tile][e],
     // the order in which a consumer lane reads them; tokens past the segment end get 0.
-    // Lane work item k covers the token pair (2j, 2j + 1) of one head, j * HKV + hh =
-    // lane + 32k: both tokens land next to each other (e = 0, 1), so each group is
-    // one 8-byte store. The shared-memory offsets are the same for every tile.
-    // The kConverterWarps warps share the items of a tile.
+    // Lane work item k covers the token pair (2j, 2j + 1) of one head: both tokens land
+    // next to each other (e = 0, 1), so each group is one 8-byte store. Item i = lane +
+    // 32 k' takes head hh = i % HKV and, from r = i / HKV, the n-tile r % NT, the pair
+    // tg = (r / NT) % 4 within it and the unit r / (4 NT): the lanes of one store then
+    // spread over heads and n-tiles, which fall in different banks of the fp32 layout
+    // (the order "pairs of one n-tile first" put 4 lanes on each bank pair; it stays
+    // with 4 kv heads, where it conflicts less). The
+    // shared-memory offsets are the same for every tile. The kConverterWarps warps share
+    // the items of a tile.
     constexpr int PAIRS = T_TILE / 2 * HKV;
     constexpr int ITEMS = (PAIRS + 32 * kConverterWarps - 1) / (32 * kConverterWarps);
     const int cw = warp - kConverterWarp;
@@ -365,7 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int k = 0; k < ITEMS; ++k) {
       const int i = lane + 32 * (cw + kConverterWarps * k);
-      const int j = i / HKV, hh = i % HKV;
+      const int r = i / HKV, hh = i % HKV;
+      // a bijection on the pairs; with 4 kv heads the plain order conflicts less
+      const int j = HKV == 4 ? r : (r / (4 * NT)) * (UNIT / 2) + 4 * (r % NT) + (r / NT) % 4;
       const int t = 2 * j;
       const int u = t / UNIT, tau = t % UNIT;
       const int nt = tau >> 3, tg = (tau & 7) >> 1;
