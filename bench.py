@@ -863,7 +863,10 @@ def run_tq(args):
     clk = clocks.stop() if clocks else None
     elapsed = start.elapsed_time(stop) / 1e3
     # second timed pass of the same steps with an event between the split-K and
-    # merge kernels: per-kernel durations for the roofline
+    # merge kernels: per-kernel durations for the roofline. Eager launches: a short
+    # GPU spin first lets the host queue the steps ahead of the device, so no host
+    # gap (tensor-map encoding, launch calls) falls between an event and its kernel.
+    torch.cuda._sleep(int(2e6))
     for i in range(args.steps):
         step(i)
     torch.cuda.synchronize()
