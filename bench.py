@@ -394,6 +394,19 @@ class OracleStep:
             return time.perf_counter() - t0
 
 
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -406,6 +419,7 @@ def cpu_baseline(w, tensors, target_tokens, fmt="int4", lam=False, tau=0.0):
     o = OracleStep(w, tensors, seqs, fmt, lam, tau)
     dt = o.run()
     line = {"value": round(o.nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cores": host_cores(),
             "sample": f"one step (append + decode) on {len(seqs)} of {w.batch} sequences "
                       f"({o.ntok} KV tokens x {w.n_q_heads} q heads), single-threaded C++ oracle, {dt:.2f} s",
             "seconds": round(dt, 3)}
@@ -754,7 +768,8 @@ def run_reference(args):
                                                      "k_format": getattr(args, "k_format", "int4"),
                                                      "lambda": bool(getattr(args, "lam", False)),
                                                      "sparse_v_threshold": getattr(args, "sparse_v", 0.0)},
-            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model(), "host_cores": host_cores()},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
