@@ -121,7 +121,7 @@ typedef struct {
 
 /* Optional knobs for tq_decode_attention_ex / _delegated (NULL = defaults; zero-fill unused fields). */
 typedef struct {
-  int32_t min_split_tokens; /* 0 = default; otherwise the smallest token range one CTA takes */
+  int32_t min_split_tokens; /* 0 = default (64); otherwise the smallest token range one CTA takes */
   int32_t max_ctas;         /* 0 = default (one per SM); otherwise the split-K grid, <= layout.max_ctas */
   void* after_split_event;  /* a cudaEvent_t recorded on `stream` between the split-K and merge kernels, or NULL */
   /* Per-channel lambda the cache was written with (tq_append_opts_t), device
