@@ -71,8 +71,9 @@ class PagedPair:
 
 
 def prefill(pair, t, lens):
-    """Each sequence's prefix in one padded batched append at position 0 would write padding; append per
-    sequence length instead: sequences grouped by equal chunks of their own tokens."""
+    """Append every sequence's prefix in 37-token chunks (so appends cross page boundaries), all sequences
+    in one call per chunk: rows past a sequence's length get zero vectors, written identically by the GPU
+    and the oracle and never read by the decode."""
     w = pair.w
     T = max(lens)
     for start in range(0, T, 37):  # chunks that cross page boundaries
@@ -101,8 +102,7 @@ def test_paged_append_and_decode(D, Hkv, Hq, k_format, P):
     pair.check_pools()
     out, ref, st = pair.decode(t.q, lens)
     assert st == 0
-    # the padded prefix rows past each length were written with zeros by the padded chunks: decode reads
-    # only [0, len), so the comparison covers exactly the real tokens
+    # rows past each length hold the chunks' zero padding; the decode reads only [0, len)
     assert_close(out, ref, what=f"paged D{D} Hkv{Hkv} P{P}")
     # one more token per sequence, crossing pages for some
     kn = torch.randn((w.batch, 1, Hkv, D)).to(w.dtype)
