@@ -14,6 +14,10 @@ sides, CUDA events on the launching stream, max over ranks. The packed cache
 flush is needed. ``--gpus N`` (under torchrun) runs N independent replicas: the
 path has no exchange step, so there is no collective on the data path.
 
+The default line also carries ``long_context``: the same step timed on the
+131072-token Llama-3.1-70B-shaped context (64 q / 8 kv heads, query groups of
+8), with its own split-K roofline record (``--no-long-context`` skips it).
+
 ``--impl reference`` times the CPU oracle (plain single-threaded C++) on a
 bounded sample of the same workload on the host cores.
 """
@@ -44,6 +48,8 @@ def parse_args(argv=None):
                     choices=["ragged_serving", "llama31_70b_long", "llama3_8b_layer", "tiny_single_head"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--no-clocks", action="store_true", help="skip nvidia-smi clock sampling")
+    ap.add_argument("--no-long-context", action="store_true",
+                    help="skip the 131072-token long-context sub-record of the default line")
     ap.add_argument("--no-references", action="store_true",
                     help="skip the quantise-throughput, bf16 dense-KV and dequantise-then-attend reference points")
     ap.add_argument("--k-format", choices=list(FORMATS), default="int4",
@@ -776,30 +782,27 @@ def run_reference(args):
     return 0
 
 
-def run_tq(args):
+class StepTiming:
+    """Device state and timings of one workload's step (append one token per sequence + decode)."""
+
+
+def time_device_steps(w, fmt, args, dev, stream, rank, local):
+    """Prefill the workload's cache (untimed), then time K steps of (append, decode).
+
+    The K timed steps are captured once as a CUDA graph and replayed between CUDA
+    events, bracketed by a barrier and a synchronize; a second pass of the same K
+    steps records an event between the split-K and merge kernels for per-kernel
+    durations. Clocks are sampled with nvidia-smi during the graph-timed region.
+    """
     import torch
     from compressed_domain_attention_b200 import synthetic as syn
-    from compressed_domain_attention_b200 import tq
-
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    init_dist("nccl")
-    w = get_workload(args.workload)
+    r = StepTiming()
     if w.n_append == 0:
         w.n_append = 1
     cap = max(w.seq_lens) + w.n_append
     t = syn.generate(w, device="cuda")
-    fmt = args.k_format
-    if args.lam and fmt == "delegated":
-        raise SystemExit("--lambda applies to the int4 and fp16 formats (the delegated tail is binary16)")
-    if args.paged and fmt == "delegated":
-        raise SystemExit("--paged applies to the int4 and fp16 formats")
     cache = DeviceCache(w, cap, fmt, dev, args.lam, args.sparse_v, args.paged)
-    L = cache.L
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream()
-    # prefill (untimed): one append per sequence through a batch-1 view of the cache
     zero = torch.zeros(1, dtype=torch.int32, device=dev)
     for b in range(w.batch):
         cache.append_seq(b, t.k[b][None].contiguous(), t.v[b][None].contiguous(), w.seq_lens[b], zero, status,
@@ -875,8 +878,9 @@ def run_tq(args):
         stop.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
-    clk = clocks.stop() if clocks else None
-    elapsed = start.elapsed_time(stop) / 1e3
+    r.clocks = clocks.stop() if clocks else None
+    r.elapsed = start.elapsed_time(stop) / 1e3
+    del sgraph
     # second timed pass of the same steps with an event between the split-K and
     # merge kernels: per-kernel durations for the roofline. Eager launches: a short
     # GPU spin first lets the host queue the steps ahead of the device, so no host
@@ -885,11 +889,78 @@ def run_tq(args):
     for i in range(args.steps):
         step(i)
     torch.cuda.synchronize()
-    split_ms = [ev_a[i].elapsed_time(ev_s[i]) for i in range(args.steps)]
-    merge_ms = [ev_s[i].elapsed_time(ev_b[i]) for i in range(args.steps)]
+    r.split_ms = [ev_a[i].elapsed_time(ev_s[i]) for i in range(args.steps)]
+    r.merge_ms = [ev_s[i].elapsed_time(ev_b[i]) for i in range(args.steps)]
     st = int(status.item())
     if st != 0:
-        raise RuntimeError(f"device status {st} during the benchmark")
+        raise RuntimeError(f"device status {st} during the benchmark ({w.name})")
+    r.w, r.t, r.cache, r.status = w, t, cache, status
+    r.lens, r.lens1, r.q, r.k_new, r.v_new, r.out = lens, lens1, q, k_new, v_new, out
+    r.step, r.step_mode = step, step_mode
+    r.lens_step = [x + w.n_append for x in w.seq_lens]
+    r.bytes_split = split_bytes(w, r.lens_step, fmt)
+    r.bytes_step = decode_bytes(w, r.lens_step, fmt) + append_bytes(w, 2 if w.dtype != torch.float32 else 4, fmt)
+    return r
+
+
+def traffic_key(w, fmt, paged):
+    return (f"decode_split_kernel/{w.name}" + {"int4": "", "fp16": "/k_fp16", "delegated": "/delegated"}[fmt]
+            + (f"/paged{paged}" if paged else ""))
+
+
+def roofline_record(r, fmt, paged, dev):
+    """Roofline of the split-K kernel: algorithmic bytes per launch / event-timed launch duration."""
+    peak, peak_kind = load_peaks()
+    split_avg = max_over_ranks(statistics.mean(r.split_ms), dev)
+    merge_avg = max_over_ranks(statistics.mean(r.merge_ms), dev)
+    achieved = r.bytes_split / (split_avg / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": "decode_split_kernel", "achieved": round(achieved, 1),
+            "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": load_traffic(traffic_key(r.w, fmt, paged)),
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": r.bytes_split, "avg_launch_ms": round(split_avg, 4),
+            "merge_avg_ms": round(merge_avg, 4)}
+
+
+def long_context_record(args, fmt, dev, stream, rank, local, ws):
+    """The 131072-token Llama-3.1-70B-shaped step (64 q / 8 kv heads), timed like the headline."""
+    from compressed_domain_attention_b200 import synthetic as syn
+    w = syn.llama31_70b_long()
+    r = time_device_steps(w, fmt, args, dev, stream, rank, local)
+    max_t = max_over_ranks(r.elapsed, dev)
+    peak, _ = load_peaks()
+    rec = {"workload": w.name, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+           "kv_tokens_per_seq_step": r.lens_step, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(max_t / args.steps * 1e3, 4),
+           "value": round(ws * r.bytes_step * args.steps / max_t / 1e9, 2), "unit": UNIT,
+           "pct_of_measured_hbm": round(100.0 * r.bytes_step * args.steps / max_t / 1e9 / peak, 2),
+           "pct_of_8tbs": round(100.0 * r.bytes_step * args.steps / max_t / 1e9 / 8000.0, 2),
+           "kv_tokens_per_s": round(ws * sum(r.lens_step) * args.steps / max_t, 1),
+           "algorithmic_bytes_per_step": r.bytes_step,
+           "roofline": roofline_record(r, fmt, args.paged, dev), "step_launch": r.step_mode,
+           "l2": f"inputs larger than L2 (cache {r.cache.nbytes() / 1e9:.2f} GB > 126 MB), no flush"}
+    if r.clocks:
+        rec["clocks"] = r.clocks
+    return rec
+
+
+def run_tq(args):
+    import torch
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    w = get_workload(args.workload)
+    fmt = args.k_format
+    if args.lam and fmt == "delegated":
+        raise SystemExit("--lambda applies to the int4 and fp16 formats (the delegated tail is binary16)")
+    if args.paged and fmt == "delegated":
+        raise SystemExit("--paged applies to the int4 and fp16 formats")
+    stream = torch.cuda.current_stream()
+    r = time_device_steps(w, fmt, args, dev, stream, rank, local)
+    cache, L, status, out, q, k_new, v_new = r.cache, r.cache.L, r.status, r.out, r.q, r.k_new, r.v_new
+    lens, lens1, t, elapsed = r.lens, r.lens1, r.t, r.elapsed
 
     # e2e: host buffers in pinned memory, every step's copies inside the timed region.
     # As a serving loop would run it: a copy stream brings step i+1's inputs in and
@@ -974,49 +1045,36 @@ def run_tq(args):
     e2e_s = e0.elapsed_time(e1) / 1e3
     if not torch.equal(h_out[(args.steps - 1) % 2], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-timed output")
+    del graph
 
     refs = {} if args.no_references else reference_points(w, t, L, cache.kc, cache.ks, cache.vc, cache.vs, lens1,
                                                           q, dev, stream, args, fmt=fmt)
 
-    lens_step = [x + w.n_append for x in w.seq_lens]
-    bytes_decode = decode_bytes(w, lens_step, fmt)
-    bytes_split = split_bytes(w, lens_step, fmt)
-    bytes_step = bytes_decode + append_bytes(w, 2 if w.dtype != torch.float32 else 4, fmt)
+    lens_step = r.lens_step
+    bytes_step = r.bytes_step
     max_t = max_over_ranks(elapsed, dev)
     max_e2e = max_over_ranks(e2e_s, dev)
-    split_avg = max_over_ranks(statistics.mean(split_ms), dev)
-    merge_avg = max_over_ranks(statistics.mean(merge_ms), dev)
-
-    peak, peak_kind = load_peaks()
-    achieved = bytes_split / (split_avg / 1e3) / 1e9
-    traffic = load_traffic(f"decode_split_kernel/{w.name}" + {"int4": "", "fp16": "/k_fp16",
-                                                                "delegated": "/delegated"}[fmt]
-                           + (f"/paged{args.paged}" if args.paged else ""))
+    peak, _ = load_peaks()
     cache_bytes = cache.nbytes()
     extra = {
         "tokens_per_s": round(ws * w.batch * w.n_append * args.steps / max_t, 1),
         "kv_tokens_per_s": round(ws * sum(lens_step) * args.steps / max_t, 1),
         "pct_of_measured_hbm": round(100.0 * bytes_step / max_t * args.steps / 1e9 / peak, 2),
         "pct_of_8tbs": round(100.0 * bytes_step / max_t * args.steps / 1e9 / 8000.0, 2),
-        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": bytes_split, "avg_launch_ms": round(split_avg, 4),
-                     "merge_avg_ms": round(merge_avg, 4)},
+        "roofline": roofline_record(r, fmt, args.paged, dev),
         "e2e": {"value": round(ws * bytes_step * args.steps / max_e2e / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(k_new.numel() * k_new.element_size() * 2 + q.numel() * q.element_size()),
                 "d2h_bytes_per_step": int(out.numel() * out.element_size()),
                 "copies": "pinned host buffers; step i+1's inputs in and step i's output out on a copy "
                           "stream while step i computes (double-buffered, event-ordered)", "launch": e2e_mode},
         "gpu_launches": (4 if fmt == "delegated" else 3) * args.steps,
-        "step_launch": step_mode,
+        "step_launch": r.step_mode,
         "kernel_timing": "split-K/merge durations from a second pass of the same K steps with an event "
                          "between the two kernels (the timed region itself launches the merge as a "
                          "programmatic dependent)",
     }
-    if clk:
-        extra["clocks"] = clk
+    if r.clocks:
+        extra["clocks"] = r.clocks
     extra.update(refs)
     cfg = {"workload": w.name, "global_batch": w.batch * ws, "kv_tokens_per_seq_step": lens_step if w.batch <= 4
            else {"min": min(lens_step), "max": max(lens_step), "sum": sum(lens_step)},
@@ -1029,6 +1087,11 @@ def run_tq(args):
     total_bytes = sum_over_ranks(bytes_step * args.steps, dev)  # every rank takes part
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         extra["cpu_baseline"] = cpu_baseline(w, t, 300000, fmt, args.lam, args.sparse_v)
+    # the long-context workload (131072 tokens, query groups of 8) as a sub-record of the same line
+    if not args.no_long_context and args.workload != "llama31_70b_long":
+        del r, cache, t, h_k, h_v, h_q, h_out, d_k, d_v, d_q, d_out
+        torch.cuda.empty_cache()
+        extra["long_context"] = long_context_record(args, fmt, dev, stream, rank, local, ws)
     if rank == 0:
         line = assemble_line(n_gpus=ws, steps=args.steps, warmup=args.warmup, total_bytes_all_ranks=total_bytes,
                              max_time_s=max_t, workload=cfg, extra=extra)

@@ -152,15 +152,8 @@ void copy_signs(const tq_layout_t* L, uint64_t (&dst)[4]) {
   for (int i = 0; i < 4; ++i) dst[i] = L->sign_bits[i];
 }
 
-// Split-K partial slots (one per CTA plus one per sequence for ranges that
-// straddle sequences) and, for the delegated cache, the hot-tail partials.
 uint64_t workspace_bytes(int batch, int n_q, int D, int max_ctas, int tail_window = 0) {
-  const uint64_t slots =
-      (uint64_t)max_ctas + (uint64_t)batch + (uint64_t)batch * (uint64_t)tqk::tail_chunk_count(tail_window);
-  const uint64_t header = 8ull * (uint64_t)(batch + 2);
-  const uint64_t ml = slots * (uint64_t)n_q * 2ull * 4ull;
-  const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
-  return ((header + ml + 255) / 256) * 256 + acc;
+  return tqk::decode_workspace_bytes(batch, n_q, D, max_ctas, tail_window);
 }
 
 constexpr int kMaxTailWindow = 1024;  // the merge kernel keeps one score per hot token in shared memory
@@ -404,19 +397,20 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
       !aligned16(v_scales) || !aligned16(out) || !aligned16(workspace) || (deleg && !aligned16(v_tail)))
     return TQ_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return TQ_ERR_INVALID_ARG;
-  int sms = 0;
-  r = device_sm_count(&sms);
-  if (r != TQ_OK) return r;
-  int grid = sms;
+  // options: every check here is on the host, before any CUDA call
+  int req_ctas = 0;
   int min_split = 64;  // measured: a 4096-token decode runs 2 us faster over 64-token ranges than 128
   cudaEvent_t ev = nullptr;
   const float* lam_k = nullptr;
   const float* lam_v = nullptr;
   float sparse_lt = -INFINITY;
+  uint64_t wait_ns = 1000000000ull;  // 1 s
   if (opts != nullptr) {
+    if (opts->wait_limit_ns < 0) return TQ_ERR_INVALID_ARG;
+    if (opts->wait_limit_ns > 0) wait_ns = (uint64_t)opts->wait_limit_ns;
     if (opts->max_ctas < 0 || opts->max_ctas > layout->max_ctas || opts->min_split_tokens < 0)
       return TQ_ERR_INVALID_ARG;
-    if (opts->max_ctas > 0) grid = opts->max_ctas;
+    req_ctas = opts->max_ctas;
     if (opts->min_split_tokens > 0) min_split = opts->min_split_tokens;
     ev = reinterpret_cast<cudaEvent_t>(opts->after_split_event);
     lam_k = opts->lambda_k;
@@ -428,6 +422,10 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
     if (!(tau >= 0.f) || !std::isfinite(tau)) return TQ_ERR_INVALID_ARG;
     if (tau > 0.f) sparse_lt = std::log2(tau);
   }
+  int sms = 0;
+  r = device_sm_count(&sms);
+  if (r != TQ_OK) return r;
+  int grid = req_ctas > 0 ? req_ctas : sms;
   if (sparse_lt > -INFINITY && D != 64 && D != 128) return TQ_ERR_UNSUPPORTED;  // sparse-V kernels: D 64, 128
   if (grid > layout->max_ctas) grid = layout->max_ctas;
   const int W = deleg ? layout->tail_window : 0;
@@ -479,6 +477,7 @@ int decode_impl(const tq_layout_t* layout, const void* q, int q_dtype, const int
   p.max_pages = layout->max_pages;
   p.n_pages = layout->n_pages;
   p.len_align = layout->page_tokens > 0 ? tile : 1;
+  p.wait_ns = wait_ns;
   cudaError_t e = tqk::launch_decode(p, km, vm, D, reinterpret_cast<cudaStream_t>(stream), ev);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }

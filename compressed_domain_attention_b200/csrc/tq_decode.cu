@@ -56,7 +56,7 @@ constexpr int kConverterWarps = 3;                  // one on each scheduler wit
 constexpr int kThreads = (kConsumerWarps + 1 + kConverterWarps) * 32;
 constexpr int kMaxBatch = 1024;
 constexpr int kMergeThreads = 128;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every pipeline wait
+constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s bound on the producer's wait for its copies in flight
 
 // KF16: K tiles are binary16 in the original domain (asymmetric cache), the V
 // side is unchanged; no K scales are copied or converted.
@@ -276,9 +276,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(&vmap) : "memory");
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    // The query is read by every block's prologue once the prefix sums are known, by when
+    // the tile copies have started: each block prefetches one slice of it into L2 now.
+    const uint32_t qbytes = (uint32_t)p.batch * (uint32_t)p.n_q * (uint32_t)(D * (p.q_dtype == TQ_F32 ? 4 : 2));
+    const uint32_t per = ((qbytes + gridDim.x - 1) / gridDim.x + 127u) & ~127u;  // whole 128-byte lines
+    const uint32_t o0 = blockIdx.x * per;
+    if (o0 < qbytes) {
+      const uint32_t n = min(per, qbytes - o0);  // a multiple of 16 (rows of D >= 32 elements)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<const uint8_t*>(p.q) + o0),
+                   "r"(n)
+                   : "memory");
+    }
+  }
   block_prefix_lengths(p, prefix, prefix + (p.batch + 1));  // its barriers also publish the set-up
   const int64_t T_sum = prefix[p.batch];
-  int64_t R = (T_sum + p.grid - 1) / p.grid;
+  // T_sum < 2^32 (batch * max_seq <= INT32_MAX, plus at most a tile of padding per
+  // sequence), so the split range takes a 32-bit division
+  int64_t R = (uint32_t)(T_sum + p.grid - 1) / (uint32_t)p.grid;
   if (R < p.min_split) R = p.min_split;
   const int64_t r_align = p.len_align > 16 ? p.len_align : 16;  // whole tiles with paged storage (a power of two)
   R = (R + r_align - 1) & ~(r_align - 1);
@@ -312,7 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; !walk.done(); walk.advance<T_TILE>()) {
       const int stage = issued % STAGES;
       const uint32_t n = (uint32_t)(issued / STAGES);
-      if (!mbar_wait_bounded(&empty[stage], (n & 1u) ^ 1u, kWaitLimitNs)) {
+      if (!mbar_wait_backoff(&empty[stage], (n & 1u) ^ 1u, p.wait_ns)) {
+        dead = true;
+        break;
+      }
+      // The copies of the tile that last used this stage have landed: a warp that gave up
+      // on a wait arrives on `empty` without reading, so `empty` alone does not show it,
+      // and `full` must never be re-armed while a phase of it is still waiting for bytes.
+      if (n > 0 && !mbar_wait_bounded(&full[stage], (n - 1u) & 1u, kDrainLimitNs)) {
         dead = true;
         break;
       }
@@ -340,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       misc[0] = 1;
       status_or(p.status, TQ_STATUS_TIMEOUT);
     }
-    // drain: no copy may still be in flight when this thread exits
+    // drain: no copy may still be in flight when this thread exits (each stage holds at
+    // most one tile's copies, those of the last STAGES tiles issued)
     for (int k = max(0, issued - STAGES); k < issued; ++k)
-      (void)mbar_wait_bounded(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), kWaitLimitNs);
+      (void)mbar_wait_bounded(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), kDrainLimitNs);
     return;
   }
 
@@ -387,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = tile_i % STAGES;
       const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
       // (a producer that gave up issues nothing more: these waits then run out)
-      if (!dead && !mbar_wait_bounded(&full[stage], par, kWaitLimitNs)) {
+      if (!dead && !mbar_wait_backoff(&full[stage], par, p.wait_ns)) {
         dead = true;
         if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
       }
@@ -398,29 +421,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int soff = (int)((row0 * C::SROW) & 15);
         const int nv = min(T_TILE, walk.seg_hi - walk.t0);
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
+        const bool part_tile = nv < T_TILE;  // the same for every lane: tokens past nv get 0
 #pragma unroll
         for (int kv = KF16 ? 1 : 0; kv < 2; ++kv) {  // binary16 K has no scales
-          // plain (not volatile) shared loads: the compiler may issue a lane's loads together
-          const uint16_t* raw =
-              reinterpret_cast<const uint16_t*>(sb + (kv ? C::OFF_RAWV : C::OFF_RAW) + soff);
+          // the NG scales of a (token, head) are NG x 2 contiguous bytes: one vector load each
+          // for the item's two tokens (plain shared loads, which the compiler may batch)
+          const uint8_t* raw = sb + (kv ? C::OFF_RAWV : C::OFF_RAW) + soff;
           const uint32_t dst = kv ? smem_u32(sb + C::OFF_SCV) : sc;
 #pragma unroll
           for (int k = 0; k < ITEMS; ++k) {
             const int t = tok_of[k];
             if (t >= T_TILE) continue;
-            const bool ok0 = t < nv, ok1 = t + 1 < nv;
+            float f0[NG], f1[NG];
+            load_scales<NG>(f0, raw + src_off[k]);
+            load_scales<NG>(f1, raw + src_off[k] + HKV * NG * 2);
+            if (part_tile) {
+              const bool ok0 = t < nv, ok1 = t + 1 < nv;
+#pragma unroll
+              for (int g = 0; g < NG; ++g) {
+                f0[g] = ok0 ? f0[g] : 0.f;
+                f1[g] = ok1 ? f1[g] : 0.f;
+              }
+            }
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
-              const uint32_t h0 = raw[src_off[k] / 2 + g];
-              const uint32_t h1 = raw[src_off[k] / 2 + HKV * NG + g];
-              const float f0 = ok0 ? __half2float(__ushort_as_half((unsigned short)h0)) : 0.f;
-              const float f1 = ok1 ? __half2float(__ushort_as_half((unsigned short)h1)) : 0.f;
               if (TOK_M && kv == 0) {
                 const uint32_t a = dst + dstk_off[k] + 4 * (g * 8 * 2 * MT);
-                sts_f32(a, f0);
-                sts_f32(a + 4 * 2 * MT, f1);
+                sts_f32(a, f0[g]);
+                sts_f32(a + 4 * 2 * MT, f1[g]);
               } else {
-                sts_f2(dst + dst_off[k] + 4 * (g * 4 * 2 * NT), f0, f1);
+                sts_f2(dst + dst_off[k] + 4 * (g * 4 * 2 * NT), f0[g], f1[g]);
               }
             }
           }
@@ -659,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The converters arrive on `ready` only after they observed `full` complete, so
       // its completion (release by the converters, acquire here) also orders this
       // warp's reads after the stage's tensor copies.
-      if (!dead && !mbar_wait_bounded(&ready[stage], par, kWaitLimitNs)) {
+      if (!dead && !mbar_wait_bounded(&ready[stage], par, p.wait_ns)) {
         dead = true;
         if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
       }
@@ -871,8 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const float2 sk = make_float2(skv[gi][2 * nt], skv[gi][2 * nt + 1]);
                   float c[4];
                   const uint32_t w = kw[i];
-                  mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u), and_xor(w, 0x00F000F0u, 0x00800080u),
-                                  0.f, 0.f, 0.f, 0.f);
+                  mma_f16_16816_c(c, qA[g][0], and_xor(w, 0x000F000Fu, 0x00080008u),
+                                  and_xor(w, 0x00F000F0u, 0x00800080u), 0.f, 0.f, 0.f, 0.f);
                   const uint32_t w8 = w >> 8;
                   mma_f16_16816_acc(c, qA[g][1], and_xor(w8, 0x000F000Fu, 0x00080008u),
                                     and_xor(w8, 0x00F000F0u, 0x00800080u));

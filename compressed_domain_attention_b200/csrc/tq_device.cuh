@@ -208,13 +208,62 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Wait for the phase with the given parity to complete, giving up after
-// `limit_ns` nanoseconds of wall time. Returns false on timeout.
+// `limit_ns` nanoseconds of wall time. Returns false on timeout. Each suspended
+// try lasts at most min(limit, 20 us), so a bound shorter than a typical wait
+// does run out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint32_t hint = limit_ns < 20000u ? (uint32_t)limit_ns : 20000u;
   while (true) {
-    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (mbar_try_wait_hint(bar, parity, hint)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// As mbar_wait_bounded, for warps that wait most of the time (the copy issuer and
+// the scale converters): after a failed test the warp sleeps, 32 ns doubling up to
+// 256 ns, so that its polling takes few issue slots from the math warps that share
+// its scheduler.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    if (ns < 256) ns <<= 1;
+  }
+}
+
+// NG consecutive binary16 values at a shared-memory address aligned to 2 NG bytes
+// (NG in {1, 2, 4, 8}), widened to binary32 (exact).
+template <int NG>
+__device__ __forceinline__ void load_scales(float (&f)[NG], const uint8_t* p) {
+  if constexpr (NG == 1) {
+    f[0] = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
+  } else {
+    uint32_t w[NG / 2];
+    if constexpr (NG == 2) {
+      w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if constexpr (NG == 4) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      w[0] = v.x;
+      w[1] = v.y;
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(p);
+      w[0] = v.x;
+      w[1] = v.y;
+      w[2] = v.z;
+      w[3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < NG / 2; ++i) {
+      const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
   }
 }
 

@@ -80,6 +80,7 @@ struct DecodeParams {
   const int32_t* block_table;
   int page_tokens, max_pages, n_pages;
   int len_align;
+  uint64_t wait_ns;  // bound on each pipeline wait of the split-K kernel (its copy drain always uses 1 s)
 };
 
 // Hot-tail partials per sequence of the delegated cache (64 tokens each).
@@ -90,6 +91,21 @@ __host__ __device__ __forceinline__ int64_t cold_tokens(int64_t len, int W, int 
   if (W <= 0) return len;
   if (len <= W) return 0;
   return (len - W + F - 1) / F * F;
+}
+
+// Decode workspace for a split-K grid of `grid` CTAs: an int64 header (prefix sums of
+// the lengths and the per-CTA token range), then (running max, running sum) and a
+// D-float accumulator per (slot, q head). Slots: one per CTA plus one per sequence
+// (a CTA range and a sequence range intersect at most once for each pair, and the
+// slot index sequence + CTA cannot repeat between intersecting pairs), plus the
+// delegated cache's hot-tail partials.
+__host__ __forceinline__ uint64_t decode_workspace_bytes(int batch, int n_q, int D, int grid, int tail_window) {
+  const uint64_t slots =
+      (uint64_t)grid + (uint64_t)batch + (uint64_t)batch * (uint64_t)tail_chunk_count(tail_window);
+  const uint64_t header = 8ull * (uint64_t)(batch + 2);
+  const uint64_t ml = slots * (uint64_t)n_q * 2ull * 4ull;
+  const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
+  return ((header + ml + 255) / 256) * 256 + acc;
 }
 
 cudaError_t launch_quantize(const QuantizeParams& p, int head_dim, cudaStream_t s);

@@ -13,14 +13,16 @@
 // library holds TQ_NOALLOC_WORKSPACE_BYTES of device memory for it until the
 // process exits. Host code cannot use the array's name as a device address
 // (in host code it names a host-side stand-in), so the first call on each
-// device looks up the real address with cudaGetSymbolAddress while that device
-// is current, and caches it.
+// device (and in each new context of it) looks up the real address with
+// cudaGetSymbolAddress while that device is current, and caches it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/tq.h"
+#include "tq_kernels.h"
 
 namespace {
 
@@ -31,10 +33,44 @@ static __device__ __align__(256) unsigned char g_noalloc_ws[TQ_NOALLOC_WORKSPACE
 
 constexpr int kMaxDevices = 64;
 
-// Per-device address of g_noalloc_ws, set up once per device on first use.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read). A
+// device's context can be destroyed and made again (cudaDeviceReset, or a caller
+// that switches contexts); the array then has a new device address, so the
+// cached address is keyed on this id as well as on the device ordinal.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_ws for the current device and context, looked up
+// (cudaGetSymbolAddress, with that device current) on the first call in each
+// context and cached. The runtime makes the device's context current if it is
+// not yet, so the id is read after the lookup.
 void* ws_address_for_current_device(int* err) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {nullptr};
+  static unsigned long long ctx_of[kMaxDevices] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -46,7 +82,8 @@ void* ws_address_for_current_device(int* err) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_ws);  // with `dev` current
     if (e != cudaSuccess || p == nullptr) {
@@ -54,22 +91,9 @@ void* ws_address_for_current_device(int* err) {
       return nullptr;
     }
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();
   }
   return addr[dev];
-}
-
-// Workspace the decode call needs for a split-K grid of `grid` CTAs: an int64
-// header (prefix sums of the lengths and the per-CTA token range), then
-// (running max, running sum) and a D-float accumulator per (slot, q head),
-// slots = grid + batch. This is the arithmetic of the documented workspace
-// layout; if it ever under-counted, the decode call itself would reject the
-// workspace size with TQ_ERR_INVALID_ARG rather than overrun it.
-uint64_t needed_bytes(int batch, int n_q, int D, int grid) {
-  const uint64_t slots = (uint64_t)grid + (uint64_t)batch;
-  const uint64_t header = 8ull * (uint64_t)(batch + 2);
-  const uint64_t ml = slots * (uint64_t)n_q * 8ull;
-  const uint64_t acc = slots * (uint64_t)n_q * (uint64_t)D * 4ull;
-  return ((header + ml + 255) / 256) * 256 + acc;
 }
 
 }  // namespace
@@ -89,8 +113,10 @@ extern "C" int tq_decode_attention_noalloc(const tq_layout_t* layout, const void
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   if (sms > layout->max_ctas) sms = layout->max_ctas;
-  // Reject requests whose workspace would not fit, before touching the device.
-  if (needed_bytes(layout->batch, layout->n_q_heads, layout->head_dim, sms) > (uint64_t)TQ_NOALLOC_WORKSPACE_BYTES)
+  // Reject requests whose workspace would not fit, before touching the device (the
+  // same workspace arithmetic the decode call checks its workspace size against).
+  if (tqk::decode_workspace_bytes(layout->batch, layout->n_q_heads, layout->head_dim, sms, 0) >
+      (uint64_t)TQ_NOALLOC_WORKSPACE_BYTES)
     return TQ_ERR_CAPACITY;
   int err = 0;
   void* ws = ws_address_for_current_device(&err);

@@ -59,7 +59,8 @@ class TqLayout(ctypes.Structure):
 class TqDecodeOpts(ctypes.Structure):
     _fields_ = [("min_split_tokens", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
                 ("after_split_event", ctypes.c_void_p), ("lambda_k", ctypes.c_void_p),
-                ("lambda_v", ctypes.c_void_p), ("sparse_v_threshold", ctypes.c_float)]
+                ("lambda_v", ctypes.c_void_p), ("sparse_v_threshold", ctypes.c_float),
+                ("wait_limit_ns", ctypes.c_int64)]
 
 
 class TqAppendOpts(ctypes.Structure):
@@ -268,16 +269,16 @@ def tq_append_delegated(layout, k, v, n_new, start_pos, k_f16, v_codes, v_scales
 
 
 def _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k=None, lambda_v=None,
-                 sparse_v_threshold=0.0):
+                 sparse_v_threshold=0.0, wait_limit_ns=0):
     """TqDecodeOpts for the given knobs, or None when all are at their defaults."""
     if not (min_split_tokens or max_ctas or after_split_event is not None or lambda_k is not None
-            or lambda_v is not None or sparse_v_threshold):
+            or lambda_v is not None or sparse_v_threshold or wait_limit_ns):
         return None
     for t in (lambda_k, lambda_v):
         assert t is None or t.is_contiguous()
     ev = ctypes.c_void_p(after_split_event.cuda_event) if after_split_event is not None else None
     return TqDecodeOpts(int(min_split_tokens), int(max_ctas), ev, _ptr(lambda_k), _ptr(lambda_v),
-                        float(sparse_v_threshold))
+                        float(sparse_v_threshold), int(wait_limit_ns))
 
 
 def tq_decode_attention_delegated(layout, q, seq_lens, k_f16, v_codes, v_scales, v_tail, sm_scale, out, workspace,
@@ -297,17 +298,19 @@ def tq_decode_attention_delegated(layout, q, seq_lens, k_f16, v_codes, v_scales,
 
 def tq_decode_attention(layout, q, seq_lens, k_codes, k_scales, v_codes, v_scales, sm_scale, out, workspace,
                         status=None, stream=None, min_split_tokens=0, max_ctas=0, after_split_event=None,
-                        lambda_k=None, lambda_v=None, sparse_v_threshold=0.0):
+                        lambda_k=None, lambda_v=None, sparse_v_threshold=0.0, wait_limit_ns=0):
     """q: [batch][Hq][D]; out: float32 [batch][Hq][D]; workspace: >= layout.decode_workspace_bytes bytes.
 
     lambda_k / lambda_v: the per-channel lambda the cache was written with; sparse_v_threshold: the
-    sparse-V rule's threshold (0 = exact). Any of these selects tq_decode_attention_ex.
+    sparse-V rule's threshold (0 = exact); wait_limit_ns: bound on each pipeline wait of the split-K
+    kernel (0 = one second). Any of these selects tq_decode_attention_ex.
     """
     for t in (q, seq_lens, k_codes, k_scales, v_codes, v_scales, out, workspace):
         assert t is None or t.is_contiguous()
     ws_bytes = workspace.numel() * workspace.element_size()
     lib = _lib()
-    opts = _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k, lambda_v, sparse_v_threshold)
+    opts = _decode_opts(min_split_tokens, max_ctas, after_split_event, lambda_k, lambda_v, sparse_v_threshold,
+                        wait_limit_ns)
     if opts is not None:
         code = lib.tq_decode_attention_ex(ctypes.byref(layout), _ptr(q), _dtype_code(q), _ptr(seq_lens),
                                           _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),

@@ -138,6 +138,15 @@ typedef struct {
    * 16-32 tokens whose weights all fall below skips its V decode and MMAs.
    * Head dims 64 and 128 (otherwise TQ_ERR_UNSUPPORTED). */
   float sparse_v_threshold;
+  /* Bound on every pipeline wait of the split-K kernel (a warp waiting for a
+   * tile's copies, its converted scales, or a free stage), in nanoseconds of
+   * the GPU's global timer: 0 = the default of one second; negative is
+   * TQ_ERR_INVALID_ARG. A wait that runs out sets TQ_STATUS_TIMEOUT, the warp
+   * stops reading tiles (its partials are then incomplete) and the call still
+   * returns; the copy engine's copies already in flight are always waited for
+   * (with the default bound) before a block exits. A short bound is a way to
+   * exercise that path; no real input needs anything but the default. */
+  int64_t wait_limit_ns;
 } tq_decode_opts_t;
 
 /* Optional knobs for tq_quantize_append_ex (NULL = defaults). */
@@ -334,8 +343,11 @@ int tq_decode_attention_ex(const tq_layout_t* layout, const void* q, int q_dtype
  * tq_decode_attention with the default one-CTA-per-SM split.
  *
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make that
- *    first call before any stream capture on that device.
+ *    (cudaGetSymbolAddress, with that device current) and caches it, keyed on
+ *    the device and on the unique id of the current context; make that first
+ *    call before any stream capture on that device. After cudaDeviceReset (or
+ *    in another context) the next call looks the address up again, so that
+ *    call too should come before any capture.
  *  - A request whose workspace would exceed TQ_NOALLOC_WORKSPACE_BYTES
  *    (roughly (SMs + batch) * n_q_heads * (head_dim + 2) * 4 bytes) returns
  *    TQ_ERR_CAPACITY and launches nothing.

@@ -1,5 +1,8 @@
 """Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
 and the CPU oracle on the same seeded inputs, and compare."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -10,7 +13,46 @@ ATOL = 2e-3     # decode tolerance: max-abs error vs the oracle's fp32 result
 RTOL_L2 = 1e-3  # and relative L2 error
 
 
+def parallel_map(fn, items):
+    """fn(item) for every item on a host thread pool. The oracle is reached through ctypes,
+    whose foreign calls release the interpreter lock, so independent sequences or heads
+    run on separate cores; each call is the unchanged single-threaded oracle."""
+    items = list(items)
+    n = max(1, min(len(items), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        return list(ex.map(fn, items))
+
+
+def oracle_decode_all(decode_fn, batch, n_q, heads_per_task=None):
+    """Every (sequence, q head) of an oracle decode, split into independent tasks.
+
+    decode_fn(which) -> (out [B][Hq][D], status) computes the rows selected by the
+    uint8 mask which [B][Hq]; tasks are whole sequences (or groups of heads of one
+    sequence when heads_per_task is given) and their rows are gathered into one
+    output. Returns (out, OR of the statuses)."""
+    hp = heads_per_task or n_q
+    tasks = [(b, h0) for b in range(batch) for h0 in range(0, n_q, hp)]
+
+    def one(task):
+        b, h0 = task
+        which = np.zeros((batch, n_q), np.uint8)
+        which[b, h0:h0 + hp] = 1
+        out, st = decode_fn(which)
+        return task, out[b, h0:h0 + hp].copy(), st
+
+    full = None
+    status = 0
+    for (b, h0), rows, st in parallel_map(one, tasks):
+        if full is None:
+            full = np.zeros((batch, n_q, rows.shape[-1]), np.float32)
+        full[b, h0:h0 + hp] = rows
+        status |= st
+    return full, status
+
+
 def np_f32(t):
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t, np.float32)
     return t.detach().to("cpu", torch.float32).contiguous().numpy()
 
 
@@ -88,6 +130,17 @@ class OracleCache:
                                         self.ks[b:b + 1], self.vc[b:b + 1], self.vs[b:b + 1])
         assert st == 0
 
+    def append_seqs(self, t, seqs):
+        """Prefill the listed sequences of tensors t (each at position 0) on a thread pool."""
+        parallel_map(lambda b: self.append_seq(b, t.k[b], t.v[b], 0), [b for b in seqs if t.k[b] is not None
+                                                                         and t.k[b].shape[0] > 0])
+
+    def decode_all(self, q, seq_lens, sm_scale, heads_per_task=None):
+        """Every (sequence, head) of the decode, on a thread pool. -> (out, status)."""
+        qn = np_f32(q)
+        return oracle_decode_all(lambda which: self.decode(qn, seq_lens, sm_scale, which), qn.shape[0],
+                                 qn.shape[1], heads_per_task)
+
     def decode(self, q, seq_lens, sm_scale, which=None):
         lens = np.asarray(seq_lens, np.int32)
         if self.kf16:
@@ -161,6 +214,11 @@ class DelegatedOracleCache:
                                      self.window, self.fold, self.k16[b:b + 1], self.vc[b:b + 1],
                                      self.vs[b:b + 1], self.tail[b:b + 1])
         assert st == 0
+
+    def decode_all(self, q, seq_lens, sm_scale, heads_per_task=None):
+        qn = np_f32(q)
+        return oracle_decode_all(lambda which: self.decode(qn, seq_lens, sm_scale, which), qn.shape[0],
+                                 qn.shape[1], heads_per_task)
 
     def decode(self, q, seq_lens, sm_scale, which=None):
         return oracle.decode_attention_delegated(self.signs, np_f32(q), np.asarray(seq_lens, np.int32), self.k16,

@@ -240,3 +240,39 @@ def test_layout_paged_sizes_and_checks():
                                   None) == tq.TQ_ERR_INVALID_ARG
     assert lib.tq_decode_attention(ctypes.byref(L), fake, 0, fake, fake, fake, fake, fake, ctypes.c_float(0.1),
                                    fake, fake, 1 << 30, None, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_decode_options_checked_before_device_work(lib):
+    # a negative wait bound is refused on the host, before any CUDA call (this runs without a GPU)
+    L = tq.tq_cache_layout(1, 64, 1, 4, 128)
+    fake = ctypes.c_void_p(1 << 20)
+    opts = tq.TqDecodeOpts(0, 0, None, None, None, 0.0, -5)
+    assert lib.tq_decode_attention_ex(ctypes.byref(L), fake, tq.TQ_BF16, fake, fake, fake, fake, fake,
+                                      ctypes.c_float(0.1), fake, fake, 1 << 30, None, ctypes.byref(opts),
+                                      None) == tq.TQ_ERR_INVALID_ARG
+    opts = tq.TqDecodeOpts(0, 0, None, None, None, -1.0, 0)
+    assert lib.tq_decode_attention_ex(ctypes.byref(L), fake, tq.TQ_BF16, fake, fake, fake, fake, fake,
+                                      ctypes.c_float(0.1), fake, fake, 1 << 30, None, ctypes.byref(opts),
+                                      None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_noalloc_refuses_paged_and_delegated_layouts_before_device_work(lib):
+    # the no-alloc entry point has no block-table or hot-tail argument: both layouts are refused
+    # before it looks at the device (this runs without a GPU)
+    fake = ctypes.c_void_p(1 << 20)
+    for L in (tq.tq_cache_layout_paged(2, 256, 8, 32, 128, tq.TQ_K_INT4, 64, 8),
+              tq.tq_cache_layout_paged(2, 256, 8, 32, 128, tq.TQ_K_FP16, 64, 8),
+              tq.tq_cache_layout_delegated(2, 256, 8, 32, 128, 64, 16)):
+        assert lib.tq_decode_attention_noalloc(ctypes.byref(L), fake, tq.TQ_BF16, fake, fake, fake, fake, fake,
+                                               ctypes.c_float(0.1), fake, None, None) == tq.TQ_ERR_INVALID_ARG
+    assert lib.tq_decode_attention_noalloc(None, fake, tq.TQ_BF16, fake, fake, fake, fake, fake,
+                                           ctypes.c_float(0.1), fake, None, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_decode_options_struct_matches_the_header():
+    # field order and types of tq_decode_opts_t as the header declares them
+    text = open(os.path.join(ROOT, "include", "tq.h")).read()
+    body = text[text.index("typedef struct {", text.index("Optional knobs for tq_decode_attention_ex")):
+                text.index("} tq_decode_opts_t;")]
+    fields = re.findall(r"^\s*(?:const\s+)?(int32_t|void\*|float\*|float|int64_t)\s+(\w+);", body, re.M)
+    assert [f for _, f in fields] == [f for f, _ in tq.TqDecodeOpts._fields_]

@@ -17,37 +17,34 @@ import torch
 from compressed_domain_attention_b200 import synthetic as syn
 from compressed_domain_attention_b200 import tq
 from tests.parity_utils import (DelegatedGpuCache, DelegatedOracleCache, assert_close,
-                                assert_delegated_caches_equal)
+                                assert_delegated_caches_equal, parallel_map)
 
 pytestmark = pytest.mark.gpu
 
 
-def build(w, W, F, seqs=None, extra=0):
+def build(w, W, F, extra=0):
     t = syn.generate(w)
     cap = w.capacity + extra
     gpu = DelegatedGpuCache(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, W, F)
     orc = DelegatedOracleCache(w.batch, cap, w.n_kv_heads, w.head_dim, W, F)
-    seqs = list(range(w.batch)) if seqs is None else list(seqs)
+    seqs = list(range(w.batch))
     for b in range(w.batch):
         if w.seq_lens[b]:
             gpu.append_seq(b, t.k[b].cuda(), t.v[b].cuda(), 0)
-    for b in seqs:
-        if w.seq_lens[b]:
-            orc.append_seq(b, t.k[b], t.v[b], 0)
+    parallel_map(lambda b: orc.append_seq(b, t.k[b], t.v[b], 0), [b for b in seqs if w.seq_lens[b]])
     torch.cuda.synchronize()
     return t, gpu, orc, seqs
 
 
-def check_decode(w, q, gpu, orc, seqs, lens, what, **opts):
+def check_decode(w, q, gpu, orc, lens, what, **opts):
+    """Every sequence and every q head against the oracle."""
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu.decode(q.cuda(), lens, w.scale, status, **opts)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    which = np.zeros((w.batch, w.n_q_heads), np.uint8)
-    which[seqs] = 1
-    ref, st = orc.decode(q, lens, w.scale, which)
+    ref, st = orc.decode_all(q, lens, w.scale, w.group if w.batch == 1 else None)
     assert st == 0
-    return assert_close(out.cpu().numpy()[seqs], ref[seqs], what=what)
+    return assert_close(out.cpu().numpy(), ref, what=what)
 
 
 @pytest.mark.parametrize("D,Hkv,Hq,W,F", [(128, 8, 32, 16, 4), (128, 8, 64, 16, 16), (128, 1, 4, 64, 16),
@@ -59,7 +56,7 @@ def test_delegated_prefill_and_decode_shapes(D, Hkv, Hq, W, F):
     w = syn.Workload(f"deleg_d{D}_kv{Hkv}_q{Hq}_w{W}_f{F}", len(lens), Hq, Hkv, D, lens, torch.bfloat16, 21)
     t, gpu, orc, seqs = build(w, W, F)
     assert_delegated_caches_equal(gpu, orc, seqs, w.seq_lens)
-    check_decode(w, t.q, gpu, orc, seqs, w.seq_lens, f"delegated D{D} Hkv{Hkv} Hq{Hq} W{W} F{F}")
+    check_decode(w, t.q, gpu, orc, w.seq_lens, f"delegated D{D} Hkv{Hkv} Hq{Hq} W{W} F{F}")
 
 
 def test_delegated_single_token_steps_cross_fold_boundaries():
@@ -81,7 +78,7 @@ def test_delegated_single_token_steps_cross_fold_boundaries():
             torch.cuda.synchronize()
             assert_delegated_caches_equal(gpu, orc, seqs, cur)
             q = torch.randn((w.batch, 32, 128), generator=g).to(torch.float16)
-            check_decode(w, q, gpu, orc, seqs, cur, f"delegated step {i}")
+            check_decode(w, q, gpu, orc, cur, f"delegated step {i}")
 
 
 @pytest.mark.parametrize("chunks", [[3, 17, 1, 40, 2], [64, 1, 1, 33]])
@@ -103,15 +100,14 @@ def test_delegated_multi_token_appends(chunks):
         torch.cuda.synchronize()
         assert_delegated_caches_equal(gpu, orc, seqs, cur)
     q = torch.randn((w.batch, 8, 64), generator=g)
-    check_decode(w, q, gpu, orc, seqs, cur, "delegated chunks")
+    check_decode(w, q, gpu, orc, cur, "delegated chunks")
 
 
-def test_delegated_ragged_serving_sampled():
+def test_delegated_ragged_serving_all_sequences():
     w = syn.ragged_serving()
-    seqs = [0, 5, 17, 31]
-    t, gpu, orc, seqs = build(w, syn.DELEGATED_WINDOW, syn.DELEGATED_FOLD, seqs)
+    t, gpu, orc, seqs = build(w, syn.DELEGATED_WINDOW, syn.DELEGATED_FOLD)
     assert_delegated_caches_equal(gpu, orc, seqs, w.seq_lens)
-    check_decode(w, t.q, gpu, orc, seqs, w.seq_lens, "delegated ragged serving")
+    check_decode(w, t.q, gpu, orc, w.seq_lens, "delegated ragged serving")
     # the bench's step: one appended token per sequence, then the decode
     cur = list(w.seq_lens)
     gpu.append_all(t.k_new.cuda(), t.v_new.cuda(), cur)
@@ -120,10 +116,10 @@ def test_delegated_ragged_serving_sampled():
     cur = [x + 1 for x in cur]
     torch.cuda.synchronize()
     assert_delegated_caches_equal(gpu, orc, seqs, cur)
-    check_decode(w, t.q, gpu, orc, seqs, cur, "delegated ragged serving step")
+    check_decode(w, t.q, gpu, orc, cur, "delegated ragged serving step")
 
 
-def test_delegated_long_context_sampled_heads():
+def test_delegated_long_context_all_heads():
     w = syn.llama31_70b_long()
     W, F = syn.DELEGATED_WINDOW, syn.DELEGATED_FOLD
     t = syn.generate(w)
@@ -136,12 +132,9 @@ def test_delegated_long_context_sampled_heads():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu.decode(t.q.cuda(), w.seq_lens, w.scale, status).cpu().numpy()
     assert int(status.item()) == 0
-    which = np.zeros((1, w.n_q_heads), np.uint8)
-    heads = [0, 7, 8, 33, 63]
-    which[0, heads] = 1
-    ref, st = orc.decode(t.q, w.seq_lens, w.scale, which)
+    ref, st = orc.decode_all(t.q, w.seq_lens, w.scale, w.group)
     assert st == 0
-    assert_close(out[0, heads], ref[0, heads], what="delegated 131072-token context")
+    assert_close(out, ref, what="delegated 131072-token context")
 
 
 def test_delegated_split_options_agree():

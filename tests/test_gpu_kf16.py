@@ -9,7 +9,7 @@ oracle's asymmetric functions on the same seeded inputs:
 
 Shapes cover both score layouts (query groups of <= 4 heads and of 8), every
 head_dim the format supports, ragged lengths with tile and unit edges, and the
-131072-token long-context shape (sampled heads).
+131072-token long-context shape (every head of every sequence).
 """
 import numpy as np
 import pytest
@@ -22,18 +22,16 @@ from tests.parity_utils import GpuCache, OracleCache, assert_close
 pytestmark = pytest.mark.gpu
 
 
-def build(w, seqs=None):
+def build(w):
     t = syn.generate(w)
     cap = w.capacity
     gpu = GpuCache(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim, k_format=tq.TQ_K_FP16)
     orc = OracleCache(w.batch, cap, w.n_kv_heads, w.head_dim, kf16=True)
-    seqs = list(range(w.batch)) if seqs is None else list(seqs)
+    seqs = list(range(w.batch))
     for b in range(w.batch):
         if w.seq_lens[b]:
             gpu.append_seq(b, t.k[b].cuda(), t.v[b].cuda(), 0)
-    for b in seqs:
-        if w.seq_lens[b]:
-            orc.append_seq(b, t.k[b], t.v[b], 0)
+    orc.append_seqs(t, [b for b in seqs if w.seq_lens[b]])
     torch.cuda.synchronize()
     return t, gpu, orc, seqs
 
@@ -47,17 +45,15 @@ def check_caches(gpu, orc, seqs, lens):
         assert np.array_equal(vs[b, :n], orc.vs[b, :n]), f"V scales differ in sequence {b}"
 
 
-def check_decode(w, t, gpu, orc, seqs, what):
+def check_decode(w, t, gpu, orc, what):
+    """Every sequence and every q head against the oracle."""
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu.decode(t.q.cuda(), w.seq_lens, w.scale, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    which = np.zeros((w.batch, w.n_q_heads), np.uint8)
-    which[seqs] = 1
-    ref, st = orc.decode(t.q, w.seq_lens, w.scale, which)
+    ref, st = orc.decode_all(t.q, w.seq_lens, w.scale, w.group if w.batch == 1 else None)
     assert st == 0
-    got = out.cpu().numpy()
-    return assert_close(got[seqs], ref[seqs], what=what)
+    return assert_close(out.cpu().numpy(), ref, what=what)
 
 
 @pytest.mark.parametrize("D,Hkv,Hq", [(128, 8, 32), (128, 8, 64), (128, 1, 4), (128, 2, 16), (64, 2, 8),
@@ -67,19 +63,18 @@ def test_kf16_append_and_decode_shapes(D, Hkv, Hq):
     w = syn.Workload(f"kf16_d{D}_kv{Hkv}_q{Hq}", len(lens), Hq, Hkv, D, lens, torch.bfloat16, 11)
     t, gpu, orc, seqs = build(w)
     check_caches(gpu, orc, seqs, w.seq_lens)
-    check_decode(w, t, gpu, orc, seqs, f"kf16 D{D} Hkv{Hkv} Hq{Hq}")
+    check_decode(w, t, gpu, orc, f"kf16 D{D} Hkv{Hkv} Hq{Hq}")
 
 
 @pytest.mark.parametrize("name", ["llama3_8b_layer", "ragged_serving"])
 def test_kf16_workload_shapes(name):
     w = {"llama3_8b_layer": syn.llama3_8b_layer, "ragged_serving": syn.ragged_serving}[name]()
-    seqs = None if w.batch == 1 else [0, 5, 17, 31]
-    t, gpu, orc, seqs = build(w, seqs)
+    t, gpu, orc, seqs = build(w)
     check_caches(gpu, orc, seqs, w.seq_lens)
-    check_decode(w, t, gpu, orc, seqs, f"kf16 {w.name}")
+    check_decode(w, t, gpu, orc, f"kf16 {w.name}")
 
 
-def test_kf16_long_context_sampled_heads():
+def test_kf16_long_context_all_heads():
     w = syn.llama31_70b_long()
     t = syn.generate(w)
     gpu = GpuCache(1, w.capacity, w.n_kv_heads, w.n_q_heads, w.head_dim, k_format=tq.TQ_K_FP16)
@@ -92,12 +87,9 @@ def test_kf16_long_context_sampled_heads():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu.decode(t.q.cuda(), w.seq_lens, w.scale, status).cpu().numpy()
     assert int(status.item()) == 0
-    which = np.zeros((1, w.n_q_heads), np.uint8)
-    heads = [0, 7, 8, 33, 63]
-    which[0, heads] = 1
-    ref, st = orc.decode(t.q, w.seq_lens, w.scale, which)
+    ref, st = orc.decode_all(t.q, w.seq_lens, w.scale, w.group)
     assert st == 0
-    assert_close(out[0, heads], ref[0, heads], what="kf16 131072-token context")
+    assert_close(out, ref, what="kf16 131072-token context")
 
 
 def test_kf16_split_invariance_and_append_then_decode():

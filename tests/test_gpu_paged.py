@@ -14,7 +14,7 @@ import torch
 import oracle
 from compressed_domain_attention_b200 import synthetic as syn
 from compressed_domain_attention_b200 import tq
-from tests.parity_utils import assert_close, np_f32
+from tests.parity_utils import assert_close, np_f32, oracle_decode_all, parallel_map
 
 pytestmark = pytest.mark.gpu
 
@@ -117,28 +117,36 @@ def test_paged_append_and_decode(D, Hkv, Hq, k_format, P):
 
 
 @pytest.mark.parametrize("k_format", [tq.TQ_K_INT4, tq.TQ_K_FP16])
-def test_paged_ragged_serving_sampled(k_format):
+def test_paged_ragged_serving_all_sequences(k_format):
+    # all 32 sequences of the serving workload, 64-token pages scattered over the pool
     w = syn.ragged_serving()
-    seqs = [0, 9, 31]
-    t = syn.generate(w, seq_subset=seqs)
-    lens = [w.seq_lens[b] if b in seqs else 0 for b in range(w.batch)]
+    t = syn.generate(w)
+    lens = list(w.seq_lens)
     pair = PagedPair(w, k_format, 64, seed=3)
-    for b in seqs:  # prefill sequence by sequence: a one-sequence layout over the same pools, table row b
-        kb, vb = t.k[b][None], t.v[b][None]
-        L1 = tq.tq_cache_layout_paged(1, pair.cap, w.n_kv_heads, w.n_q_heads, w.head_dim, k_format, 64,
-                                      pair.L.n_pages)
-        tq.tq_quantize_append_paged(L1, kb.cuda().contiguous(), vb.cuda().contiguous(), lens[b],
-                                    torch.zeros(1, dtype=torch.int32, device="cuda"), pair.dtable[b:b + 1],
-                                    pair.kc, pair.ks, pair.vc, pair.vs)
-        assert oracle.quantize_append_paged(pair.signs, np_f32(kb), np_f32(t.v[b][None]), np.zeros(1, np.int32),
-                                            pair.table[b:b + 1], 64, pair.cap, pair.pools) == 0
+    L1 = tq.tq_cache_layout_paged(1, pair.cap, w.n_kv_heads, w.n_q_heads, w.head_dim, k_format, 64, pair.L.n_pages)
+    zero = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for b in range(w.batch):  # prefill sequence by sequence: a one-sequence layout over the same pools, table row b
+        tq.tq_quantize_append_paged(L1, t.k[b][None].cuda().contiguous(), t.v[b][None].cuda().contiguous(), lens[b],
+                                    zero, pair.dtable[b:b + 1], pair.kc, pair.ks, pair.vc, pair.vs)
+
+    def oracle_prefill(b):  # sequences own disjoint pages, so the oracle's appends run side by side
+        return oracle.quantize_append_paged(pair.signs, np_f32(t.k[b][None]), np_f32(t.v[b][None]),
+                                            np.zeros(1, np.int32), pair.table[b:b + 1], 64, pair.cap, pair.pools)
+
+    assert all(st == 0 for st in parallel_map(oracle_prefill, range(w.batch)))
     pair.check_pools()
-    which = np.zeros((w.batch, w.n_q_heads), np.uint8)
-    which[seqs] = 1
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out, ref, st = pair.decode(t.q, lens, status, which)
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), dtype=torch.float32, device="cuda")
+    tq.tq_decode_attention_paged(pair.L, t.q.cuda().contiguous(), torch.tensor(lens, dtype=torch.int32).cuda(),
+                                 pair.dtable, pair.kc, pair.ks, pair.vc, pair.vs, w.scale, out,
+                                 tq.alloc_workspace(pair.L), status)
+    qn = np_f32(t.q)
+    ref, st = oracle_decode_all(lambda which: oracle.decode_attention_paged(
+        pair.signs, qn, np.array(lens, np.int32), pair.table, 64, pair.cap, pair.pools, w.scale, which),
+        w.batch, w.n_q_heads)
+    torch.cuda.synchronize()
     assert st == 0 and int(status.item()) == 0
-    assert_close(out[seqs], ref[seqs], what="paged ragged serving")
+    assert_close(out.cpu().numpy(), ref, what="paged ragged serving")
 
 
 def test_paged_unmapped_page_sets_capacity():

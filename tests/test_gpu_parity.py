@@ -19,16 +19,13 @@ from tests.parity_utils import GpuCache, OracleCache, assert_close, np_f32
 pytestmark = pytest.mark.gpu
 
 
-def fill_both(w, t, gpu, orc, seqs=None):
-    """Prefill every sequence on the GPU; the oracle encodes only `seqs` (default all)."""
-    seqs = range(w.batch) if seqs is None else seqs
+def fill_both(w, t, gpu, orc):
+    """Prefill every sequence, on the GPU and in the oracle (a host thread pool)."""
     for b in range(w.batch):
         if w.seq_lens[b] == 0 or t.k[b] is None:
             continue
         gpu.append_seq(b, t.k[b].cuda(), t.v[b].cuda(), 0)
-    for b in seqs:
-        if w.seq_lens[b]:
-            orc.append_seq(b, t.k[b], t.v[b], 0)
+    orc.append_seqs(t, [b for b in range(w.batch) if w.seq_lens[b]])
 
 
 def compare_caches(gpu, orc, seqs, lens):
@@ -41,26 +38,26 @@ def compare_caches(gpu, orc, seqs, lens):
         assert np.array_equal(vs[b, :L], orc.vs[b, :L]), f"V scales differ in sequence {b}"
 
 
-def run_workload(w, seqs=None, check_append=True):
+def run_workload(w, check_append=True):
+    """Every sequence and every q head of the workload against the oracle."""
     t = syn.generate(w)
     cap = w.capacity
     gpu = GpuCache(w.batch, cap, w.n_kv_heads, w.n_q_heads, w.head_dim)
     orc = OracleCache(w.batch, cap, w.n_kv_heads, w.head_dim)
-    fill_both(w, t, gpu, orc, seqs)
+    fill_both(w, t, gpu, orc)
     torch.cuda.synchronize()
-    seqs = list(range(w.batch)) if seqs is None else list(seqs)
+    seqs = list(range(w.batch))
     compare_caches(gpu, orc, seqs, w.seq_lens)
     q = t.q.cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu.decode(q, w.seq_lens, w.scale, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    which = np.zeros((w.batch, w.n_q_heads), np.uint8)
-    which[seqs] = 1
-    ref, st = orc.decode(t.q, w.seq_lens, w.scale, which)
+    hpt = w.group if w.batch == 1 else None  # one long sequence: one task per kv head's query group
+    ref, st = orc.decode_all(t.q, w.seq_lens, w.scale, hpt)
     assert st == 0
     got = out.cpu().numpy()
-    res = assert_close(got[seqs], ref[seqs], what=w.name)
+    res = assert_close(got, ref, what=w.name)
     print(f"\n{w.name}: max_abs {res[0]:.3e} rel_l2 {res[1]:.3e}")
     if check_append and w.n_append:
         # append one token per sequence at its length, then decode over len + 1
@@ -71,10 +68,10 @@ def run_workload(w, seqs=None, check_append=True):
         torch.cuda.synchronize()
         compare_caches(gpu, orc, seqs, lens1)
         out1 = gpu.decode(q, lens1, w.scale, status)
-        ref1, _ = orc.decode(t.q, lens1, w.scale, which)
+        ref1, _ = orc.decode_all(t.q, lens1, w.scale, hpt)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        assert_close(out1.cpu().numpy()[seqs], ref1[seqs], what=w.name + " +append")
+        assert_close(out1.cpu().numpy(), ref1, what=w.name + " +append")
     return res
 
 
@@ -95,12 +92,9 @@ def test_llama31_70b_long_context():
     run_workload(syn.llama31_70b_long())
 
 
-def test_ragged_serving_sampled():
-    w = syn.ragged_serving()
-    lens = w.seq_lens
-    order = np.argsort(lens)
-    seqs = sorted({int(order[0]), int(order[-1]), 3, 17})
-    run_workload(w, seqs=seqs)
+def test_ragged_serving_all_sequences():
+    # all 32 sequences (about 0.55 M tokens) and all 32 q heads of each
+    run_workload(syn.ragged_serving())
 
 
 def test_ragged_serving_prefill_4096():
