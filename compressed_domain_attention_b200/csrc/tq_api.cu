@@ -297,7 +297,9 @@ int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_codes) || !aligned16(v_codes) || (deleg && !aligned16(v_tail)))
     return TQ_ERR_INVALID_ARG;
   const int64_t v_rows = (int64_t)n_new + (deleg ? layout->tail_window : 0);
-  if ((int64_t)layout->batch * v_rows * layout->n_kv_heads * layout->n_groups * 2 > (int64_t)INT32_MAX * 256)
+  // the kernel indexes its threads in 32 bits: K and V items (padded to whole warps)
+  // must number fewer than 2^32
+  if ((int64_t)layout->batch * v_rows * layout->n_kv_heads * layout->n_groups * 2 + 64 >= (int64_t)1 << 32)
     return TQ_ERR_UNSUPPORTED;
   tqk::QuantizeParams p;
   p.k = k;
@@ -325,6 +327,9 @@ int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_
   p.page_tokens = layout->page_tokens;
   p.max_pages = layout->max_pages;
   p.n_pages = layout->n_pages;
+  p.div_kv = tqk::make_fastdiv((uint32_t)layout->n_kv_heads);
+  p.div_new = tqk::make_fastdiv((uint32_t)n_new);
+  p.div_vrows = tqk::make_fastdiv((uint32_t)v_rows);
   cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }

@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; !walk.done(); walk.advance<T_TILE>()) {
       const int stage = issued % STAGES;
       const uint32_t n = (uint32_t)(issued / STAGES);
-      if (!mbar_wait_backoff(&empty[stage], (n & 1u) ^ 1u, p.wait_ns)) {
+      if (!mbar_wait_bounded(&empty[stage], (n & 1u) ^ 1u, p.wait_ns)) {
         dead = true;
         break;
       }
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int stage = tile_i % STAGES;
       const uint32_t par = (uint32_t)((tile_i / STAGES) & 1);
       // (a producer that gave up issues nothing more: these waits then run out)
-      if (!dead && !mbar_wait_backoff(&full[stage], par, p.wait_ns)) {
+      if (!dead && !mbar_wait_bounded(&full[stage], par, p.wait_ns)) {
         dead = true;
         if (lane == 0) status_or(p.status, TQ_STATUS_TIMEOUT);
       }
@@ -419,7 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool mapped;
         const int64_t row0 = tile_first_row(p, walk.b, walk.t0, mapped);  // the producer's scale row
         const int soff = (int)((row0 * C::SROW) & 15);
-        const int nv = min(T_TILE, walk.seg_hi - walk.t0);
+        // an unmapped page's tile reads as zeros: its codes come from past the pool (zero
+        // fill) and its scales are set to 0 here (the slab the producer copied is row 0's)
+        const int nv = mapped ? min(T_TILE, walk.seg_hi - walk.t0) : 0;
         const uint32_t sc = smem_u32(sb + C::OFF_SC32);
         const bool part_tile = nv < T_TILE;  // the same for every lane: tokens past nv get 0
 #pragma unroll
@@ -1597,15 +1599,38 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
     lsv[d] = o;  // lsv[] is free again: reused for the normalised vector
   }
   __syncthreads();
-  if (tid < 32) {
-    const int part = tid % NG;
-    float u[32];
+  if constexpr (D <= NTH) {
+    // one element per thread: the butterflies of stride 1 .. 16 between lanes, the wider
+    // ones through shared memory, in the forward transform's stage order (each stage
+    // forms u_i + u_{i+h} and u_i - u_{i+h} with one rounding, as the scalar steps do)
+    float u = tid < D ? lsv[tid] : 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = lsv[part * 32 + i];
-    fwht_group<NG>(u, part);
-    if (tid < NG) {
+    for (int h = 1; h < 32 && h < D; h <<= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, u, h);
+      u = (lane & h) ? __fsub_rn(o, u) : __fadd_rn(u, o);
+    }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) out[part * 32 + i] = apply_sign(u[i] * p.c_d, p.sign_bits, part * 32 + i);
+    for (int h = 32; h < D; h <<= 1) {
+      __syncthreads();  // every read of lsv[] from the previous stage is done
+      if (tid < D) lsv[tid] = u;
+      __syncthreads();
+      if (tid < D) {
+        const float o = lsv[tid ^ h];
+        u = (tid & h) ? __fsub_rn(o, u) : __fadd_rn(u, o);
+      }
+    }
+    if (tid < D) out[tid] = apply_sign(u * p.c_d, p.sign_bits, tid);
+  } else {
+    if (tid < 32) {
+      const int part = tid % NG;
+      float u[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = lsv[part * 32 + i];
+      fwht_group<NG>(u, part);
+      if (tid < NG) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) out[part * 32 + i] = apply_sign(u[i] * p.c_d, p.sign_bits, part * 32 + i);
+      }
     }
   }
 }

@@ -175,20 +175,8 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// As mbar_try_wait, but the hardware may suspend the thread up to `hint_ns`
-// before reporting that the phase is still incomplete.
+// Test whether the phase with the given parity has completed; the hardware may
+// suspend the thread up to `hint_ns` before reporting that it has not.
 __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
@@ -207,33 +195,36 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wait for the phase with the given parity to complete, giving up after
-// `limit_ns` nanoseconds of wall time. Returns false on timeout. Each suspended
-// try lasts at most min(limit, 20 us), so a bound shorter than a typical wait
-// does run out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  const uint32_t hint = limit_ns < 20000u ? (uint32_t)limit_ns : 20000u;
-  while (true) {
-    if (mbar_try_wait_hint(bar, parity, hint)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
-// As mbar_wait_bounded, for warps that wait most of the time (the copy issuer and
-// the scale converters): after a failed test the warp sleeps, 32 ns doubling up to
-// 256 ns, so that its polling takes few issue slots from the math warps that share
-// its scheduler.
-__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Wait for the phase with the given parity to complete, giving up after
+// `limit_ns` nanoseconds of wall time. Returns false on timeout. A suspending
+// test (try_wait) may stay suspended until the phase completes, however short
+// its hint, so a bound under 20 us is kept by polling the non-blocking test
+// instead; longer bounds suspend up to 20 us per test.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t ns = 32;
+  if (limit_ns < 20000u) {
+    while (true) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
   while (true) {
-    __nanosleep(ns);
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
-    if (ns < 256) ns <<= 1;
   }
 }
 

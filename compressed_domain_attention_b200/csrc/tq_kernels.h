@@ -6,6 +6,32 @@
 
 namespace tqk {
 
+// Division of a 32-bit unsigned n by an invariant divisor d >= 1 with a multiply and
+// shifts (the round-up method of Granlund and Montgomery, "Division by invariant
+// integers using multiplication"): m = floor(2^32 (2^l - d) / d) + 1 with
+// l = ceil(log2 d); q = (t + ((n - t) >> 1)) >> (l - 1), t = umulhi(m, n); d = 1 is
+// the identity (l = 0). Exact for every n < 2^32.
+struct FastDiv {
+  uint32_t d, m, l;
+};
+
+__host__ __forceinline__ FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = d <= 1 ? 0u : (uint32_t)((((1ull << 32) * ((1ull << f.l) - d)) / d) + 1);
+  return f;
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+  if (f.l == 0) return n;
+  const uint32_t t = __umulhi(f.m, n);
+  return (t + ((n - t) >> 1)) >> (f.l - 1);
+}
+#endif
+
 struct QuantizeParams {
   const void* k;
   const void* v;
@@ -29,6 +55,9 @@ struct QuantizeParams {
   // block_table[b * max_pages + t / page_tokens] * page_tokens + t % page_tokens
   const int32_t* block_table;
   int page_tokens, max_pages, n_pages;
+  // 32-bit thread indexing (the launch has fewer than 2^32 threads): divisors n_kv,
+  // n_new and n_new + tail_window
+  FastDiv div_kv, div_new, div_vrows;
 };
 
 struct DequantParams {

@@ -23,6 +23,18 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
+// three-input max that propagates NaN, and the plain three-input max
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Cache row of token t of sequence b: b * max_seq + t, or through the block table
 // with paged storage (ok = false for an entry outside [0, n_pages)).
 __device__ __forceinline__ int64_t token_row(const QuantizeParams& p, int b, int64_t t, bool& ok) {
@@ -36,16 +48,17 @@ __device__ __forceinline__ int64_t token_row(const QuantizeParams& p, int b, int
 // Asymmetric cache (mlxcel guide, cache modes: K kept in FP16): thread kt stores
 // the binary16 (round to nearest even) of 32 consecutive K elements.
 template <int D>
-__device__ __forceinline__ void copy_k_f16(const QuantizeParams& p, int64_t kt) {
+__device__ __forceinline__ void copy_k_f16(const QuantizeParams& p, uint32_t kt) {
   constexpr int NG = D / 32;
-  const int64_t r = kt / NG;
+  const uint32_t r = kt / NG;
   const int part = (int)(kt % NG);
-  const int h = (int)(r % p.n_kv);
-  const int64_t bt = r / p.n_kv;
-  const int t = (int)(bt % p.n_new);
-  const int b = (int)(bt / p.n_new);
+  const uint32_t bt = fast_div(r, p.div_kv);
+  const int h = (int)(r - bt * (uint32_t)p.n_kv);
+  const uint32_t b_ = fast_div(bt, p.div_new);
+  const int t = (int)(bt - b_ * (uint32_t)p.n_new);
+  const int b = (int)b_;
   float u[32];
-  load32(u, p.k, r * D + part * 32, p.in_dtype);
+  load32(u, p.k, (int64_t)r * D + part * 32, p.in_dtype);
   const int64_t pos = p.start_pos[b];
   if (pos < 0 || pos + p.n_new > p.max_seq) {
     if (t == 0 && h == 0 && part == 0) status_or(p.status, TQ_STATUS_CAPACITY);
@@ -94,28 +107,30 @@ __device__ __forceinline__ void write_tail_f16(const QuantizeParams& p, int64_t 
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_constant__ QuantizeParams p) {
+__global__ void __launch_bounds__(256, 4) quantize_append_kernel(const __grid_constant__ QuantizeParams p) {
   // Launched as a programmatic dependent of the previous kernel on the stream:
   // nothing is read before this wait. The decode that usually follows may be
   // scheduled from here on; it waits for this grid's completion before reading.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int NG = D / 32;
-  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // 32-bit indexing throughout (the host launches fewer than 2^32 threads); divisions
+  // by the runtime sizes are multiply-and-shift (FastDiv)
+  const uint32_t gt = blockIdx.x * blockDim.x + threadIdx.x;
   const int W = p.tail_window;  // > 0 only for the delegated cache
-  const int64_t vecs_k = (int64_t)p.batch * p.n_new * p.n_kv;
+  const uint32_t vecs_k = (uint32_t)p.batch * (uint32_t)p.n_new * (uint32_t)p.n_kv;
   // V work items per (sequence, head): the new tokens, then (delegated) W fold candidates
   const int v_rows = p.n_new + W;
-  int64_t vec = gt / NG;
+  const uint32_t vec = gt / NG;
   const int part = (int)(gt % NG);
   int which;
-  int64_t r;
+  uint32_t r;
   bool in_range;
   if (p.k_f16) {
     // V threads first, then the K copies from the next warp boundary on, so that a
     // warp is all V (its lanes exchange butterflies) or all K.
-    const int64_t thr_v = (int64_t)p.batch * v_rows * p.n_kv * NG;
-    const int64_t kbase = (thr_v + 31) / 32 * 32;
+    const uint32_t thr_v = (uint32_t)p.batch * (uint32_t)v_rows * (uint32_t)p.n_kv * NG;
+    const uint32_t kbase = (thr_v + 31) / 32 * 32;
     if (gt >= kbase) {
       if (gt - kbase < vecs_k * NG) copy_k_f16<D>(p, gt - kbase);
       return;
@@ -125,14 +140,15 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
     r = in_range ? vec : 0;
   } else {
     in_range = vec < 2 * vecs_k;
-    which = in_range ? (int)(vec / vecs_k) : 0;  // 0 = K, 1 = V
-    r = in_range ? vec % vecs_k : 0;
+    which = (in_range && vec >= vecs_k) ? 1 : 0;  // 0 = K, 1 = V
+    r = in_range ? vec - (which ? vecs_k : 0u) : 0u;
   }
   const int rows = which ? v_rows : p.n_new;
-  const int h = (int)(r % p.n_kv);
-  const int64_t bt = r / p.n_kv;
-  const int t = (int)(bt % rows);
-  const int b = (int)(bt / rows);
+  const uint32_t bt = fast_div(r, p.div_kv);
+  const int h = (int)(r - bt * (uint32_t)p.n_kv);
+  const uint32_t b_ = fast_div(bt, which ? p.div_vrows : p.div_new);
+  const int t = (int)(bt - b_ * (uint32_t)rows);
+  const int b = (int)b_;
   const int64_t in_row = ((int64_t)b * p.n_new + t) * p.n_kv + h;  // input vector of a new token
 
   float u[32];
@@ -237,7 +253,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
       const float2 y = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(p.c_d));
       u[i] = y.x;
       u[i + 1] = y.y;
-      a = fmax_nan(a, fmax_nan(fabsf(y.x), fabsf(y.y)));
+      a = fmax3_nan(a, fabsf(y.x), fabsf(y.y));
     }
   }
   if (!valid) {
@@ -266,16 +282,26 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const __grid_const
     if (!slow) {
       const float inv = __frcp_rn(sigma);
       constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+      uint32_t rb[32];  // the rounded sums: the low byte holds the code (two's complement)
+      float dmax = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         const float2 rv = __fmul2_rn(make_float2(u[i], u[i + 1]), f2(inv));
         const float2 rm = __fadd2_rn(rv, f2(kMagic));
         const float2 rr = __fadd2_rn(rm, f2(-kMagic));
         const float2 d = __ffma2_rn(rr, f2(-1.f), rv);  // r - rint(r), exact
-        slow |= fabsf(d.x) >= 0.49999809265136719f;    // 0.5 - 2^-19
-        slow |= fabsf(d.y) >= 0.49999809265136719f;
-        const uint32_t pair = (__float_as_uint(rm.x) & 0xFu) | ((__float_as_uint(rm.y) & 0xFu) << 4);
-        packed[i >> 3] |= pair << (4 * (i & 7));
+        dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
+        rb[i] = __float_as_uint(rm.x);
+        rb[i + 1] = __float_as_uint(rm.y);
+      }
+      slow = dmax >= 0.49999809265136719f;  // 0.5 - 2^-19
+      // byte j of a packed word: code 2j in the low nibble, code 2j + 1 in the high one
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t* e = rb + 8 * k;
+        const uint32_t lo = __byte_perm(__byte_perm(e[0], e[2], 0x0040u), __byte_perm(e[4], e[6], 0x0040u), 0x5410u);
+        const uint32_t hi = __byte_perm(__byte_perm(e[1], e[3], 0x0040u), __byte_perm(e[5], e[7], 0x0040u), 0x5410u);
+        packed[k] = (lo & 0x0F0F0F0Fu) | ((hi << 4) & 0xF0F0F0F0u);
       }
     }
     if (slow) {
