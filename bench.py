@@ -631,21 +631,45 @@ def _pct(xs, q):
     return xs[lo] + (xs[hi] - xs[lo]) * (k - lo)
 
 
-def _time_reps(fn, reps, flush, stream):
-    """Device times (ms) of fn(), one per rep; flush (a buffer > L2 rewritten) before each rep if given."""
+def _time_graph_pairs(launch, flush, stream, n=10, reps=9):
+    """Device time (ms) per call of launch(stream), L2 flushed before each call (flush given)
+    or back to back (flush None), finer than one event pair allows (event timestamps on this
+    part tick in about 2 us): a CUDA graph of n (flush, call) pairs and one of the n flushes
+    alone are replayed in turn between events; per call = (pairs - flushes) / n."""
     import torch
+    ga = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ga):
+        for _ in range(n):
+            if flush is not None:
+                flush.add_(1)
+            launch(torch.cuda.current_stream())
+    gb = None
+    if flush is not None:
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb):
+            for _ in range(n):
+                flush.add_(1)
+    torch.cuda.synchronize()
     ts = []
-    for _ in range(reps):
-        if flush is not None:
-            flush.add_(1)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
+    for _ in range(reps + 1):
+        pair = []
+        for g in (ga, gb):
+            if g is None:
+                pair.append(0.0)
+                continue
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            pair.append(a.elapsed_time(b))
+        ts.append((pair[0] - pair[1]) / n)
+    ts = ts[1:]  # the first replay of each graph uploads it
+    del ga, gb
     return {"median": round(statistics.median(ts), 4), "p10": round(_pct(ts, 0.1), 4),
-            "p90": round(_pct(ts, 0.9), 4), "reps": reps}
+            "p90": round(_pct(ts, 0.9), 4), "reps": reps, "calls_per_rep": n,
+            "method": "graph of (L2 flush, call) pairs minus a graph of the flushes" if flush is not None
+            else "graph of back-to-back calls"}
 
 
 def run_sweep(args):
@@ -682,12 +706,12 @@ def run_sweep(args):
         kb = [t.k[b][None].contiguous() for b in range(w.batch)]
         vb = [t.v[b][None].contiguous() for b in range(w.batch)]
 
-        def prefill():
+        def prefill(s=stream):
             for b in range(w.batch):
-                cache.append_seq(b, kb[b], vb[b], w.seq_lens[b], zero, status, stream)
+                cache.append_seq(b, kb[b], vb[b], w.seq_lens[b], zero, status, s)
 
         prefill()
-        pre = _time_reps(prefill, 5, flush, stream)
+        pre = _time_graph_pairs(prefill, flush, stream, n=3, reps=5)
         vecs = 2 * sum(w.seq_lens) * w.n_kv_heads
         lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
         q = t.q.contiguous()
@@ -698,16 +722,16 @@ def run_sweep(args):
 
         for _ in range(10):
             decode()
-        reps = 20 if sum(w.seq_lens) * w.n_kv_heads >= 1 << 20 else 100
-        cold = _time_reps(decode, reps, flush, stream)
+        # every timed arm replays CUDA graphs (the dense SDPA below too), so that no host
+        # launch work sits between the events
+        dec = lambda s: cache.decode(q, lens, w.scale, out, status, s)  # noqa: E731
+        cold = _time_graph_pairs(dec, flush, stream)
         nbytes = decode_bytes(w, w.seq_lens, fmt)
-        warm = _time_reps(decode, reps, None, stream) if nbytes < 64e6 else None
+        warm = _time_graph_pairs(dec, None, stream) if nbytes < 64e6 else None
         kn, vn = t.k_new.contiguous() if w.n_append else None, t.v_new.contiguous() if w.n_append else None
         app = None
         if w.n_append:
-            def append():
-                cache.append(kn, vn, w.n_append, lens, status, stream)
-            app = _time_reps(append, 50, flush, stream)
+            app = _time_graph_pairs(lambda s: cache.append(kn, vn, w.n_append, lens, status, s), flush, stream)
         dense = None
         if w.dtype != torch.float32:
             ks_d = [t.k[b].permute(1, 0, 2).contiguous()[None] for b in range(w.batch)]
@@ -719,11 +743,8 @@ def run_sweep(args):
                     F.scaled_dot_product_attention(qd[b:b + 1], ks_d[b], vs_d[b], scale=w.scale, enable_gqa=True)
 
             dense_fn()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                dense_fn()
-            dense = _time_reps(g.replay, min(reps, 20), flush, stream)
-            del g, ks_d, vs_d
+            dense = _time_graph_pairs(lambda s: dense_fn(), flush, stream)
+            del ks_d, vs_d
         torch.cuda.synchronize()
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the sweep ({w.name})")

@@ -105,6 +105,35 @@ int encode_codes_map(const tq_layout_t* L, const uint8_t* base, int tile, tqk::T
   return TQ_OK;
 }
 
+// Appends of more than this many vectors (K and V) take the one-thread-per-vector
+// kernel; smaller ones (a decode step's new tokens, short prefills) the
+// thread-per-group kernel, whose four-fold parallelism per vector gives a shorter
+// launch (measured back to back: 2.8 against 4.1 us on a 512-vector append, 9.6
+// against 10.1 us on 65 536 vectors; 224 against 168 us on 2.1 M vectors).
+constexpr uint64_t kRowsKernelMinVectors = 65537;
+
+// 2-D view of an append input (K or V) for the row-wise kernel: `rows` vectors of
+// D elements of esz bytes, box (128 bytes of a row, rows_kernel_box_rows(D) rows)
+// with the 128-byte swizzle.
+int encode_rows_map(const void* base, int D, int esz, uint64_t rows, tqk::TensorMap128* out) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * (cuuint64_t)esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)tqk::rows_kernel_box_rows(D)};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMap m;
+  CUresult r = enc(&m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = (int)r;
+    return TQ_ERR_CUDA;
+  }
+  std::memcpy(out, &m, sizeof(m));
+  return TQ_OK;
+}
+
 // 4-D view of a binary16 K buffer: (64 halves, batch*max_seq tokens, D/64 lines,
 // n_kv heads) with strides (token stride, 128 B, 2D B), box (64, tile, D/64, n_kv):
 // the shared-memory image is [head][line][tile][64] binary16 with the 128-byte
@@ -330,7 +359,26 @@ int append_impl(const tq_layout_t* layout, const void* k, const void* v, int in_
   p.div_kv = tqk::make_fastdiv((uint32_t)layout->n_kv_heads);
   p.div_new = tqk::make_fastdiv((uint32_t)n_new);
   p.div_vrows = tqk::make_fastdiv((uint32_t)v_rows);
-  cudaError_t e = tqk::launch_quantize(p, layout->head_dim, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int D = layout->head_dim;
+  cudaError_t e;
+  const uint64_t vectors = 2ull * (uint64_t)layout->batch * (uint64_t)n_new * (uint64_t)layout->n_kv_heads;
+  if (!deleg && (D == 64 || D == 128) && vectors >= kRowsKernelMinVectors) {
+    // one thread per vector, input rows by tensor copies
+    const int esz = in_dtype == TQ_F32 ? 4 : 2;
+    const uint64_t rows = (uint64_t)layout->batch * (uint64_t)n_new * (uint64_t)layout->n_kv_heads;
+    tqk::TensorMap128 kin, vin;
+    int rc = encode_rows_map(k, D, esz, rows, &kin);
+    if (rc != TQ_OK) return rc;
+    rc = encode_rows_map(v, D, esz, rows, &vin);
+    if (rc != TQ_OK) return rc;
+    int sms = 0;
+    rc = device_sm_count(&sms);
+    if (rc != TQ_OK) return rc;
+    e = tqk::launch_quantize_rows(p, D, kin, vin, sms, s);
+  } else {
+    e = tqk::launch_quantize(p, D, s);
+  }
   return e == cudaSuccess ? TQ_OK : cuda_fail(e);
 }
 

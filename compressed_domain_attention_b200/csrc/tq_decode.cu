@@ -55,7 +55,8 @@ constexpr int kConverterWarp = kConsumerWarps + 1;  // first of the binary16 -> 
 constexpr int kConverterWarps = 3;                  // one on each scheduler without the producer
 constexpr int kThreads = (kConsumerWarps + 1 + kConverterWarps) * 32;
 constexpr int kMaxBatch = 1024;
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 128;     // merge blocks when (sequence, head) pairs are many
+constexpr int kMergeThreadsFew = 512;  // and when they number fewer than twice the split CTAs
 constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s bound on the producer's wait for its copies in flight
 
 // KF16: K tiles are binary16 in the original domain (asymmetric cache), the V
@@ -263,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Launched as a programmatic dependent of whatever kernel precedes it on the stream
   // (typically the append). Set-up that reads nothing another kernel writes (barrier
   // initialisation, tensor-map prefetch) runs before the dependency wait; no global
-  // memory is read before it.
+  // memory is read before it. L2 prefetches (hints that return no data) of the
+  // lengths and the query may go first: L2 is where any later store to them lands.
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -274,21 +276,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(&kmap) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&vmap) : "memory");
-  }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) {
-    // The query is read by every block's prologue once the prefix sums are known, by when
-    // the tile copies have started: each block prefetches one slice of it into L2 now.
-    const uint32_t qbytes = (uint32_t)p.batch * (uint32_t)p.n_q * (uint32_t)(D * (p.q_dtype == TQ_F32 ? 4 : 2));
-    const uint32_t per = ((qbytes + gridDim.x - 1) / gridDim.x + 127u) & ~127u;  // whole 128-byte lines
-    const uint32_t o0 = blockIdx.x * per;
-    if (o0 < qbytes) {
-      const uint32_t n = min(per, qbytes - o0);  // a multiple of 16 (rows of D >= 32 elements)
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<const uint8_t*>(p.q) + o0),
-                   "r"(n)
-                   : "memory");
+  } else if (warp == 1) {
+    // every block reads all lengths for its prefix sums (one 128-byte line per 32)
+    for (int i = lane * 32; i < p.batch; i += 32 * 32) prefetch_l2(p.seq_lens + i);
+    if (lane == 0) {
+      // the query is read by every block's prologue once the prefix sums are known:
+      // each block prefetches one slice of it
+      const uint32_t qbytes =
+          (uint32_t)p.batch * (uint32_t)p.n_q * (uint32_t)(D * (p.q_dtype == TQ_F32 ? 4 : 2));
+      const uint32_t per = ((qbytes + gridDim.x - 1) / gridDim.x + 127u) & ~127u;  // whole 128-byte lines
+      const uint32_t o0 = blockIdx.x * per;
+      if (o0 < qbytes) {
+        const uint32_t n = min(per, qbytes - o0);  // a multiple of 16 (rows of D >= 32 elements)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                     ::"l"(reinterpret_cast<const uint8_t*>(p.q) + o0), "r"(n)
+                     : "memory");
+      }
     }
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   block_prefix_lengths(p, prefix, prefix + (p.batch + 1));  // its barriers also publish the set-up
   const int64_t T_sum = prefix[p.batch];
   // T_sum < 2^32 (batch * max_seq <= INT32_MAX, plus at most a tile of padding per
@@ -1123,12 +1129,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Combine the partials of one (sequence, q head), normalise, inverse SRHT.
 // Launched as a programmatic dependent of the split-K kernel: blocks may start
 // early and wait at griddepcontrol.wait until every split-K block has finished
-// and its writes are visible. Phase 1 stages the weights 2^(m_c - m*) of all
-// partials in shared memory; phase 2 streams the accumulators with PF
-// independent loads in flight per thread.
+// and its writes are visible; before the wait they prefetch the lines of their
+// partials into L2 (the address translations are then warm). Phase 1 stages
+// the weights 2^(m_c - m*) of all partials in shared memory; phase 2 streams
+// the accumulators with PF independent loads in flight per thread; one warp
+// then sums the slot phases and runs the inverse transform with shuffles.
 // NTH = 128 threads (8 blocks per SM) when there are many (sequence, head)
-// pairs, 1024 when there are fewer than twice the SMs: a long sequence then has
-// up to one partial per SM, and its loads should all be in flight at once.
+// pairs, 512 when there are fewer than twice the SMs: a long sequence then has
+// up to one partial per SM, and its loads (10 per thread, 160 partials at
+// head_dim 128) should all be in flight at once.
 // Kernel 1b (decode_tail_kernel, delegated cache only): attention partials over
 // the hot tail (mlxcel guide, delegated cache variant: the recent tokens keep
 // binary16 K and V). One block per (sequence, kv head, chunk of kTailTokens hot
@@ -1451,12 +1460,14 @@ static cudaError_t launch_tail(const DecodeParams& p, cudaStream_t s, bool pdl) 
 }
 
 template <int D, int NTH>
-__global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int NG = D / 32;
+__global__ void __launch_bounds__(NTH, NTH >= 512 ? 1 : 1024 / NTH)
+    decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int F4 = D / 4;            // float4 columns
   constexpr int PH = NTH / F4;         // slot phases
-  constexpr int PF = 8;                // loads in flight per thread
+  constexpr int PF = NTH >= 512 ? 10 : 8;  // loads in flight per thread
+  constexpr int E = D / 32;            // elements per lane in the closing transform
   constexpr int MAX_SLOTS = 1024;      // a sequence meets at most one partial per split-K CTA
+  static_assert(PH >= 1 && PH * F4 == NTH, "whole float4 rows per slot phase");
   __shared__ float wts[MAX_SLOTS + kMaxTailChunks];
   __shared__ float lsv[MAX_SLOTS + kMaxTailChunks];
   __shared__ float red[NTH / 32];
@@ -1508,13 +1519,9 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   // Delegated cache: the hot tail's partials (one per chunk of hot tokens, in the
   // rotated domain like the rest) follow in slots tail_slot0 + b * tail_chunks + k.
   const int n_tail = (p.tail_window > 0 && len_all > 0) ? p.tail_chunks : 0;
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const bool empty = P1 <= P0 && n_tail == 0;
   const float* ml = p.ws_ml + 2 * (p.batch + 2);
   float* out = p.out + ((int64_t)b * p.n_q + hq) * D;
-  if (P1 <= P0 && n_tail == 0) {  // empty sequence
-    for (int d = tid; d < D; d += NTH) out[d] = 0.f;
-    return;
-  }
   const int c0 = P1 > P0 ? (int)(P0 / R) : 0, c1 = P1 > P0 ? (int)((P1 - 1) / R) : -1;
   const int ns_cold = min(c1 - c0 + 1, MAX_SLOTS);
   const int ns = ns_cold + n_tail;
@@ -1529,18 +1536,47 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   auto acc_at = [&](int i) {  // partial i: the cold run first, then the tail run
     return i < ns_cold ? base + (int64_t)i * stride : tbase + (int64_t)(i - ns_cold) * stride;
   };
-  // The accumulator loads of the first chunk do not depend on the weights: issue them
-  // together with the (m, l) loads, so the merge costs about one memory round trip.
+  auto ml_at = [&](int i) {
+    return reinterpret_cast<const float2*>(i < ns_cold ? mlb + i * mls : mlt + (i - ns_cold) * mls);
+  };
+  // While the split-K grid runs, warm the address translation and L2 lines of the
+  // partials this thread reads first. Prefetches only: the values are loaded after
+  // the wait, from L2, where the split-K blocks' stores land.
+  if (!empty) {
+    for (int i = tid; i < ns; i += NTH) prefetch_l2(ml_at(i));
+    if ((col & 7) == 0) {  // one 128-byte line per 8 float4 columns
+#pragma unroll
+      for (int k = 0; k < PF; ++k) {
+        const int i = ph + k * PH;
+        if (i < ns) prefetch_l2(acc_at(i));
+      }
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (empty) {  // empty sequence
+    for (int d = tid; d < D; d += NTH) out[d] = 0.f;
+    return;
+  }
+  // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l.
+  // The (m, l) loads go first; the accumulator loads of the first chunk, which do not
+  // depend on the weights, follow at once and stream in behind them, so the merge
+  // costs about one memory round trip.
+  float m = -INFINITY;
+  float2 e0 = make_float2(-INFINITY, 0.f);
+  if (tid < ns) e0 = __ldcg(ml_at(tid));
   float4 v[PF];
 #pragma unroll
   for (int k = 0; k < PF; ++k) {
     const int i = ph + k * PH;
     v[k] = i < ns ? __ldcg(acc_at(i)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // phase 1: (m, l) of every partial in one pass -> m*, weights, sum of weighted l
-  float m = -INFINITY;
-  for (int i = tid; i < ns; i += NTH) {
-    const float2 e = __ldcg(reinterpret_cast<const float2*>(i < ns_cold ? mlb + i * mls : mlt + (i - ns_cold) * mls));
+  if (tid < ns) {
+    wts[tid] = e0.x;
+    lsv[tid] = e0.y;
+    m = e0.x;
+  }
+  for (int i = tid + NTH; i < ns; i += NTH) {
+    const float2 e = __ldcg(ml_at(i));
     wts[i] = e.x;
     lsv[i] = e.y;
     m = fmaxf(m, e.x);
@@ -1563,10 +1599,6 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
   __syncthreads();  // red[] reused, wts[] complete
   if (lane == 0) red[wp] = lsum;
-  __syncthreads();
-  float L = 0.f;
-#pragma unroll
-  for (int w = 0; w < NTH / 32; ++w) L += red[w];
   // phase 2: weighted accumulator sums, PH slot phases x F4 float4 columns
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i0 = ph;; i0 += PH * PF) {
@@ -1587,51 +1619,58 @@ __global__ void __launch_bounds__(NTH, 1024 / NTH) decode_merge_kernel(const __g
     }
   }
   reinterpret_cast<float4*>(accs[ph])[col] = a;
-  __syncthreads();
-  // sum the slot phases per channel and normalise, then the inverse SRHT
+  __syncthreads();  // accs[] and the l sums of every warp are complete
+  if (wp != 0) return;
+  // One warp closes: lane l sums the slot phases of elements l E .. l E + E - 1,
+  // normalises, and runs the inverse SRHT (butterflies of stride below E in
+  // registers, the wider ones between lanes, in the forward transform's stage
+  // order; each stage forms u_i + u_{i+h} and u_i - u_{i+h} with one rounding).
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < NTH / 32; ++w) L += red[w];
   const float inv_l = (L > 0.f) ? 1.f / L : 0.f;
-  for (int d = tid; d < D; d += NTH) {
-    float sum = 0.f;
+  float u[E];
 #pragma unroll
-    for (int q = 0; q < PH; ++q) sum += accs[q][d];
-    float o = sum * inv_l;
-    if (p.lambda_v != nullptr) o = __fdividef(o, __ldg(p.lambda_v + d));  // the V codes hold lambda o y
-    lsv[d] = o;  // lsv[] is free again: reused for the normalised vector
+  for (int j = 0; j < E; ++j) u[j] = 0.f;
+#pragma unroll
+  for (int q = 0; q < PH; ++q) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) u[j] += accs[q][lane * E + j];
   }
-  __syncthreads();
-  if constexpr (D <= NTH) {
-    // one element per thread: the butterflies of stride 1 .. 16 between lanes, the wider
-    // ones through shared memory, in the forward transform's stage order (each stage
-    // forms u_i + u_{i+h} and u_i - u_{i+h} with one rounding, as the scalar steps do)
-    float u = tid < D ? lsv[tid] : 0.f;
 #pragma unroll
-    for (int h = 1; h < 32 && h < D; h <<= 1) {
-      const float o = __shfl_xor_sync(0xffffffffu, u, h);
-      u = (lane & h) ? __fsub_rn(o, u) : __fadd_rn(u, o);
-    }
+  for (int j = 0; j < E; ++j) {
+    float o = u[j] * inv_l;
+    if (p.lambda_v != nullptr) o = __fdividef(o, __ldg(p.lambda_v + lane * E + j));  // the V codes hold lambda o y
+    u[j] = o;
+  }
 #pragma unroll
-    for (int h = 32; h < D; h <<= 1) {
-      __syncthreads();  // every read of lsv[] from the previous stage is done
-      if (tid < D) lsv[tid] = u;
-      __syncthreads();
-      if (tid < D) {
-        const float o = lsv[tid ^ h];
-        u = (tid & h) ? __fsub_rn(o, u) : __fadd_rn(u, o);
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      if ((j & h) == 0) {
+        const float x = u[j], y = u[j + h];
+        u[j] = __fadd_rn(x, y);
+        u[j + h] = __fsub_rn(x, y);
       }
     }
-    if (tid < D) out[tid] = apply_sign(u * p.c_d, p.sign_bits, tid);
+  }
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const float o = __shfl_xor_sync(0xffffffffu, u[j], h);
+      u[j] = (lane & h) ? __fsub_rn(o, u[j]) : __fadd_rn(u[j], o);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < E; ++j) u[j] = apply_sign(u[j] * p.c_d, p.sign_bits, lane * E + j);
+  if constexpr (E % 4 == 0) {
+#pragma unroll
+    for (int j = 0; j < E; j += 4)
+      *reinterpret_cast<float4*>(out + lane * E + j) = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
   } else {
-    if (tid < 32) {
-      const int part = tid % NG;
-      float u[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) u[i] = lsv[part * 32 + i];
-      fwht_group<NG>(u, part);
-      if (tid < NG) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) out[part * 32 + i] = apply_sign(u[i] * p.c_d, p.sign_bits, part * 32 + i);
-      }
-    }
+    for (int j = 0; j < E; ++j) out[lane * E + j] = u[j];
   }
 }
 
@@ -1672,7 +1711,7 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
       }
     }
     if (few)
-      decode_merge_kernel<D, 1024><<<p.batch * p.n_q, 1024, 0, s>>>(p);
+      decode_merge_kernel<D, kMergeThreadsFew><<<p.batch * p.n_q, kMergeThreadsFew, 0, s>>>(p);
     else
       decode_merge_kernel<D, kMergeThreads><<<p.batch * p.n_q, kMergeThreads, 0, s>>>(p);
     return cudaGetLastError();
@@ -1689,7 +1728,7 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.batch * p.n_q));
-  cfg.blockDim = dim3(few ? 1024 : kMergeThreads);
+  cfg.blockDim = dim3(few ? kMergeThreadsFew : kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1697,7 +1736,7 @@ static cudaError_t launch_decode_dht(const DecodeParams& p, const TensorMap128& 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (few) return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 1024>, p);
+  if (few) return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, kMergeThreadsFew>, p);
   return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, kMergeThreads>, p);
 }
 

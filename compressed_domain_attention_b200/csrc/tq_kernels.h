@@ -137,7 +137,24 @@ __host__ __forceinline__ uint64_t decode_workspace_bytes(int batch, int n_q, int
   return ((header + ml + 255) / 256) * 256 + acc;
 }
 
+// Threads per block of the row-wise append kernel, the threads that share one head
+// vector, and the rows (vectors) of its input tensor-copy box. One thread per vector:
+// splitting a head_dim-128 vector over two threads (one shuffle stage, 128 instead
+// of 168 registers, 4 instead of 3 blocks per SM) measured slower (190 against
+// 175 us on a 2.1 M-vector prefill).
+constexpr int kRowsThreads = 128;
+__host__ __device__ constexpr int rows_threads_per_vector(int /*head_dim*/) { return 1; }
+__host__ __device__ constexpr int rows_kernel_box_rows(int head_dim) {
+  return kRowsThreads / rows_threads_per_vector(head_dim);
+}
+
 cudaError_t launch_quantize(const QuantizeParams& p, int head_dim, cudaStream_t s);
+// The row-wise append (head_dim 64 or 128, no hot tail): kin / vin view the K / V
+// inputs as [batch * n_new * n_kv][head_dim] with boxes of 128 bytes by
+// rows_kernel_box_rows(head_dim) rows and the 128-byte swizzle; persistent blocks on
+// `sms` SMs.
+cudaError_t launch_quantize_rows(const QuantizeParams& p, int head_dim, const TensorMap128& kin,
+                                 const TensorMap128& vin, int sms, cudaStream_t s);
 cudaError_t launch_dequantize(const DequantParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, const TensorMap128& kmap, const TensorMap128& vmap, int head_dim,
                           cudaStream_t s, cudaEvent_t after_split);
