@@ -829,6 +829,16 @@ def time_device_steps(w, fmt, args, dev, stream, rank, local):
         cache.append_seq(b, t.k[b][None].contiguous(), t.v[b][None].contiguous(), w.seq_lens[b], zero, status,
                          stream)
     torch.cuda.synchronize()
+    r.prefill = None
+    if w.batch == 1 and fmt != "delegated" and rank == 0:
+        # the one-sequence prefill again (same data, same rows), device-timed with L2 flushed before
+        # each call: the append kernel on a long prompt
+        flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+        kp, vp = t.k[0][None].contiguous(), t.v[0][None].contiguous()
+        r.prefill = _time_graph_pairs(lambda s: cache.append_seq(0, kp, vp, w.seq_lens[0], zero, status, s),
+                                      flush, stream, n=3, reps=5)
+        del flush, kp, vp
+        torch.cuda.synchronize()
     lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
     lens1 = lens + w.n_append
     q = t.q.contiguous()
@@ -945,7 +955,9 @@ def roofline_record(r, fmt, paged, dev):
 
 
 def long_context_record(args, fmt, dev, stream, rank, local, ws):
-    """The 131072-token Llama-3.1-70B-shaped step (64 q / 8 kv heads), timed like the headline."""
+    """The 131072-token Llama-3.1-70B-shaped step (64 q / 8 kv heads), timed like the headline, and its
+    131072-token prefill (the append kernel on a long prompt)."""
+    import torch
     from compressed_domain_attention_b200 import synthetic as syn
     w = syn.llama31_70b_long()
     r = time_device_steps(w, fmt, args, dev, stream, rank, local)
@@ -963,6 +975,17 @@ def long_context_record(args, fmt, dev, stream, rank, local, ws):
            "l2": f"inputs larger than L2 (cache {r.cache.nbytes() / 1e9:.2f} GB > 126 MB), no flush"}
     if r.clocks:
         rec["clocks"] = r.clocks
+    if r.prefill is not None:
+        T = w.seq_lens[0]
+        pw = syn.Workload(w.name, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, [0], w.dtype, 0, n_append=T)
+        nb = append_bytes(pw, 2 if w.dtype != torch.float32 else 4, fmt)
+        ms = r.prefill["median"]
+        rec["prefill_quantize"] = {
+            "tokens": T, "vectors": 2 * T * w.n_kv_heads, "ms": ms, "timing": r.prefill,
+            "algorithmic_bytes": nb, "gb_per_s": round(nb / ms / 1e6, 1),
+            "frac_of_measured_hbm": round(nb / ms / 1e6 / peak, 4),
+            "kernel": "quantize_rows_kernel" if w.head_dim in (64, 128) else "quantize_append_kernel",
+            "l2": "flushed before each call"}
     return rec
 
 
