@@ -294,8 +294,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  __syncthreads();  // the barriers' initialisation is visible to every thread
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  block_prefix_lengths(p, prefix, prefix + (p.batch + 1));  // its barriers also publish the set-up
+  if (p.batch == 1) {
+    // one sequence: every thread takes its length itself and writes the same two prefix
+    // words (each thread reads back its own values), with no block barrier on the way
+    // to the first tile copies
+    int x = p.seq_lens[0];
+    if (x < 0 || x > p.max_seq) {
+      if (blockIdx.x == 0 && tid == 0) status_or(p.status, TQ_STATUS_CAPACITY);
+      x = 0;
+    }
+    int64_t L = cold_tokens(x, p.tail_window, p.fold_chunk);
+    L = (L + p.len_align - 1) & ~(int64_t)(p.len_align - 1);
+    prefix[0] = 0;
+    prefix[1] = L;
+  } else {
+    block_prefix_lengths(p, prefix, prefix + (p.batch + 1));
+  }
   const int64_t T_sum = prefix[p.batch];
   // T_sum < 2^32 (batch * max_seq <= INT32_MAX, plus at most a tile of padding per
   // sequence), so the split range takes a 32-bit division
