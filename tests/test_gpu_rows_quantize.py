@@ -8,7 +8,10 @@ dims, int4 and binary16 K, the per-channel lambda, special values (non-finite
 elements, all-zero vectors, vectors whose scale is a binary16 subnormal) and a
 two-sequence batch with different start positions; the status bits agree; rows
 outside the append stay untouched. The two kernels also agree with each other
-bit for bit on the same data.
+bit for bit on the same data. A sequence whose append would pass max_seq is
+skipped with TQ_STATUS_CAPACITY while the other is written; through a block table
+with an unmapped entry, that page's tokens are skipped and every other pool row
+equals the oracle's.
 """
 import numpy as np
 import pytest
@@ -106,3 +109,53 @@ def test_rows_and_group_kernels_agree(D):
     torch.cuda.synchronize()
     for x, y in zip(one.host_arrays(), two.host_arrays()):
         assert np.array_equal(x, y)
+
+
+def test_rows_kernel_capacity_skips_one_sequence():
+    # sequence 1 starts at 20: 20 + 4200 > 4210, so its vectors are skipped (status
+    # TQ_STATUS_CAPACITY) while sequence 0 is written exactly
+    D = 128
+    k, v = inputs(D, torch.bfloat16, 700)
+    gpu = GpuCache(B, CAP, HKV, HKV, D)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gpu.append_all(k.cuda(), v.cuda(), [0, 20], status)
+    orc = OracleCache(B, CAP, HKV, D)
+    st = oracle.quantize_append(orc.signs, np_f32(k), np_f32(v), np.array([0, 20], np.int32), orc.kc, orc.ks, orc.vc,
+                                orc.vs)
+    torch.cuda.synchronize()
+    assert int(status.item()) & tq.TQ_STATUS_CAPACITY and st & oracle.STATUS_CAPACITY
+    kc, ks, vc, vs = gpu.host_arrays()
+    assert np.array_equal(kc, orc.kc) and np.array_equal(ks, orc.ks)
+    assert np.array_equal(vc, orc.vc) and np.array_equal(vs, orc.vs)
+    assert not vc[1].any() and not kc[1].any(), "the skipped sequence was written"
+
+
+def test_rows_kernel_paged_with_an_unmapped_page():
+    # one sequence of 16 800 tokens x 2 kv heads (67 200 vectors) through a permuted block
+    # table of 256-token pages with one entry unmapped: that page's tokens are skipped
+    # (TQ_STATUS_CAPACITY), every other pool row equals the oracle's
+    D, H, n, P = 128, 2, 16800, 256
+    g = torch.Generator().manual_seed(800)
+    k = (torch.randn((1, n, H, D), generator=g) * 2).to(torch.bfloat16)
+    v = torch.randn((1, n, H, D), generator=g).to(torch.bfloat16)
+    max_pages = -(-n // P)
+    n_pages = max_pages + 3
+    L = tq.tq_cache_layout_paged(1, n, H, 4 * H, D, tq.TQ_K_INT4, P, n_pages)
+    rng = np.random.default_rng(5)
+    table = rng.permutation(n_pages)[:max_pages].reshape(1, max_pages).astype(np.int32)
+    table[0, 5] = -1
+    kc, ks, vc, vs = tq.alloc_cache(L)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_quantize_append_paged(L, k.cuda(), v.cuda(), n, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                                torch.from_numpy(table).cuda(), kc, ks, vc, vs, status)
+    signs = oracle.sign_vector(0, D)
+    pools = oracle.new_pool(n_pages, P, H, D, False)
+    st = oracle.quantize_append_paged(signs, np_f32(k), np_f32(v), np.zeros(1, np.int32), table, P, n, pools)
+    torch.cuda.synchronize()
+    assert int(status.item()) & tq.TQ_STATUS_CAPACITY and st & oracle.STATUS_CAPACITY
+    rows = n_pages * P
+    pk, pks, pv, pvs = pools
+    assert np.array_equal(kc.cpu().numpy().reshape(rows, H, D // 2), pk)
+    assert np.array_equal(ks[: rows * H * D // 32].cpu().numpy().view(np.uint16).reshape(rows, H, D // 32), pks)
+    assert np.array_equal(vc.cpu().numpy().reshape(rows, H, D // 2), pv)
+    assert np.array_equal(vs[: rows * H * D // 32].cpu().numpy().view(np.uint16).reshape(rows, H, D // 32), pvs)
