@@ -346,8 +346,8 @@ struct RowsCfg {
   static constexpr int ESZ = DT == TQ_F32 ? 4 : 2;    // input element bytes
   static constexpr int EPB = 128 / ESZ;               // elements per 128-byte box row
   static constexpr int NCOL = D / EPB;                // boxes per vector
-  static constexpr int TPV = rows_threads_per_vector(D);  // threads per vector (2 at head_dim 128)
-  static constexpr int EPT = D / TPV;                 // elements per thread (64)
+  static constexpr int TPV = rows_threads_per_vector(D);  // threads per vector (1; the code also runs 2)
+  static constexpr int EPT = D / TPV;                 // elements per thread
   static constexpr int BPT = EPT / EPB;               // boxes per thread
   static constexpr int NGT = EPT / 32;                // groups per thread
   static constexpr int VPW = 32 / TPV;                // vectors per warp
