@@ -228,6 +228,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// binary32 a / 7 rounded to nearest, by one product with RN(1/7) and one fused
+// correction (Markstein's method for division: q0 = RN(a y), r = a - 7 q0 exactly,
+// q1 = RN(q0 + r y)); checked equal to the IEEE division for every finite a >= 0 (a GPU test).
+__device__ __forceinline__ float div7_rn(float a) {
+  constexpr float y = 0.142857149f;  // RN(1/7)
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-7.0f, q0, a);
+  return __fmaf_rn(r, y, q0);
+}
+
+// Reciprocal with at most one unit in the last place of error (rcp.approx.f32).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // NG consecutive binary16 values at a shared-memory address aligned to 2 NG bytes
 // (NG in {1, 2, 4, 8}), widened to binary32 (exact).
 template <int NG>

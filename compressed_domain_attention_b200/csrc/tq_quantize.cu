@@ -488,23 +488,6 @@ __device__ __forceinline__ void fwht_row_from2(float (&u)[N]) {
   }
 }
 
-// binary32 a / 7 rounded to nearest, by one product with RN(1/7) and one fused
-// correction (Markstein's method for division: q0 = RN(a y), r = a - 7 q0 exactly,
-// q1 = RN(q0 + r y)); checked equal to the IEEE division for every finite a >= 0.
-__device__ __forceinline__ float div7_rn(float a) {
-  constexpr float y = 0.142857149f;  // RN(1/7)
-  const float q0 = __fmul_rn(a, y);
-  const float r = __fmaf_rn(-7.0f, q0, a);
-  return __fmaf_rn(r, y, q0);
-}
-
-// Reciprocal with at most one unit in the last place of error (rcp.approx.f32).
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
 // Fast encoding of one group (see encode_group for the definition and the exact path):
 // returns false, and leaves the group to encode_group, when a is not finite, the
 // binary16 scale is zero, subnormal or infinite, or some element lies within
