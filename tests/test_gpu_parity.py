@@ -164,6 +164,39 @@ def test_multi_sequence_per_cta():
     assert_close(out.cpu().numpy(), ref, what="straddling ranges")
 
 
+def test_maximum_batch():
+    # the largest batch the decode takes, 1024 sequences: block-wide prefix sums with
+    # several lengths per thread, default-grid ranges straddling many sequences, empty
+    # sequences among them; then one batched append of a token to every sequence
+    # (start = its length) and the decode over len + 1
+    rng = np.random.default_rng(21)
+    lens = [int(x) for x in rng.integers(0, 41, size=1024)]
+    lens[0] = lens[511] = 0
+    lens[1023] = 47
+    Hkv, G, D = 2, 2, 64
+    w, t, gpu, orc = random_case(1024, lens, Hkv, G, D, seed=21, cap=48)
+    out = gpu.decode(t.q.cuda(), lens, w.scale)
+    ref, _ = orc.decode(t.q, lens, w.scale)
+    got = out.cpu().numpy()
+    assert np.all(got[[0, 511]] == 0.0)
+    assert_close(got, ref, what="batch 1024")
+
+    g = torch.Generator().manual_seed(22)
+    k1 = torch.randn((1024, 1, Hkv, D), generator=g).to(torch.bfloat16)
+    v1 = torch.randn((1024, 1, Hkv, D), generator=g).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gpu.append_all(k1.cuda(), v1.cuda(), lens, status)
+    for b in range(1024):
+        orc.append_seq(b, k1[b], v1[b], lens[b])
+    lens1 = [L + 1 for L in lens]
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    compare_caches(gpu, orc, range(1024), lens1)
+    out1 = gpu.decode(t.q.cuda(), lens1, w.scale)
+    ref1, _ = orc.decode(t.q, lens1, w.scale)
+    assert_close(out1.cpu().numpy(), ref1, what="batch 1024 + append")
+
+
 @pytest.mark.parametrize("qdt", [torch.float32, torch.float16, torch.bfloat16])
 def test_query_dtypes(qdt):
     lens = [500, 1]
